@@ -1,0 +1,384 @@
+"""Benchmark: varlen causal MLA prefill on B200 through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one ``mla_prefill`` call (plan kernel + attention kernel) over the
+whole workload, inputs resident in HBM.  Prints ONE JSON line (rank 0).
+
+* value: algorithmic TFLOP/s = causally visible (query, key, head) triples x 640
+  FLOPs (2*192 for Q.K^T plus 2*128 for P.V) / device time per step, summed over
+  ranks (each rank runs an independent replica: "scaling": "weak").
+* roofline: the attention kernel alone (timed with CUDA events recorded by the
+  library around its launch) against the measured dense bf16 peak.
+* e2e: the same metric through the public call with pinned HOST inputs: every
+  step copies the inputs host->device, runs the call and copies attenOut back.
+* cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload.
+* --impl reference: the fp64 CPU oracle as the reference arm (rank 0 only).
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FLOPS_PER_TRIPLE = 640  # 2*(128+64) for the two-part Q.K^T, 2*128 for P.V
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def visible_triples(wl):
+    """Causally visible (query, key) pairs over all sequences, times the head count."""
+    n = 0
+    for lq, lk in zip(wl.q_seqlens, wl.kv_seqlens):
+        per_row = np.clip(np.arange(lq) + (lk - lq) + 1, 0, lk) if wl.causal else np.full(lq, lk)
+        n += int(per_row.sum())
+    return n * wl.head_num
+
+
+def algorithmic_bytes(wl):
+    """Read Q, Q_rope, K, K_rope, V once and write O once (16-bit elements)."""
+    return 2 * (wl.t_q * wl.head_num * (wl.d_nope + wl.d_rope) + wl.t_k * wl.kv_head_num * (
+        wl.d_nope + wl.d_rope + wl.d_nope) + wl.t_q * wl.head_num * wl.d_nope)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_oracle_sample(wl, x_cpu, target_s, seed=0):
+    """Runs the CPU oracle on seeded sample rows (every head) for about target_s seconds.
+
+    Returns (seconds, triples_computed, description)."""
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    starts = np.concatenate([[0], np.cumsum(wl.q_seqlens)])
+
+    def rows_triples(rows):
+        tot = 0
+        for t in rows:
+            b = int(np.searchsorted(starts, t, side="right") - 1)
+            lq, lk = wl.q_seqlens[b], wl.kv_seqlens[b]
+            i = t - starts[b]
+            tot += int(min(lk, max(0, i + lk - lq + 1))) if wl.causal else lk
+        return tot * wl.head_num
+
+    def run(rows):
+        t0 = time.perf_counter()
+        oracle.prefill(x_cpu["q"], x_cpu["q_rope"], x_cpu["k"], x_cpu["k_rope"], x_cpu["v"], x_cpu["q_seqlen"],
+                       x_cpu["kv_seqlen"], wl.head_num, wl.kv_head_num, wl.qk_scale, rows=rows)
+        return time.perf_counter() - t0
+
+    rows = np.sort(rng.choice(wl.t_q, size=min(4, wl.t_q), replace=False))
+    dt = run(rows)
+    rate = rows_triples(rows) / max(dt, 1e-6)  # triples per second
+    want_triples = rate * target_s
+    avg = max(1.0, rows_triples(np.arange(wl.t_q)) / wl.t_q)
+    n = int(min(wl.t_q, max(4, want_triples / avg)))
+    rows = np.sort(rng.choice(wl.t_q, size=n, replace=False))
+    dt = run(rows)
+    trip = rows_triples(rows)
+    desc = "%d seeded query rows x %d heads of workload %s (%d visible triples)" % (n, wl.head_num, wl.name, trip)
+    return dt, trip, desc
+
+
+def to_numpy_f64(x):
+    return {k: (v.double().numpy() if v.is_floating_point() else v.numpy()) for k, v in x.items()}
+
+
+def reference_arm(args, wl):
+    """The fp64 CPU oracle timed as the reference implementation (rank 0 only)."""
+    import torch
+
+    from mla_prefill_attention_varlen_b200 import workloads as W
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = to_numpy_f64(W.make_inputs(wl, device="cpu"))
+    import oracle
+
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        time_oracle_sample(wl, x, min(per_step, 2.0), seed=1)
+    times, trips, desc = [], [], ""
+    for k in range(args.steps):
+        dt, tr, desc = time_oracle_sample(wl, x, per_step, seed=10 + k)
+        times.append(dt)
+        trips.append(tr)
+    tflops = sum(trips) * FLOPS_PER_TRIPLE / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": "causal MLA prefill TFLOP/s (visible pairs x 640 FLOPs)",
+        "value": tflops, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "sampled": True},
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": oracle.core_count(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from mla_prefill_attention_varlen_b200 import workloads as W
+
+    wl = W.get(args.workload)
+    if args.impl == "reference":
+        return reference_arm(args, wl)
+
+    import torch
+
+    import mla_prefill_attention_varlen_b200 as mla
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    mla.load_library()
+    x = W.make_inputs(wl, device=dev)
+    out = torch.empty(wl.t_q, wl.head_num, wl.d_nope, dtype=wl.dtype, device=dev)
+    H, G, scale = wl.head_num, wl.kv_head_num, wl.qk_scale
+    stream = torch.cuda.current_stream()
+
+    def step(o=out):
+        mla.mla_prefill(x["q"], x["q_rope"], x["k"], x["k_rope"], x["v"], x["q_seqlen"], x["kv_seqlen"],
+                        mla.MLA_MASK_CAUSAL, H, G, scale, o, stream)
+
+    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+    flush = None
+    if in_bytes < 2 * L2_BYTES:
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = mla.mla_prefill_device_status()
+    if st != 0:
+        raise RuntimeError("device status after warm-up: %s" % mla.mla_status_string(st))
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    smi = ClockSampler(local if world > 1 else torch.cuda.current_device())
+    torch.cuda.synchronize()
+    barrier(world)
+    with smi:
+        time.sleep(0.3)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            mla.set_profile_events(k_starts[i], k_stops[i])
+            starts[i].record(stream)
+            step()
+            stops[i].record(stream)
+        mla.set_profile_events(None, None)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    kern_ms = [a.elapsed_time(b) for a, b in zip(k_starts, k_stops)]
+    ms = max_over_ranks(float(np.mean(step_ms)), world)
+    kms = max_over_ranks(float(np.mean(kern_ms)), world)
+    st = mla.mla_prefill_device_status()
+    if st != 0:
+        raise RuntimeError("device status after timing: %s" % mla.mla_status_string(st))
+
+    triples = visible_triples(wl)
+    flops = triples * FLOPS_PER_TRIPLE
+    value = world * flops / (ms * 1e-3) / 1e12
+    tokens_per_s = world * wl.t_q / (ms * 1e-3)
+    peaks, peak_src = load_peaks()
+    kern_tflops = flops / (kms * 1e-3) / 1e12
+
+    # end to end through the public call: pinned host inputs in, attenOut back to the host
+    e2e = None
+    if not args.no_e2e:
+        hx = {k: v.cpu().pin_memory() for k, v in x.items()}
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dx = {k: torch.empty_like(v) for k, v in x.items()}
+        h2d = sum(t.numel() * t.element_size() for t in hx.values())
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for k in dx:
+                dx[k].copy_(hx[k], non_blocking=True)
+            mla.mla_prefill(dx["q"], dx["q_rope"], dx["k"], dx["k_rope"], dx["v"], dx["q_seqlen"], dx["kv_seqlen"],
+                            mla.MLA_MASK_CAUSAL, H, G, scale, out, stream)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e_start = torch.cuda.Event(enable_timing=True)
+        e_stop = torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e_start.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e_stop.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(e_start.elapsed_time(e_stop) / n_e2e, world)
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        xc = to_numpy_f64({k: v.cpu() for k, v in x.items()})
+        dt, trip, desc = time_oracle_sample(wl, xc, args.cpu_seconds)
+        cpu_baseline = {"value": trip * FLOPS_PER_TRIPLE / dt / 1e12, "unit": "TFLOP/s",
+                        "cores": oracle.core_count(), "kind": "oracle", "sample": desc}
+
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    clocks = smi.summary()
+    line = {
+        "metric": "causal MLA prefill TFLOP/s (visible pairs x 640 FLOPs), % of B200 dense bf16 peak, tokens/s",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f16", "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "batch": wl.batch, "t_q": wl.t_q,
+                   "t_k": wl.t_k, "head_num": H, "kv_head_num": G, "qk_scale": scale, "mask": "causal",
+                   "parallelism": "replicas" if world > 1 else "single", "l2": (
+                       "flushed between steps (512 MB write)" if flush is not None else
+                       "inputs %.2f GB > 126 MB L2" % (in_bytes / 1e9)),
+                   "visible_triples": triples},
+        "pct_of_peak": 100.0 * value / world / peak,
+        "tokens_per_s": tokens_per_s,
+        "north_star_literal_tflops": 2 * value,
+        "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": kern_tflops / peak, "traffic": None, "peak_source": peak_src,
+                     "peak_kind": "burst", "frac_of_sustained": kern_tflops / peak_sus,
+                     "kernel": "mla_prefill_sm100_kernel", "kernel_ms": kms,
+                     "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": algorithmic_bytes(wl)},
+        "cpu_baseline": cpu_baseline,
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,149 @@
+/*
+ * mla_prefill.h -- C ABI of the B200 (sm_100a) varlen MLA prefill library
+ * (libmla_prefill.so).
+ *
+ * The operation is the one the "MLA Prefill" page of the Ascend Transformer
+ * Boost C API defines through AtbMLAPreFillGetWorkspaceSize / AtbMLAPreFill
+ * ("Definition" section and the members table): attention of packed,
+ * variable-length queries over packed keys and values, where the query-key
+ * product has two parts -- the "nope" channels of Q and K (embeddimV = 128
+ * wide) and the rotary channels of QRope and kRope (64 wide) -- both summed
+ * into one score, scaled by qkScale (the "scaling coefficient post-multiplied
+ * by Q*K^T"), masked causally (MASK_TYPE_CAUSAL_MASK in the Mask row), turned
+ * into weights by a row softmax, and applied to V.  For sequence b, query
+ * head h, kv head kh = h / (head_num / kv_head_num), query row i < Lq_b and
+ * key j < Lk_b (Lq_b = q_seqlen[b], Lk_b = kv_seqlen[b]):
+ *
+ *   s_ij = qk_scale * (Q[i,h,:128] . K[j,kh,:128] + QR[i,h,:64] . KR[j,kh,:64])
+ *   causal: key j is visible to row i iff j <= i + (Lk_b - Lq_b)
+ *           (the mask is aligned to the bottom-right corner, so a chunk of Lq
+ *           new queries sees the whole cached prefix of Lk - Lq keys)
+ *   out[i,h,:] = sum_j softmax_j(s_ij) * V[j,kh,:128]     (0 if no key visible)
+ *
+ * Differences from the page's two-phase API: the workspace query and the
+ * operation object are folded into one asynchronous call on a CUDA stream;
+ * calcType is fixed to prefill, cacheMode to 0, and the Mask tensor is not
+ * taken (the causal mask is computed from indices).
+ */
+#ifndef MLA_PREFILL_H
+#define MLA_PREFILL_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream; the same type as cudaStream_t / CUstream. */
+struct CUstream_st;
+typedef struct CUstream_st *mla_stream_t;
+
+/* Element types (the page's float16 / bf16 data types, int32 seqlens). */
+typedef enum { MLA_F16 = 0, MLA_BF16 = 1, MLA_I32 = 2 } mla_dtype;
+
+/*
+ * A strided view of device memory, in the spirit of the page's aclTensor.
+ * data: device pointer (caller-owned).  dtype: an mla_dtype value.
+ * ndim: 1..4.  shape[d], stride[d]: extents and strides in ELEMENTS for
+ * d < ndim; entries past ndim are ignored.
+ */
+typedef struct {
+    void *data;
+    int32_t dtype;
+    int32_t ndim;
+    int64_t shape[4];
+    int64_t stride[4];
+} mla_tensor;
+
+/* maskType: the page's UNDEFINED (all-zero mask: nothing hidden) and
+ * MASK_TYPE_CAUSAL_MASK (bottom-right aligned causal mask). */
+typedef enum { MLA_MASK_NONE = 0, MLA_MASK_CAUSAL = 1 } mla_mask_type;
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_NULL = 1,          /* a required pointer is NULL */
+    MLA_ERR_DTYPE = 2,         /* dtype mismatch or unsupported dtype */
+    MLA_ERR_SHAPE = 3,         /* shapes inconsistent with each other / the head counts */
+    MLA_ERR_ALIGN = 4,         /* base pointer not 16-byte aligned, or a stride not a multiple of 8 elements */
+    MLA_ERR_HEADS = 5,         /* head_num < 1, kv_head_num < 1, or head_num % kv_head_num != 0 */
+    MLA_ERR_UNSUPPORTED = 6,   /* unsupported mask type, layout or argument value */
+    MLA_ERR_CUDA = 7,          /* a CUDA runtime/driver call failed */
+    MLA_ERR_SEQLEN = 8,        /* device-detected: a negative seqlen, or sum(seqlen) above the tensor extent */
+    MLA_ERR_DEVICE_TIMEOUT = 9 /* device-detected: a pipeline wait gave up (never expected) */
+} mla_status;
+
+/*
+ * mla_prefill -- varlen MLA prefill attention, asynchronous on `stream`.
+ *
+ * Inputs (all device memory, read only, one dtype: MLA_BF16 or MLA_F16):
+ *   q       [T_q, H, 128] or [T_q, H*128]   Q "nope" part        (page: Q row)
+ *   q_rope  [T_q, H, 64]  or [T_q, H*64]    Q rotary part        (page: QRope row)
+ *   k       [T_k, G, 128] or [T_k, G*128]   K "nope" part        (page: K row, packed form)
+ *   k_rope  [T_k, G, 64]  or [T_k, G*64]    K rotary part, per kv head (page: kRope row)
+ *   v       [T_k, G, 128] or [T_k, G*128]   values               (page: V row, packed form)
+ *   q_seqlen, kv_seqlen  [batch] MLA_I32 in DEVICE memory (page: qSeqLen / kvSeqLen rows).
+ *     Sequence b owns query tokens [sum_{b'<b} Lq_b', + Lq_b) and key tokens
+ *     [sum_{b'<b} Lk_b', + Lk_b) of the packed tensors.
+ *   mask_type   MLA_MASK_CAUSAL or MLA_MASK_NONE.
+ *   head_num    H >= 1 (page: headNum); kv_head_num G >= 1 with H % G == 0 (page: kvHeadNum).
+ *               Query head h reads kv head h / (H / G).
+ *   qk_scale    any finite float (page: qkScale), multiplied onto the full two-part product.
+ * Output:
+ *   out     [T_q, H, 128] or [T_q, H*128], same dtype as the inputs (page: attenOut row).
+ *           Rows of tokens past sum(q_seqlen) are not written.  A row with no
+ *           visible key (possible when Lq_b > Lk_b) is written as zeros.
+ *
+ * Layout rules: the last dimension is contiguous (stride 1); token and head
+ * strides are positive multiples of 8 elements (so q_rope / k_rope may be views
+ * into wider buffers); every base pointer is 16-byte aligned.  The padded
+ * [batch, max_seq, G*128] K/V form of the page is rejected with
+ * MLA_ERR_UNSUPPORTED.  `out` must not overlap any input.
+ *
+ * Ownership and errors: the caller owns every buffer.  Argument errors are
+ * detected on the host and returned before anything is launched; `out` is then
+ * untouched.  The call enqueues work on `stream` and returns without waiting.
+ * The library keeps one device workspace per GPU (created on the first call on
+ * that GPU, grown when a call needs more; a call that grows it allocates
+ * device memory).  Calls that share a GPU must be ordered on one stream, or
+ * otherwise serialised, because they share that workspace.
+ * Inconsistent seqlens (negative, or summing past T_q / T_k) are detected on
+ * the device: the kernel clamps to the tensor extents -- it never reads or
+ * writes out of bounds -- and records MLA_ERR_SEQLEN in a sticky status word
+ * that mla_prefill_device_status() returns.
+ * Returns MLA_OK or an mla_status error code.
+ */
+int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+                const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+                int head_num, int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream);
+
+/*
+ * mla_prefill_device_status -- synchronises `stream`, then reads and clears the
+ * device status word of the current GPU (MLA_OK, MLA_ERR_SEQLEN or
+ * MLA_ERR_DEVICE_TIMEOUT; the first error recorded since the last read).
+ * Writes it to *status and returns MLA_OK, or returns MLA_ERR_NULL /
+ * MLA_ERR_CUDA.
+ */
+int mla_prefill_device_status(mla_stream_t stream, int *status);
+
+/* A static, human-readable name for a status code (never NULL). */
+const char *mla_status_string(int status);
+
+/*
+ * mla_prefill_set_profile_events -- profiling hook.  When both events are
+ * non-NULL, every later mla_prefill call on this host thread records `start`
+ * on its stream immediately before the attention kernel launch and `stop`
+ * immediately after it, so the caller can time that kernel alone with
+ * cudaEventElapsedTime.  The events are CUDA events (cudaEvent_t) owned by
+ * the caller.  Passing NULL, NULL turns the hook off.  Returns MLA_OK.
+ */
+struct CUevent_st;
+int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *stop);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int mla_prefill_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_PREFILL_H */

@@ -1,0 +1,155 @@
+"""B200 (sm_100a) varlen causal MLA prefill.
+
+Python binding of ``libmla_prefill.so`` (C ABI in ``include/mla_prefill.h``).
+This module only marshals torch tensors into ``mla_tensor`` descriptors and
+forwards them; every step of the computation runs in the library's CUDA
+kernels.  There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+import ctypes
+import os
+
+from . import workloads  # noqa: F401  (seeded synthetic inputs)
+
+__all__ = [
+    "MLA_MASK_NONE", "MLA_MASK_CAUSAL", "MlaError", "load_library", "mla_prefill", "mla_prefill_device_status",
+    "mla_status_string", "prefill", "workloads",
+]
+
+MLA_F16, MLA_BF16, MLA_I32 = 0, 1, 2
+MLA_MASK_NONE, MLA_MASK_CAUSAL = 0, 1
+STATUS_NAMES = {
+    0: "MLA_OK", 1: "MLA_ERR_NULL", 2: "MLA_ERR_DTYPE", 3: "MLA_ERR_SHAPE", 4: "MLA_ERR_ALIGN",
+    5: "MLA_ERR_HEADS", 6: "MLA_ERR_UNSUPPORTED", 7: "MLA_ERR_CUDA", 8: "MLA_ERR_SEQLEN",
+    9: "MLA_ERR_DEVICE_TIMEOUT",
+}
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmla_prefill.so")
+
+
+class MlaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+class MlaError(RuntimeError):
+    def __init__(self, code, where="mla_prefill"):
+        self.code = int(code)
+        super().__init__("%s failed: %s (%d)" % (where, mla_status_string(code), self.code))
+
+
+_lib = None
+
+
+def load_library(path=None):
+    """Load (once) and return the ctypes handle of libmla_prefill.so."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError("libmla_prefill.so not built (run `python -m mla_prefill_attention_varlen_b200.build`)")
+    lib = ctypes.CDLL(p)
+    T = ctypes.POINTER(MlaTensor)
+    lib.mla_prefill.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, T,
+                                ctypes.c_void_p]
+    lib.mla_prefill.restype = ctypes.c_int
+    lib.mla_prefill_device_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]
+    lib.mla_prefill_device_status.restype = ctypes.c_int
+    lib.mla_status_string.argtypes = [ctypes.c_int]
+    lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_prefill_set_profile_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    lib.mla_prefill_set_profile_events.restype = ctypes.c_int
+    lib.mla_prefill_version.argtypes = []
+    lib.mla_prefill_version.restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def mla_status_string(code):
+    try:
+        return load_library().mla_status_string(int(code)).decode()
+    except ImportError:
+        return STATUS_NAMES.get(int(code), "unknown")
+
+
+def _dtype_code(t):
+    import torch
+
+    return {torch.float16: MLA_F16, torch.bfloat16: MLA_BF16, torch.int32: MLA_I32}.get(t.dtype, -1)
+
+
+def as_mla_tensor(t):
+    """Describe a torch tensor (any device) as an mla_tensor; no copy."""
+    d = MlaTensor()
+    d.data = t.data_ptr() if t.numel() > 0 or t.data_ptr() else None
+    d.dtype = _dtype_code(t)
+    d.ndim = t.dim()
+    if d.ndim > 4:
+        raise ValueError("at most 4 dimensions")
+    for i in range(d.ndim):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _stream_handle(stream, device):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def mla_prefill(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
+                stream=None):
+    """Call the C ABI ``mla_prefill`` on torch tensors (same argument order).
+
+    All tensors must live on the current CUDA device; ``out`` is written in
+    place.  ``stream``: a torch.cuda.Stream, a raw handle, or None for the
+    current stream.  Raises MlaError on any non-zero status.
+    """
+    lib = load_library()
+    descs = [as_mla_tensor(t) for t in (q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, out)]
+    rc = lib.mla_prefill(*(ctypes.byref(d) for d in descs[:7]), int(mask_type), int(head_num), int(kv_head_num),
+                         float(qk_scale), ctypes.byref(descs[7]), _stream_handle(stream, q.device))
+    if rc != 0:
+        raise MlaError(rc)
+    return out
+
+
+def prefill(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, head_num, kv_head_num, qk_scale,
+            mask_type=MLA_MASK_CAUSAL, out=None, stream=None):
+    """Allocate ``out`` [T_q, H, 128] (if not given) and run ``mla_prefill``."""
+    import torch
+
+    if out is None:
+        out = torch.empty(q.shape[0], head_num, v.shape[-1] if v.dim() == 3 else 128, dtype=q.dtype,
+                          device=q.device)
+    return mla_prefill(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale,
+                       out, stream)
+
+
+def set_profile_events(start=None, stop=None):
+    """Record torch.cuda.Events around the attention-kernel launch of later calls."""
+    lib = load_library()
+    if start is None or stop is None:
+        lib.mla_prefill_set_profile_events(None, None)
+    else:
+        lib.mla_prefill_set_profile_events(start.cuda_event, stop.cuda_event)
+
+
+def mla_prefill_device_status(stream=None):
+    """Synchronise the stream and return (and clear) the device status word."""
+    import torch
+
+    lib = load_library()
+    st = ctypes.c_int(0)
+    rc = lib.mla_prefill_device_status(_stream_handle(stream, torch.cuda.current_device()), ctypes.byref(st))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_device_status")
+    return st.value

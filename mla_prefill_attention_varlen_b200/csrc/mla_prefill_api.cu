@@ -1,0 +1,345 @@
+// Host side of libmla_prefill.so: argument validation, the per-GPU workspace,
+// TMA tensor-map encoding and the two launches (plan kernel, attention kernel)
+// behind the C ABI declared in include/mla_prefill.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mla_prefill.h"
+#include "mla_prefill_sm100.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kVersion = 10000 * 0 + 100 * 1 + 0;
+
+struct DeviceState {
+    bool ready = false;
+    int sm_count = 0;
+    int *status = nullptr;  // sticky device status word (own 256-byte allocation)
+    void *ws = nullptr;     // plan workspace
+    size_t ws_bytes = 0;
+    bool attr_set[8] = {};  // dynamic shared memory opt-in done, per kernel instantiation
+};
+
+std::mutex g_mu;
+thread_local cudaEvent_t t_prof_start = nullptr, t_prof_stop = nullptr;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Views of one input after validation, as [tokens, heads, width] with element strides.
+struct View3 {
+    void *data;
+    int64_t tokens, heads, width;
+    int64_t st_tok, st_head;
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Accepts [T, N, W] or [T, N*W]; the last dimension must be contiguous.
+int view3(const mla_tensor *t, int dtype, int64_t heads, int64_t width, View3 *v) {
+    if (!t) return MLA_ERR_NULL;
+    if (!t->data && !(t->ndim >= 1 && t->ndim <= 4 && t->shape[0] == 0)) return MLA_ERR_NULL;
+    if (t->dtype != dtype) return MLA_ERR_DTYPE;
+    if (t->ndim == 3) {
+        if (t->shape[1] != heads || t->shape[2] != width) return MLA_ERR_SHAPE;
+        if (t->stride[2] != 1) return MLA_ERR_ALIGN;
+        v->tokens = t->shape[0];
+        v->st_tok = t->stride[0];
+        v->st_head = t->stride[1];
+    } else if (t->ndim == 2) {
+        if (t->shape[1] != heads * width) return MLA_ERR_SHAPE;
+        if (t->stride[1] != 1) return MLA_ERR_ALIGN;
+        v->tokens = t->shape[0];
+        v->st_tok = t->stride[0];
+        v->st_head = width;
+    } else {
+        return MLA_ERR_SHAPE;
+    }
+    v->data = t->data;
+    v->heads = heads;
+    v->width = width;
+    if (v->tokens < 0 || v->tokens > INT32_MAX) return MLA_ERR_SHAPE;
+    if (v->data && !aligned16(v->data)) return MLA_ERR_ALIGN;
+    if (v->tokens > 1 && (v->st_tok <= 0 || v->st_tok % 8 != 0)) return MLA_ERR_ALIGN;
+    if (heads > 1 && (v->st_head <= 0 || v->st_head % 8 != 0)) return MLA_ERR_ALIGN;
+    if (v->st_tok % 8 != 0 || v->st_head % 8 != 0) return MLA_ERR_ALIGN;
+    if (v->st_tok * 2 >= (int64_t(1) << 40) || v->st_head * 2 >= (int64_t(1) << 40)) return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+// The padded [batch, max_seq, G*128] K/V form: 3-D with a last dim of G*W (G > 1),
+// or with a middle extent other than G when G == 1.
+bool is_padded_kv(const mla_tensor *t, int64_t heads, int64_t width) {
+    return t && t->ndim == 3 && t->shape[2] == heads * width && !(t->shape[1] == heads && t->shape[2] == width);
+}
+
+// [lo, hi) byte range a view touches (for the no-alias check).
+void byte_range(const View3 &v, uintptr_t *lo, uintptr_t *hi) {
+    const uintptr_t base = reinterpret_cast<uintptr_t>(v.data);
+    int64_t last = 0;
+    if (v.tokens > 0) last = (v.tokens - 1) * v.st_tok + (v.heads - 1) * v.st_head + v.width;
+    *lo = base;
+    *hi = base + static_cast<uintptr_t>(last) * 2;
+}
+
+bool overlaps(const View3 &a, const View3 &b) {
+    uintptr_t alo, ahi, blo, bhi;
+    byte_range(a, &alo, &ahi);
+    byte_range(b, &blo, &bhi);
+    return alo < bhi && blo < ahi && ahi > alo && bhi > blo;
+}
+
+int ensure_encode() {
+    if (g_encode) return MLA_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return MLA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return MLA_OK;
+}
+
+// 3-D map {width, heads, tokens} with a {64, 1, 128} box and 128-byte swizzle.
+int encode_map(CUtensorMap *m, const View3 &v, bool bf16, void *dummy) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(v.width), static_cast<cuuint64_t>(v.heads),
+                                static_cast<cuuint64_t>(v.tokens > 0 ? v.tokens : 1)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>((v.heads > 1 ? v.st_head : v.width) * 2),
+                                   static_cast<cuuint64_t>((v.tokens > 1 ? v.st_tok : v.heads * v.width) * 2)};
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    // An empty tensor is never read (no work item touches it); encode a valid dummy base.
+    void *base = (v.tokens > 0 && v.data) ? v.data : dummy;
+    CUresult r = g_encode(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base,
+                          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_UNSUPPORTED;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+    size_t seq_info, tile_off, hist, tiles, num_tiles, total;
+    int hist_len;
+};
+
+WsLayout ws_layout(int64_t batch, int64_t t_q, int64_t t_k) {
+    WsLayout l;
+    const int64_t max_tiles = (t_q + mla::kBM - 1) / mla::kBM + batch;
+    l.hist_len = static_cast<int>((t_k + mla::kBN - 1) / mla::kBN + 2);
+    size_t off = 0;
+    l.num_tiles = off;
+    off = align_up(off + 16, 256);
+    l.seq_info = off;
+    off = align_up(off + sizeof(int4) * batch, 256);
+    l.tile_off = off;
+    off = align_up(off + sizeof(int) * (batch + 1), 256);
+    l.hist = off;
+    off = align_up(off + sizeof(int) * l.hist_len, 256);
+    l.tiles = off;
+    off = align_up(off + sizeof(int2) * max_tiles, 256);
+    l.total = off;
+    return l;
+}
+
+int device_state(int dev, cudaStream_t stream, size_t ws_need, DeviceState **out) {
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;  // built for sm_100a only
+        if (cudaMalloc(&d.status, 256) != cudaSuccess) return MLA_ERR_CUDA;
+        if (cudaMemset(d.status, 0, 256) != cudaSuccess) return MLA_ERR_CUDA;
+        d.ready = true;
+    }
+    if (d.ws_bytes < ws_need) {
+        if (d.ws) {
+            if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;
+            cudaFree(d.ws);
+            d.ws = nullptr;
+            d.ws_bytes = 0;
+        }
+        const size_t bytes = align_up(ws_need * 2 > (1u << 20) ? ws_need * 2 : (1u << 20), 4096);
+        if (cudaMalloc(&d.ws, bytes) != cudaSuccess) return MLA_ERR_CUDA;
+        d.ws_bytes = bytes;
+    }
+    *out = &d;
+    return MLA_OK;
+}
+
+template <typename T, bool kCausal, bool kPos>
+int launch_attention(DeviceState *ds, int slot, int grid, cudaStream_t stream, const CUtensorMap (&maps)[5],
+                     const mla::Params &p) {
+    auto kern = mla::mla_prefill_sm100_kernel<T, kCausal, kPos>;
+    if (!ds->attr_set[slot]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kSmemAlloc) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        ds->attr_set[slot] = true;
+    }
+    if (t_prof_start && cudaEventRecord(t_prof_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
+    kern<<<grid, mla::kThreads, mla::kSmemAlloc, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if (t_prof_stop && cudaEventRecord(t_prof_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+                const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+                int head_num, int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!q || !q_rope || !k || !k_rope || !v || !q_seqlen || !kv_seqlen || !out) return MLA_ERR_NULL;
+    if (head_num < 1 || kv_head_num < 1 || head_num % kv_head_num != 0) return MLA_ERR_HEADS;
+    if (mask_type != MLA_MASK_CAUSAL && mask_type != MLA_MASK_NONE) return MLA_ERR_UNSUPPORTED;
+    if (!std::isfinite(qk_scale)) return MLA_ERR_UNSUPPORTED;
+    const int dt = q->dtype;
+    if (dt != MLA_BF16 && dt != MLA_F16) return MLA_ERR_DTYPE;
+    if (is_padded_kv(k, kv_head_num, mla::kDn) || is_padded_kv(v, kv_head_num, mla::kDn) ||
+        is_padded_kv(k_rope, kv_head_num, mla::kDr))
+        return MLA_ERR_UNSUPPORTED;
+
+    View3 vq, vqr, vk, vkr, vv, vo;
+    int rc;
+    if ((rc = view3(q, dt, head_num, mla::kDn, &vq)) != MLA_OK) return rc;
+    if ((rc = view3(q_rope, dt, head_num, mla::kDr, &vqr)) != MLA_OK) return rc;
+    if ((rc = view3(k, dt, kv_head_num, mla::kDn, &vk)) != MLA_OK) return rc;
+    if ((rc = view3(k_rope, dt, kv_head_num, mla::kDr, &vkr)) != MLA_OK) return rc;
+    if ((rc = view3(v, dt, kv_head_num, mla::kDn, &vv)) != MLA_OK) return rc;
+    if ((rc = view3(out, dt, head_num, mla::kDn, &vo)) != MLA_OK) return rc;
+    if (vqr.tokens != vq.tokens || vo.tokens != vq.tokens || vkr.tokens != vk.tokens || vv.tokens != vk.tokens)
+        return MLA_ERR_SHAPE;
+
+    if (q_seqlen->dtype != MLA_I32 || kv_seqlen->dtype != MLA_I32) return MLA_ERR_DTYPE;
+    if (q_seqlen->ndim != 1 || kv_seqlen->ndim != 1 || q_seqlen->shape[0] != kv_seqlen->shape[0])
+        return MLA_ERR_SHAPE;
+    if (q_seqlen->shape[0] > 0 && (!q_seqlen->data || !kv_seqlen->data)) return MLA_ERR_NULL;
+    if (q_seqlen->shape[0] > 1 && (q_seqlen->stride[0] != 1 || kv_seqlen->stride[0] != 1)) return MLA_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(q_seqlen->data) & 3u) || (reinterpret_cast<uintptr_t>(kv_seqlen->data) & 3u))
+        return MLA_ERR_ALIGN;
+    const int64_t batch = q_seqlen->shape[0];
+    if (batch < 0 || batch > INT32_MAX / 2) return MLA_ERR_SHAPE;
+
+    for (const View3 *in : {&vq, &vqr, &vk, &vkr, &vv})
+        if (overlaps(vo, *in)) return MLA_ERR_UNSUPPORTED;
+
+    if (batch == 0 || vq.tokens == 0) return MLA_OK;  // nothing to compute
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const WsLayout lay = ws_layout(batch, vq.tokens, vk.tokens);
+    DeviceState *ds = nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((rc = device_state(dev, stream, lay.total, &ds)) != MLA_OK) return rc;
+    if ((rc = ensure_encode()) != MLA_OK) return rc;
+
+    const bool bf16 = dt == MLA_BF16;
+    CUtensorMap maps[5];
+    if ((rc = encode_map(&maps[0], vq, bf16, ds->ws)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[1], vqr, bf16, ds->ws)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[2], vk, bf16, ds->ws)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[3], vkr, bf16, ds->ws)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[4], vv, bf16, ds->ws)) != MLA_OK) return rc;
+
+    uint8_t *ws = static_cast<uint8_t *>(ds->ws);
+    int *num_tiles = reinterpret_cast<int *>(ws + lay.num_tiles);
+    int4 *seq_info = reinterpret_cast<int4 *>(ws + lay.seq_info);
+    int *tile_off = reinterpret_cast<int *>(ws + lay.tile_off);
+    int *hist = reinterpret_cast<int *>(ws + lay.hist);
+    int2 *tiles = reinterpret_cast<int2 *>(ws + lay.tiles);
+    const bool causal = mask_type == MLA_MASK_CAUSAL;
+
+    mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
+        static_cast<const int *>(q_seqlen->data), static_cast<const int *>(kv_seqlen->data), static_cast<int>(batch),
+        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, tile_off, hist, lay.hist_len, tiles, num_tiles, ds->status);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+
+    mla::Params p;
+    p.seq_info = seq_info;
+    p.tiles = tiles;
+    p.num_tiles = num_tiles;
+    p.status = ds->status;
+    p.out = vo.data;
+    p.out_st = vo.st_tok;
+    p.out_sh = vo.st_head;
+    p.head_num = head_num;
+    p.group = head_num / kv_head_num;
+    p.scale_log2 = qk_scale * 1.4426950408889634f;
+
+    const int64_t max_items = ((vq.tokens + mla::kBM - 1) / mla::kBM + batch) * head_num;
+    const int grid = static_cast<int>(max_items < ds->sm_count ? max_items : ds->sm_count);
+    const bool pos = qk_scale > 0.f;
+    if (bf16) {
+        if (causal)
+            return pos ? launch_attention<__nv_bfloat16, true, true>(ds, 0, grid, stream, maps, p)
+                       : launch_attention<__nv_bfloat16, true, false>(ds, 1, grid, stream, maps, p);
+        return pos ? launch_attention<__nv_bfloat16, false, true>(ds, 2, grid, stream, maps, p)
+                   : launch_attention<__nv_bfloat16, false, false>(ds, 3, grid, stream, maps, p);
+    }
+    if (causal)
+        return pos ? launch_attention<__half, true, true>(ds, 4, grid, stream, maps, p)
+                   : launch_attention<__half, true, false>(ds, 5, grid, stream, maps, p);
+    return pos ? launch_attention<__half, false, true>(ds, 6, grid, stream, maps, p)
+               : launch_attention<__half, false, false>(ds, 7, grid, stream, maps, p);
+}
+
+int mla_prefill_device_status(mla_stream_t stream_, int *status) {
+    if (!status) return MLA_ERR_NULL;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        *status = MLA_OK;
+        return MLA_OK;
+    }
+    int h = 0;
+    if (cudaMemcpy(&h, d.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+    *status = h;
+    return MLA_OK;
+}
+
+const char *mla_status_string(int status) {
+    switch (status) {
+        case MLA_OK: return "MLA_OK";
+        case MLA_ERR_NULL: return "MLA_ERR_NULL: a required pointer is NULL";
+        case MLA_ERR_DTYPE: return "MLA_ERR_DTYPE: unsupported or mismatched dtype";
+        case MLA_ERR_SHAPE: return "MLA_ERR_SHAPE: inconsistent shapes";
+        case MLA_ERR_ALIGN: return "MLA_ERR_ALIGN: misaligned pointer or stride";
+        case MLA_ERR_HEADS: return "MLA_ERR_HEADS: invalid head_num / kv_head_num";
+        case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: unsupported argument, layout or device";
+        case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA call failed";
+        case MLA_ERR_SEQLEN: return "MLA_ERR_SEQLEN: seqlens inconsistent with tensor extents (clamped)";
+        case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT: a device pipeline wait gave up";
+        default: return "unknown mla_status";
+    }
+}
+
+int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *stop) {
+    if (start && stop) {
+        t_prof_start = reinterpret_cast<cudaEvent_t>(start);
+        t_prof_stop = reinterpret_cast<cudaEvent_t>(stop);
+    } else {
+        t_prof_start = t_prof_stop = nullptr;
+    }
+    return MLA_OK;
+}
+
+int mla_prefill_version(void) { return kVersion; }
+
+}  // extern "C"

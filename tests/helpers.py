@@ -1,0 +1,73 @@
+"""Shared test helpers: oracle runs on seeded inputs and the parity bound.
+
+Parity bound (stated for N(0,1) inputs, applied to every workload):
+  * mean |gpu - oracle| <= 1e-3 over all checked elements;
+  * max over elements of (|gpu - oracle| - ulp(oracle)/2) <= 1e-2, where ulp is
+    the spacing of the output dtype at the oracle value.  attenOut is stored in
+    fp16 / bf16, so an exactly computed result still carries up to half an
+    ulp of storage rounding (0.0156 for bf16 values in [4, 8)); the 1e-2 bound
+    applies to the error of the computation on top of that rounding.
+The literal max |gpu - oracle| is reported alongside.
+"""
+import numpy as np
+import torch
+
+import oracle
+
+MAX_ABS = 1e-2
+MEAN_ABS = 1e-3
+
+
+def half_ulp(ref, dtype):
+    """Half the spacing of ``dtype`` (fp16 / bf16) at |ref| (normal range)."""
+    mant = {torch.bfloat16: 7, torch.float16: 10}[dtype]
+    a = np.abs(ref)
+    tiny = {torch.bfloat16: 2.0 ** -126, torch.float16: 2.0 ** -14}[dtype]
+    e = np.floor(np.log2(np.maximum(a, tiny)))
+    return 0.5 * 2.0 ** (e - mant)
+
+
+def compare(got, ref, dtype, mask=None):
+    """Returns (ok, stats) for gpu output ``got`` vs oracle ``ref`` (both [T,H,D])."""
+    g = got.detach().cpu().double().numpy() if hasattr(got, "detach") else np.asarray(got, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    if mask is not None:
+        g, r = g[mask], r[mask]
+    if r.size == 0:
+        return True, {"n": 0}
+    if not np.all(np.isfinite(g)):
+        return False, {"n": int(r.size), "nonfinite": int((~np.isfinite(g)).sum())}
+    err = np.abs(g - r)
+    excess = err - half_ulp(r, dtype)
+    stats = {"n": int(r.size), "max_abs": float(err.max()), "mean_abs": float(err.mean()),
+             "max_excess_over_half_ulp": float(excess.max())}
+    ok = stats["max_excess_over_half_ulp"] <= MAX_ABS and stats["mean_abs"] <= MEAN_ABS
+    return ok, stats
+
+
+def oracle_rows(x, head_num, kv_head_num, qk_scale, rows=None, mask_type=oracle.MASK_CAUSAL, head_chunk=None):
+    """Oracle output for the given packed token rows (all rows if None).
+
+    Large problems are split by head groups (query heads [h0, h1) with their
+    kv heads): heads are independent, so each slice is itself a valid problem.
+    """
+    H, G = head_num, kv_head_num
+    g = H // G
+    t_q = x["q"].shape[0]
+    if head_chunk is None or head_chunk >= H:
+        return oracle.prefill(x["q"], x["q_rope"], x["k"], x["k_rope"], x["v"], x["q_seqlen"], x["kv_seqlen"],
+                              H, G, qk_scale, mask_type=mask_type, rows=rows)
+    assert head_chunk % g == 0
+    out = np.full((t_q, H, x["v"].shape[-1]), np.nan)
+    for h0 in range(0, H, head_chunk):
+        h1 = min(H, h0 + head_chunk)
+        k0, k1 = h0 // g, h1 // g
+        rows_q = x["q"][:, h0:h1] if rows is None else x["q"][:, h0:h1]
+        out[:, h0:h1] = oracle.prefill(rows_q, x["q_rope"][:, h0:h1], x["k"][:, k0:k1], x["k_rope"][:, k0:k1],
+                                       x["v"][:, k0:k1], x["q_seqlen"], x["kv_seqlen"], h1 - h0, k1 - k0, qk_scale,
+                                       mask_type=mask_type, rows=rows)
+    return out
+
+
+def cpu_copy(x):
+    return {k: v.detach().cpu() for k, v in x.items()}

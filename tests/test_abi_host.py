@@ -1,0 +1,180 @@
+"""C ABI checks that need no GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import mla_prefill_attention_varlen_b200 as mla
+from mla_prefill_attention_varlen_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return mla.load_library()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(HEADER_DIR, fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ \*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(n for n in names if n.startswith("mla_")))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("mla_prefill", "mla_prefill_device_status", "mla_status_string", "mla_prefill_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), "missing export %s" % n
+
+
+def test_library_is_sm100a_only():
+    out = os.popen("cuobjdump --list-elf %s 2>/dev/null" % build.LIB).read()
+    if not out:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out
+
+
+def test_status_strings(lib):
+    for code, name in mla.STATUS_NAMES.items():
+        assert lib.mla_status_string(code).decode().startswith(name)
+    assert lib.mla_status_string(12345).decode() == "unknown mla_status"
+    assert lib.mla_prefill_version() >= 100
+
+
+# ---------------------------------------------------------------------------
+# Host-side validation.  These descriptors point at host memory that is never
+# dereferenced: every call below must be rejected before any CUDA call.
+# ---------------------------------------------------------------------------
+
+def make_args(T=256, Tk=256, H=4, G=2, batch=2, dtype=torch.bfloat16):
+    t = dict(
+        q=torch.zeros(T, H, 128, dtype=dtype), q_rope=torch.zeros(T, H, 64, dtype=dtype),
+        k=torch.zeros(Tk, G, 128, dtype=dtype), k_rope=torch.zeros(Tk, G, 64, dtype=dtype),
+        v=torch.zeros(Tk, G, 128, dtype=dtype), q_seqlen=torch.zeros(batch, dtype=torch.int32),
+        kv_seqlen=torch.zeros(batch, dtype=torch.int32), out=torch.zeros(T, H, 128, dtype=dtype))
+    return t, H, G
+
+
+def call(lib, t, H, G, mask=1, scale=0.5, override=None):
+    d = {k: mla.as_mla_tensor(v) for k, v in t.items()}
+    for k, fn in (override or {}).items():
+        fn(d[k])
+    p = lambda k: ctypes.byref(d[k]) if d[k] is not None else None
+    return lib.mla_prefill(p("q"), p("q_rope"), p("k"), p("k_rope"), p("v"), p("q_seqlen"), p("kv_seqlen"), mask, H,
+                           G, scale, p("out"), None)
+
+
+def test_rejects_null(lib):
+    t, H, G = make_args()
+    d = {k: mla.as_mla_tensor(v) for k, v in t.items()}
+    rc = lib.mla_prefill(None, ctypes.byref(d["q_rope"]), ctypes.byref(d["k"]), ctypes.byref(d["k_rope"]),
+                         ctypes.byref(d["v"]), ctypes.byref(d["q_seqlen"]), ctypes.byref(d["kv_seqlen"]), 1, H, G,
+                         0.5, ctypes.byref(d["out"]), None)
+    assert rc == 1
+
+    def null_data(x):
+        x.data = None
+    assert call(lib, t, H, G, override={"v": null_data}) == 1
+
+
+@pytest.mark.parametrize("H,G", [(0, 1), (4, 0), (4, 3), (-1, 1)])
+def test_rejects_bad_heads(lib, H, G):
+    t, _, _ = make_args()
+    assert call(lib, t, H, G) == 5
+
+
+def test_rejects_heads_not_matching_shapes(lib):
+    t, H, G = make_args()
+    assert call(lib, t, 8, G) == 3  # q is [T, 4, 128]
+    assert call(lib, t, H, 4) == 3  # k is [T, 2, 128]
+
+
+def test_rejects_dtypes(lib):
+    t, H, G = make_args()
+    t["v"] = t["v"].half()
+    assert call(lib, t, H, G) == 2
+    t, H, G = make_args()
+    t["q_seqlen"] = t["q_seqlen"].long()
+    assert call(lib, t, H, G) == 2
+    t, H, G = make_args(dtype=torch.float32)
+    assert call(lib, t, H, G) == 2
+
+
+def test_rejects_shapes(lib):
+    t, H, G = make_args()
+    t["q_rope"] = torch.zeros(255, H, 64, dtype=torch.bfloat16)
+    assert call(lib, t, H, G) == 3
+    t, H, G = make_args()
+    t["k"] = torch.zeros(256, G, 96, dtype=torch.bfloat16)
+    assert call(lib, t, H, G) == 3
+    t, H, G = make_args()
+    t["kv_seqlen"] = torch.zeros(3, dtype=torch.int32)
+    assert call(lib, t, H, G) == 3
+    t, H, G = make_args()
+    t["out"] = torch.zeros(256, H, 64, dtype=torch.bfloat16)
+    assert call(lib, t, H, G) == 3
+
+
+def test_rejects_padded_kv_layout(lib):
+    # the page's [batch, max_seq, kv_head*embeddimV] form is not supported
+    t, H, G = make_args()
+    t["k"] = torch.zeros(2, 128, G * 128, dtype=torch.bfloat16)
+    assert call(lib, t, H, G) == 6
+
+
+def test_rejects_misalignment(lib):
+    t, H, G = make_args()
+
+    def shift(x):
+        x.data = x.data + 2
+    assert call(lib, t, H, G, override={"q": shift}) == 4
+
+    def odd_stride(x):
+        x.stride[0] = 4 * 128 + 4
+    assert call(lib, t, H, G, override={"k": odd_stride}) == 4
+
+    def inner_stride(x):
+        x.stride[2] = 2
+    assert call(lib, t, H, G, override={"v": inner_stride}) == 4
+
+
+def test_rejects_mask_scale_and_alias(lib):
+    t, H, G = make_args()
+    assert call(lib, t, H, G, mask=2) == 6
+    assert call(lib, t, H, G, scale=float("inf")) == 6
+    assert call(lib, t, H, G, scale=float("nan")) == 6
+    t, H, G = make_args(H=2, G=2)
+    t["out"] = t["v"]  # out aliasing an input
+    assert call(lib, t, H, G) == 6
+
+
+def test_accepts_2d_and_strided_views_on_host(lib):
+    # a well-formed call passes validation and only then reaches CUDA; with no
+    # GPU the result is MLA_ERR_CUDA (7), with a GPU the data would be device memory.
+    if torch.cuda.is_available():
+        pytest.skip("host-only check")
+    t, H, G = make_args()
+    t["q"] = t["q"].reshape(256, H * 128)
+    wide = torch.zeros(256, H, 192, dtype=torch.bfloat16)
+    t["q_rope"] = wide[:, :, 128:]
+    assert call(lib, t, H, G) == 7
+
+
+def test_empty_batch_is_a_no_op(lib):
+    t, H, G = make_args(batch=0)
+    assert call(lib, t, H, G) == 0

@@ -1,0 +1,282 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Element-by-element comparisons on seeded inputs: full oracle runs on small
+cases spanning several tiles and ragged tails, and sampled rows (every head)
+on the full-size workloads in the launch configuration the benchmark times.
+Indexing is checked bit-exactly (sentinel rows, guard regions, single-key rows,
+metamorphic identities).
+"""
+import numpy as np
+import pytest
+import torch
+
+import mla_prefill_attention_varlen_b200 as mla
+from mla_prefill_attention_varlen_b200 import workloads as W
+from helpers import compare, cpu_copy, oracle_rows
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    mla.load_library()
+    torch.cuda.set_device(0)
+    yield
+    torch.cuda.synchronize()
+
+
+def problem(lens_q, lens_k, H, G, dtype=torch.bfloat16, std=1.0, seed=0, extra_tokens=0):
+    wl = W.Workload("case", list(lens_q), list(lens_k), H, G, dtype=dtype, std=std, seed=seed)
+    x = W.make_inputs(wl, device=DEV)
+    if extra_tokens:
+        for key in ("q", "q_rope"):
+            pad = torch.randn(extra_tokens, *x[key].shape[1:], device=DEV).to(dtype)
+            x[key] = torch.cat([x[key], pad])
+    return wl, x
+
+
+def run(x, H, G, scale, mask=mla.MLA_MASK_CAUSAL, out=None, stream=None):
+    if out is None:
+        out = torch.full((x["q"].shape[0], H, 128), 7.0, dtype=x["q"].dtype, device=DEV)
+    mla.mla_prefill(x["q"], x["q_rope"], x["k"], x["k_rope"], x["v"], x["q_seqlen"], x["kv_seqlen"], mask, H, G,
+                    scale, out, stream)
+    return out
+
+
+def status():
+    return mla.mla_prefill_device_status()
+
+
+def check_against_oracle(x, out, H, G, scale, mask=mla.MLA_MASK_CAUSAL, rows=None, head_chunk=None):
+    torch.cuda.synchronize()
+    ref = oracle_rows(cpu_copy(x), H, G, scale, rows=rows, mask_type=mask, head_chunk=head_chunk)
+    computed = ~np.isnan(ref[:, 0, 0])
+    ok, st = compare(out.cpu(), ref, x["q"].dtype, mask=computed)
+    assert ok, st
+    return ref, st
+
+
+# ---------------------------------------------------------------------------
+# the five workloads
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny", "uniform"])
+def test_workload_full(name):
+    wl = W.get(name)
+    x = W.make_inputs(wl, device=DEV)
+    out = run(x, wl.head_num, wl.kv_head_num, wl.qk_scale)
+    _, st = check_against_oracle(x, out, wl.head_num, wl.kv_head_num, wl.qk_scale)
+    assert status() == 0
+    print(name, st)
+
+
+@pytest.mark.parametrize("name,per_seq,head_chunk", [("varlen_gqa", 24, None), ("long", 256, 16),
+                                                     ("chunked", 24, 32)])
+def test_workload_sampled(name, per_seq, head_chunk):
+    wl = W.get(name)
+    x = W.make_inputs(wl, device=DEV)
+    out = run(x, wl.head_num, wl.kv_head_num, wl.qk_scale)
+    rows = []
+    base = 0
+    for b, lq in enumerate(wl.q_seqlens):
+        rows += list(base + W.sample_rows(lq, per_seq, seed=100 + b))
+        base += lq
+    _, st = check_against_oracle(x, out, wl.head_num, wl.kv_head_num, wl.qk_scale, rows=rows,
+                                 head_chunk=head_chunk)
+    assert status() == 0
+    print(name, st)
+
+
+# ---------------------------------------------------------------------------
+# ragged and degenerate shapes (full oracle)
+# ---------------------------------------------------------------------------
+
+CASES = [
+    # lens_q, lens_k, H, G, dtype, scale, mask
+    ([1], [1], 1, 1, torch.bfloat16, 0.07, 1),
+    ([2, 3], [2, 3], 2, 1, torch.bfloat16, 0.07, 1),
+    ([127, 128, 129], [127, 128, 129], 4, 4, torch.bfloat16, 0.07, 1),
+    ([255, 1, 257], [255, 1, 257], 2, 2, torch.float16, 0.07, 1),
+    ([0, 5, 0, 130], [0, 5, 0, 130], 3, 1, torch.bfloat16, 0.07, 1),
+    ([300], [100], 2, 1, torch.bfloat16, 0.07, 1),          # Lq > Lk: leading rows see nothing
+    ([100, 37], [700, 300], 4, 2, torch.bfloat16, 0.07, 1),  # chunk over a prefix, unaligned
+    ([64, 200], [513, 200], 8, 1, torch.float16, 0.07, 1),
+    ([333], [333], 16, 4, torch.bfloat16, 0.07, 1),
+    ([129, 61], [129, 61], 6, 3, torch.bfloat16, 0.07, 1),
+    ([150, 20], [150, 20], 2, 2, torch.bfloat16, 0.0, 1),   # equal scores: cumulative means
+    ([150, 20], [150, 20], 2, 2, torch.bfloat16, -0.05, 1),  # negative scale
+    ([200], [200], 2, 1, torch.bfloat16, 0.5, 1),            # sharp softmax
+    ([130, 7], [130, 7], 2, 2, torch.bfloat16, 0.07, 0),     # no mask
+    ([100, 50], [260, 40], 2, 1, torch.float16, 0.07, 0),    # no mask, Lq != Lk
+    ([5], [0], 1, 1, torch.bfloat16, 0.07, 1),               # no keys at all
+]
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_ragged_cases(case):
+    lq, lk, H, G, dtype, scale, mask = CASES[case]
+    _, x = problem(lq, lk, H, G, dtype=dtype, seed=1000 + case, extra_tokens=3)
+    out = run(x, H, G, scale, mask)
+    ref, st = check_against_oracle(x, out, H, G, scale, mask)
+    # rows past sum(Lq) keep the sentinel, bit for bit
+    t_used = sum(lq)
+    assert torch.all(out[t_used:] == 7.0)
+    assert status() == 0
+
+
+def test_rows_without_keys_are_zero():
+    _, x = problem([300], [100], 2, 1, seed=7)
+    out = run(x, 2, 1, 0.07)
+    torch.cuda.synchronize()
+    assert torch.all(out[:200] == 0)
+
+
+# ---------------------------------------------------------------------------
+# layouts
+# ---------------------------------------------------------------------------
+
+def test_strided_and_2d_views():
+    H, G = 4, 2
+    lq = [200, 77]
+    _, x = problem(lq, lq, H, G, seed=11)
+    T = sum(lq)
+    ref_out = run(x, H, G, 0.07)
+    # q and q_rope as views into one [T, H, 192] buffer, k as [T, G*128], out as a view into a wider buffer
+    qbuf = torch.cat([x["q"], x["q_rope"]], dim=2).contiguous()
+    y = dict(x, q=qbuf[:, :, :128], q_rope=qbuf[:, :, 128:], k=x["k"].reshape(T, G * 128))
+    kbuf = torch.cat([x["k"], x["k_rope"]], dim=2).contiguous()
+    y["k_rope"] = kbuf[:, :, 128:]
+    wide = torch.full((T, H, 256), 3.0, dtype=torch.bfloat16, device=DEV)
+    out = wide[:, :, 64:192]
+    run(y, H, G, 0.07, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out)
+    assert torch.all(wide[:, :, :64] == 3.0) and torch.all(wide[:, :, 192:] == 3.0)
+    out2d = torch.empty(T, H * 128, dtype=torch.bfloat16, device=DEV)
+    run(x, H, G, 0.07, out=out2d)
+    torch.cuda.synchronize()
+    assert torch.equal(out2d.view(T, H, 128), ref_out)
+
+
+# ---------------------------------------------------------------------------
+# closed forms and metamorphic identities (bit-exact)
+# ---------------------------------------------------------------------------
+
+def test_first_row_is_exactly_v0():
+    lens = [37, 300, 129]
+    H, G = 8, 2
+    _, x = problem(lens, lens, H, G, seed=21)
+    out = run(x, H, G, 0.07)
+    torch.cuda.synchronize()
+    start = 0
+    for L in lens:
+        for h in range(H):
+            assert torch.equal(out[start, h], x["v"][start, h // (H // G)])
+        start += L
+
+
+def test_future_keys_do_not_leak():
+    L, H, G = 600, 2, 2
+    _, x = problem([L], [L], H, G, seed=31)
+    a = run(x, H, G, 0.07).clone()
+    r = 250  # rows < r cannot see keys >= r
+    y = {k: v.clone() for k, v in x.items()}
+    for key in ("k", "k_rope", "v"):
+        y[key][r:] = 1000.0
+    b = run(y, H, G, 0.07)
+    torch.cuda.synchronize()
+    assert torch.equal(a[:r], b[:r])
+
+
+def test_neighbour_sequences_do_not_leak():
+    lens, H, G = [150, 260, 90], 4, 1
+    _, x = problem(lens, lens, H, G, seed=41)
+    a = run(x, H, G, 0.07).clone()
+    y = {k: v.clone() for k, v in x.items()}
+    for key in ("q", "q_rope", "k", "k_rope", "v"):
+        y[key][150:410] = -1000.0
+    b = run(y, H, G, 0.07)
+    torch.cuda.synchronize()
+    assert torch.equal(a[:150], b[:150]) and torch.equal(a[410:], b[410:])
+
+
+def test_batch_invariance():
+    lens, H, G = [130, 1, 400, 77], 4, 2
+    _, x = problem(lens, lens, H, G, seed=51)
+    whole = run(x, H, G, 0.07).clone()
+    start = 0
+    for L in lens:
+        y = dict(x, q=x["q"][start:start + L], q_rope=x["q_rope"][start:start + L], k=x["k"][start:start + L],
+                 k_rope=x["k_rope"][start:start + L], v=x["v"][start:start + L],
+                 q_seqlen=torch.tensor([L], dtype=torch.int32, device=DEV),
+                 kv_seqlen=torch.tensor([L], dtype=torch.int32, device=DEV))
+        one = run(y, H, G, 0.07)
+        torch.cuda.synchronize()
+        assert torch.equal(one, whole[start:start + L])
+        start += L
+
+
+def test_gqa_equals_repeated_kv():
+    lens, H, G = [200, 311], 8, 2
+    _, x = problem(lens, lens, H, G, seed=61)
+    a = run(x, H, G, 0.07).clone()
+    g = H // G
+    y = dict(x, k=x["k"].repeat_interleave(g, dim=1).contiguous(),
+             k_rope=x["k_rope"].repeat_interleave(g, dim=1).contiguous(),
+             v=x["v"].repeat_interleave(g, dim=1).contiguous())
+    b = run(y, H, H, 0.07)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_chunk_equals_suffix_of_full_run():
+    Lk, Lq, H = 1024, 256, 4
+    _, x = problem([Lk], [Lk], H, H, seed=71)
+    full = run(x, H, H, 0.07).clone()
+    y = dict(x, q=x["q"][Lk - Lq:].contiguous(), q_rope=x["q_rope"][Lk - Lq:].contiguous(),
+             q_seqlen=torch.tensor([Lq], dtype=torch.int32, device=DEV))
+    chunk = run(y, H, H, 0.07)
+    torch.cuda.synchronize()
+    assert torch.equal(chunk, full[Lk - Lq:])
+
+
+def test_repeatable_and_stream_ordered():
+    lens, H, G = [500, 123], 4, 4
+    _, x = problem(lens, lens, H, G, seed=81)
+    a = run(x, H, G, 0.07).clone()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = run(x, H, G, 0.07, stream=s)
+    s.synchronize()
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# device-detected seqlen errors: clamped, reported, never out of bounds
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bad", ["sum_too_large", "negative", "kv_too_large"])
+def test_inconsistent_seqlens_are_clamped_and_reported(bad):
+    H, G = 2, 1
+    lens = [100, 60]
+    _, x = problem(lens, lens, H, G, seed=91)
+    if bad == "sum_too_large":
+        x["q_seqlen"] = torch.tensor([100, 90], dtype=torch.int32, device=DEV)
+    elif bad == "negative":
+        x["q_seqlen"] = torch.tensor([-5, 60], dtype=torch.int32, device=DEV)
+    else:
+        x["kv_seqlen"] = torch.tensor([100, 500], dtype=torch.int32, device=DEV)
+    T = sum(lens)
+    guard = 64
+    buf = torch.full((T + 2 * guard, H, 128), 5.0, dtype=torch.bfloat16, device=DEV)
+    out = buf[guard:guard + T]
+    assert status() == 0
+    run(x, H, G, 0.07, out=out)
+    assert status() == 8
+    assert torch.all(buf[:guard] == 5.0) and torch.all(buf[guard + T:] == 5.0)
+    assert torch.isfinite(out.float()).all() or bad == "negative"
+    assert status() == 0  # reading clears it
