@@ -139,8 +139,13 @@ def set_profile_events(start=None, stop=None):
     lib = load_library()
     if start is None or stop is None:
         lib.mla_prefill_set_profile_events(None, None)
-    else:
-        lib.mla_prefill_set_profile_events(start.cuda_event, stop.cuda_event)
+        return
+    for ev in (start, stop):
+        if not ev.cuda_event:  # torch creates the CUDA event on its first record
+            ev.record()
+    if not (start.cuda_event and stop.cuda_event):
+        raise RuntimeError("could not create CUDA events")
+    lib.mla_prefill_set_profile_events(start.cuda_event, stop.cuda_event)
 
 
 def mla_prefill_device_status(stream=None):

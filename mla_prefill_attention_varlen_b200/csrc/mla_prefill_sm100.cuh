@@ -289,6 +289,24 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
     }
 }
 
+// Max of a 128-element row as a balanced tree (short dependency chains).
+__device__ __forceinline__ float row_max(const float (&s)[kBN]) {
+    float m[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m[i] = fmaxf(s[i], s[i + 16]);
+#pragma unroll
+    for (int c = 32; c < kBN; c += 16) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m[i] = fmaxf(m[i], s[c + i]);
+    }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+    }
+    return m[0];
+}
+
 // ---------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------
@@ -537,18 +555,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int c = 0; c < kBN; ++c) s[c] = c < lim ? s[c] : -INFINITY;
                     }
-                    float mx = s[0];
-#pragma unroll
-                    for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
-                    m_tile = mx * sl2;
+                    m_tile = row_max(s) * sl2;
                 } else {
                     const int lim = tile_masked ? lim_row - kv0 : kBN;
 #pragma unroll
                     for (int c = 0; c < kBN; ++c) s[c] = c < lim ? s[c] * sl2 : -INFINITY;
-                    float mx = s[0];
-#pragma unroll
-                    for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
-                    m_tile = mx;
+                    m_tile = row_max(s);
                 }
                 // Lazy rescaling: keep the old reference max unless the new one is 2^8 larger.
                 float alpha = 1.f;
@@ -558,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
                 uint32_t pk[kBN / 2];
-                float rowsum = 0.f;
+                float psum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
                 for (int c = 0; c < kBN; c += 2) {
                     float p0, p1;
@@ -569,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         p0 = ptx::ex2(s[c] - m_use);
                         p1 = ptx::ex2(s[c + 1] - m_use);
                     }
-                    rowsum += p0 + p1;
+                    psum[(c / 2) & 7] += p0 + p1;
                     pk[c / 2] = DType<T>::pack(p0, p1);
                 }
                 if (j > 0) {
@@ -591,6 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                const float rowsum = ((psum[0] + psum[1]) + (psum[2] + psum[3])) +
+                                     ((psum[4] + psum[5]) + (psum[6] + psum[7]));
                 l_run = l_run * alpha + rowsum;
 #pragma unroll
                 for (int c = 0; c < kBN / 2 / 32; ++c) {
