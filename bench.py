@@ -58,54 +58,116 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+    """SM clock and clock-event (throttle) samples taken while the timed region runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Samples come from NVML every ~20 ms in a background thread, stamped with the
+    host clock; only samples inside [mark_start, mark_stop] are summarised.  The
+    GPU is found by its UUID (CUDA and NVML may number devices differently).
+    Falls back to `nvidia-smi -lms 100` when NVML is unavailable.
+    """
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index, period=0.02):
+        self.cuda_index = cuda_index
+        self.period = period
+        self.samples = []
+        self.t0 = self.t1 = None
+        self._stop = False
+        self._thread = None
+        self._proc = None
+        self.source = None
+
+    def _uuid(self):
+        import torch
+
+        try:
+            u = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return None
 
     def __enter__(self):
+        import threading
+
+        uuid = self._uuid()
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else pynvml.nvmlDeviceGetHandleByIndex(0)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+
+            def loop():
+                while not self._stop:
+                    t = time.perf_counter()
+                    try:
+                        self.samples.append((t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                             pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                             int(get_reasons(h))))
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            self.source = "nvml"
+        except Exception:
+            self.source = "nvidia-smi"
+            sel = ["-i", uuid] if uuid else []
+            try:
+                self._proc = subprocess.Popen(
+                    ["nvidia-smi"] + sel + ["--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                                            "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self._proc_t0 = time.perf_counter()
+            except (OSError, ValueError):
+                self._proc = None
         return self
 
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_stop(self):
+        self.t1 = time.perf_counter()
+
     def __exit__(self, *exc):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(1.0)
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                out, _ = self._proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self._proc.kill()
+                out, _ = self._proc.communicate()
+            # nvidia-smi lines carry no host stamps: spread them evenly over the process lifetime
+            lines = [l for l in (out or "").strip().splitlines() if l.count(",") >= 2]
+            t_end = time.perf_counter()
+            for k, line in enumerate(lines):
+                parts = [x.strip() for x in line.split(",")]
+                try:
+                    t = self._proc_t0 + (t_end - self._proc_t0) * (k + 0.5) / max(1, len(lines))
+                    self.samples.append((t, float(parts[0]), float(parts[1]), int(parts[2], 16)))
+                except ValueError:
+                    continue
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in (self.out or "").strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [s for s in self.samples if self.t0 is None or (self.t0 <= s[0] <= (self.t1 or s[0]))]
+        if not inside:
+            inside = self.samples
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = set()
+        for s in inside:
+            for bit, name in self.REASONS.items():
+                if s[3] & bit:
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([s[1] for s in inside])), "sm_max_mhz": float(max(s[2] for s in inside)),
+                "reasons": sorted(reasons), "samples": len(inside), "source": self.source}
 
 
 def dist_setup(n_gpus):
@@ -132,14 +194,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The maximum of a per-rank float over all ranks (device time is judged by the slowest rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, units_per_rank, ms_max):
+    """Whole-job rate: every rank processes units_per_rank in (at most) ms_max milliseconds."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 def time_oracle_sample(wl, x_cpu, target_s, seed=0):
@@ -272,11 +341,12 @@ def main():
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     k_stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    smi = ClockSampler(local if world > 1 else torch.cuda.current_device())
+    smi = ClockSampler(torch.cuda.current_device())
     torch.cuda.synchronize()
     barrier(world)
     with smi:
-        time.sleep(0.3)
+        time.sleep(0.1)
+        smi.mark_start()
         for i in range(args.steps):
             if flush is not None:
                 flush.zero_()
@@ -286,6 +356,7 @@ def main():
             stops[i].record(stream)
         mla.set_profile_events(None, None)
         torch.cuda.synchronize()
+        smi.mark_stop()
     barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
     kern_ms = [a.elapsed_time(b) for a, b in zip(k_starts, k_stops)]
@@ -297,8 +368,8 @@ def main():
 
     triples = visible_triples(wl)
     flops = triples * FLOPS_PER_TRIPLE
-    value = world * flops / (ms * 1e-3) / 1e12
-    tokens_per_s = world * wl.t_q / (ms * 1e-3)
+    value = job_throughput(world, flops, ms) / 1e12
+    tokens_per_s = job_throughput(world, wl.t_q, ms)
     peaks, peak_src = load_peaks()
     kern_tflops = flops / (kms * 1e-3) / 1e12
 

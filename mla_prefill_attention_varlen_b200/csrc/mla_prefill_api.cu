@@ -106,13 +106,13 @@ int ensure_encode() {
     return MLA_OK;
 }
 
-// 3-D map {width, heads, tokens} with a {64, 1, 128} box and 128-byte swizzle.
-int encode_map(CUtensorMap *m, const View3 &v, bool bf16, void *dummy) {
+// 3-D map {width, heads, tokens} with a {64, 1, box_tokens} box and 128-byte swizzle.
+int encode_map(CUtensorMap *m, const View3 &v, bool bf16, void *dummy, int box_tokens) {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(v.width), static_cast<cuuint64_t>(v.heads),
                                 static_cast<cuuint64_t>(v.tokens > 0 ? v.tokens : 1)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>((v.heads > 1 ? v.st_head : v.width) * 2),
                                    static_cast<cuuint64_t>((v.tokens > 1 ? v.st_tok : v.heads * v.width) * 2)};
-    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_tokens)};
     const cuuint32_t estr[3] = {1, 1, 1};
     // An empty tensor is never read (no work item touches it); encode a valid dummy base.
     void *base = (v.tokens > 0 && v.data) ? v.data : dummy;
@@ -125,25 +125,25 @@ int encode_map(CUtensorMap *m, const View3 &v, bool bf16, void *dummy) {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t seq_info, tile_off, hist, tiles, num_tiles, total;
+    size_t seq_info, unit_off, hist, units, num_units, total;
     int hist_len;
 };
 
 WsLayout ws_layout(int64_t batch, int64_t t_q, int64_t t_k) {
     WsLayout l;
-    const int64_t max_tiles = (t_q + mla::kBM - 1) / mla::kBM + batch;
+    const int64_t max_units = (t_q + mla::kUnitRows - 1) / mla::kUnitRows + batch;
     l.hist_len = static_cast<int>((t_k + mla::kBN - 1) / mla::kBN + 2);
     size_t off = 0;
-    l.num_tiles = off;
+    l.num_units = off;
     off = align_up(off + 16, 256);
     l.seq_info = off;
     off = align_up(off + sizeof(int4) * batch, 256);
-    l.tile_off = off;
+    l.unit_off = off;
     off = align_up(off + sizeof(int) * (batch + 1), 256);
     l.hist = off;
     off = align_up(off + sizeof(int) * l.hist_len, 256);
-    l.tiles = off;
-    off = align_up(off + sizeof(int2) * max_tiles, 256);
+    l.units = off;
+    off = align_up(off + sizeof(int2) * max_units, 256);
     l.total = off;
     return l;
 }
@@ -247,29 +247,29 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
 
     const bool bf16 = dt == MLA_BF16;
     CUtensorMap maps[5];
-    if ((rc = encode_map(&maps[0], vq, bf16, ds->ws)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[1], vqr, bf16, ds->ws)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[2], vk, bf16, ds->ws)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[3], vkr, bf16, ds->ws)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[4], vv, bf16, ds->ws)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[0], vq, bf16, ds->ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[1], vqr, bf16, ds->ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[2], vk, bf16, ds->ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[3], vkr, bf16, ds->ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[4], vv, bf16, ds->ws, 64)) != MLA_OK) return rc;
 
     uint8_t *ws = static_cast<uint8_t *>(ds->ws);
-    int *num_tiles = reinterpret_cast<int *>(ws + lay.num_tiles);
+    int *num_units = reinterpret_cast<int *>(ws + lay.num_units);
     int4 *seq_info = reinterpret_cast<int4 *>(ws + lay.seq_info);
-    int *tile_off = reinterpret_cast<int *>(ws + lay.tile_off);
+    int *unit_off = reinterpret_cast<int *>(ws + lay.unit_off);
     int *hist = reinterpret_cast<int *>(ws + lay.hist);
-    int2 *tiles = reinterpret_cast<int2 *>(ws + lay.tiles);
+    int2 *units = reinterpret_cast<int2 *>(ws + lay.units);
     const bool causal = mask_type == MLA_MASK_CAUSAL;
 
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
         static_cast<const int *>(q_seqlen->data), static_cast<const int *>(kv_seqlen->data), static_cast<int>(batch),
-        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, tile_off, hist, lay.hist_len, tiles, num_tiles, ds->status);
+        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, ds->status);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
     mla::Params p;
     p.seq_info = seq_info;
-    p.tiles = tiles;
-    p.num_tiles = num_tiles;
+    p.units = units;
+    p.num_units = num_units;
     p.status = ds->status;
     p.out = vo.data;
     p.out_st = vo.st_tok;
@@ -278,7 +278,7 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
     p.group = head_num / kv_head_num;
     p.scale_log2 = qk_scale * 1.4426950408889634f;
 
-    const int64_t max_items = ((vq.tokens + mla::kBM - 1) / mla::kBM + batch) * head_num;
+    const int64_t max_items = ((vq.tokens + mla::kUnitRows - 1) / mla::kUnitRows + batch) * head_num;
     const int grid = static_cast<int>(max_items < ds->sm_count ? max_items : ds->sm_count);
     const bool pos = qk_scale > 0.f;
     if (bf16) {

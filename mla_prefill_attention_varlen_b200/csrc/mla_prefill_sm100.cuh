@@ -10,17 +10,24 @@
 //   key j visible iff j <= i + (Lk - Lq)          (causal, bottom-right)
 //   O[i,h] = sum_j softmax_j(s_ij) V[j,kh]
 //
-// Work unit: one 128-row query tile of one sequence for one query head.  Per
-// unit the kernel walks 128-key tiles j = 0 .. n_kv-1 (tiles wholly above the
-// causal diagonal are never visited):
-//   MMA warp   S_j = [Qn|Qr] [Kn|Kr]_j^T   (12 MMAs 128x128x16 into TMEM, the
-//              nope and rope k-steps accumulate into the same accumulator)
-//              O  += P_{j-1} V_{j-1}        (8 MMAs, P read from TMEM)
-//   softmax    rows of S_j -> mask -> running max / sum -> P_j (16-bit) in TMEM,
-//              lazy rescale of O when the running max grows by more than 2^8
-//   load warp  TMA tiles of Q (once per unit), K_j and V_j (2-deep rings)
-// Tensor memory (512 columns): S double buffer [0,256), O [256,384),
-// P double buffer [384,512) (16-bit pairs packed per 32-bit column).
+// Work unit: 256 query rows (two 128-row tiles t = 0, 1) of one sequence for
+// one query head.  Both tiles share every K/V tile the kernel loads.  Per
+// unit the kernel walks 128-key tiles j = 0 .. n-1; tiles wholly above the
+// causal diagonal of a query tile are never visited for that tile:
+//   MMA warp    S_t = [Qn|Qr]_t [Kn|Kr]_j^T  (12 MMAs 128x128x16 into TMEM; the
+//               nope and rope k-steps accumulate into one accumulator)
+//               O_t += P_t V_j                (8 MMAs, P read from TMEM)
+//   softmax     warpgroup t owns tile t: rows of S_t -> mask -> running max /
+//               sum -> P_t (16-bit) written back over S_t in TMEM; lazy rescale
+//               of O_t when the running max grows by more than 2^8
+//   load warp   TMA: Q tiles once per unit, then K_j (3 x 16 KB) and V_j
+//               (2 x 16 KB) through a ring of eight 16 KB chunks
+// MMA issue order per key tile: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while
+// one warpgroup computes a softmax the tensor pipe works on the other tile.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384),
+// O1 [384,512); P_t occupies columns [64,128) of S_t.  S_t(j+1) is issued
+// behind PV_t(j), which reads P_t(j); tcgen05.mma operations issued by one
+// thread execute in issue order.
 #pragma once
 
 #include <cuda.h>
@@ -33,31 +40,35 @@
 
 namespace mla {
 
-constexpr int kBM = 128;  // query rows per tile (= TMEM lanes)
-constexpr int kBN = 128;  // keys per tile
-constexpr int kDn = 128;  // nope width of Q/K, width of V (embeddimV)
-constexpr int kDr = 64;   // rope width
+constexpr int kBM = 128;         // query rows per tile (= TMEM lanes)
+constexpr int kUnitRows = 256;   // query rows per work unit (two tiles)
+constexpr int kBN = 128;         // keys per key tile
+constexpr int kDn = 128;         // nope width of Q/K, width of V (embeddimV)
+constexpr int kDr = 64;          // rope width
 
-constexpr int kChunkBytes = 128 * 64 * 2;  // one [128 rows x 64 cols] 16-bit block, 128-B swizzled
-constexpr int kQBytes = 3 * kChunkBytes;   // Qn cols 0-63, Qn cols 64-127, Qr
-constexpr int kKBytes = 3 * kChunkBytes;   // Kn cols 0-63, Kn cols 64-127, Kr
-constexpr int kVBytes = 2 * kChunkBytes;   // V cols 0-63, V cols 64-127
-constexpr int kKStages = 2;
-constexpr int kVStages = 2;
+constexpr int kChunkBytes = 16384;            // one ring chunk
+constexpr int kQTileBytes = 3 * kChunkBytes;  // Qn cols 0-63 | Qn cols 64-127 | Qr  (128 rows each)
+constexpr int kRing = 8;                      // ring chunks
+constexpr int kKChunks = 3;                   // Kn lo | Kn hi | Kr            (128 keys each)
+constexpr int kVChunks = 2;                   // keys 0-63 | keys 64-127      (V cols 0-63 then 64-127 inside)
+constexpr int kVHalfBytes = 8192;             // 64 keys x 64 V columns
 
 constexpr int kSmemQ = 0;
-constexpr int kSmemK = kSmemQ + kQBytes;
-constexpr int kSmemV = kSmemK + kKStages * kKBytes;
-constexpr int kSmemBar = kSmemV + kVStages * kVBytes;
-constexpr int kSmemBytes = kSmemBar + 256;
+constexpr int kSmemRing = kSmemQ + 2 * kQTileBytes;
+constexpr int kSmemBar = kSmemRing + kRing * kChunkBytes;
+constexpr int kSmemBytes = kSmemBar + 512;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 
-constexpr uint32_t kTmemS = 0;
-constexpr uint32_t kTmemO = 256;
-constexpr uint32_t kTmemP = 384;
+constexpr uint32_t kTmemS = 0;      // S_t at t * 128
+constexpr uint32_t kTmemO = 256;    // O_t at 256 + t * 128
+constexpr uint32_t kTmemPOff = 64;  // P_t at S_t + 64
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kThreads = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-5: softmax / epilogue
+constexpr int kThreads = 384;  // warpgroup 0: TMA (warp 0), MMA (warp 1); warpgroups 1, 2: softmax of tiles 0, 1
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 224;
+static_assert(kRegsLow * 128 + kRegsHigh * 256 <= 65536 / kThreads / 8 * 8 * kThreads,
+              "register split exceeds the launch's register file share");
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a pipeline wait gives up after 2 s
 
@@ -67,60 +78,73 @@ constexpr int kStatusTimeout = 9;
 
 struct Params {
     const int4 *seq_info;  // per sequence {cq, ck, lq, lk} after clamping
-    const int2 *tiles;     // (sequence, query-tile) pairs, most key tiles first
-    const int *num_tiles;  // number of valid entries in tiles
+    const int2 *units;     // (sequence, 256-row unit) pairs, most key tiles first
+    const int *num_units;  // number of valid entries in units
     int *status;           // sticky device status word
     void *out;
     long long out_st, out_sh;  // token / head strides of out, elements
     int head_num;
-    int group;  // head_num / kv_head_num
+    int group;         // head_num / kv_head_num
     float scale_log2;  // qk_scale * log2(e)
 };
 
 struct Barriers {
-    uint64_t q_full, q_empty;
-    uint64_t k_full[kKStages], k_empty[kKStages];
-    uint64_t v_full[kVStages], v_empty[kVStages];
-    uint64_t s_full[2], s_empty[2];
-    uint64_t p_full[2];
-    uint64_t o_done, o_empty;
+    uint64_t q_full[2], q_empty[2];
+    uint64_t ch_full[kRing], ch_empty[kRing];
+    uint64_t s_full[2], p_full[2];
+    uint64_t o_full[2], o_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
-static_assert(sizeof(Barriers) <= 256, "barrier block too large");
+static_assert(sizeof(Barriers) <= 512, "barrier block too large");
 
-// Number of 128-key tiles a query tile touches: the keys visible to its last
-// row (causal) or all keys.  0 when no row sees any key.
+// Number of 128-key tiles a 128-row query tile touches: the keys visible to its
+// last row (causal) or all keys.  0 when the tile has no rows or sees no key.
 __host__ __device__ __forceinline__ int kv_tiles_for(int q0, int rows, int lq, int lk, bool causal) {
+    if (rows <= 0) return 0;
     const int kv_end = causal ? min(q0 + rows + (lk - lq), lk) : lk;
     return kv_end > 0 ? (kv_end + kBN - 1) / kBN : 0;
 }
 
+__host__ __device__ __forceinline__ int tile_rows(int q0, int lq) { return max(0, min(kBM, lq - q0)); }
+
+// Key tiles a 256-row unit walks (the larger of its two tiles' counts).
+__host__ __device__ __forceinline__ int unit_cost(int u0, int lq, int lk, bool causal) {
+    const int a = kv_tiles_for(u0, tile_rows(u0, lq), lq, lk, causal);
+    const int b = kv_tiles_for(u0 + kBM, tile_rows(u0 + kBM, lq), lq, lk, causal);
+    return a > b ? a : b;
+}
+
 struct WorkItem {
     int h, kh;
-    int q_tok0, k_tok0;  // first packed token of the query tile / of the sequence's keys
-    int q0;              // first query row of the tile within its sequence
-    int rows;            // valid query rows in the tile (<= 128)
-    int off;             // Lk - Lq
-    int lk;
-    int n_kv;
+    int u0;              // first query row of the unit within its sequence
+    int q_tok0, k_tok0;  // first packed token of the unit / of the sequence's keys
+    int lq, lk, off;     // off = Lk - Lq
+    int rows[2];         // valid rows of tile 0 / 1
+    int n[2];            // key tiles of tile 0 / 1
+    int n_max;
 };
 
 __device__ __forceinline__ WorkItem decode_item(const Params &p, int it, bool causal) {
-    const int tile = it / p.head_num;
+    const int u = it / p.head_num;
     WorkItem x;
-    x.h = it - tile * p.head_num;
+    x.h = it - u * p.head_num;
     x.kh = x.h / p.group;
-    const int2 bm = p.tiles[tile];
+    const int2 bm = p.units[u];
     const int4 s = p.seq_info[bm.x];
-    x.q0 = bm.y * kBM;
-    x.rows = min(kBM, s.z - x.q0);
-    x.q_tok0 = s.x + x.q0;
+    x.u0 = bm.y * kUnitRows;
+    x.q_tok0 = s.x + x.u0;
     x.k_tok0 = s.y;
-    x.off = s.w - s.z;
+    x.lq = s.z;
     x.lk = s.w;
-    x.n_kv = kv_tiles_for(x.q0, x.rows, s.z, s.w, causal);
+    x.off = s.w - s.z;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        x.rows[t] = tile_rows(x.u0 + t * kBM, s.z);
+        x.n[t] = kv_tiles_for(x.u0 + t * kBM, x.rows[t], s.z, s.w, causal);
+    }
+    x.n_max = max(x.n[0], x.n[1]);
     return x;
 }
 
@@ -164,7 +188,7 @@ struct DType<__half> {
 // ---------------------------------------------------------------------------
 // Plan kernel: one block of 1024 threads.  Clamps the seqlens to the tensor
 // extents (recording kStatusSeqlen on any inconsistency), writes per-sequence
-// offsets, and writes the (sequence, query tile) list sorted by descending
+// offsets, and writes the (sequence, 256-row unit) list sorted by descending
 // number of key tiles (a counting sort; ties in arbitrary order).
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
@@ -195,19 +219,28 @@ __device__ __forceinline__ long long block_exclusive_scan(long long v, long long
     return before;
 }
 
+__device__ __forceinline__ int seq_of_unit(const int *unit_off, int batch, int t) {
+    int lo = 0, hi = batch - 1;  // last b with unit_off[b] <= t (sequences without units are skipped)
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (unit_off[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__restrict__ q_seqlen,
                                                                 const int *__restrict__ kv_seqlen, int batch,
                                                                 long long t_q, long long t_k, int causal,
-                                                                int4 *seq_info, int *tile_off, int *hist,
-                                                                int hist_len, int2 *tiles, int *num_tiles,
+                                                                int4 *seq_info, int *unit_off, int *hist,
+                                                                int hist_len, int2 *units, int *num_units,
                                                                 int *status) {
     __shared__ long long warp_sums[32];
     __shared__ int bad;
     if (threadIdx.x == 0) bad = 0;
     __syncthreads();
 
-    // 1. clamped prefix sums and query-tile counts, in chunks of blockDim.x sequences
-    long long carry_q = 0, carry_k = 0, carry_t = 0;
+    // 1. clamped prefix sums and unit counts, in chunks of blockDim.x sequences
+    long long carry_q = 0, carry_k = 0, carry_u = 0;
     for (int base = 0; base < batch; base += blockDim.x) {
         const int b = base + threadIdx.x;
         long long lq = 0, lk = 0;
@@ -225,33 +258,27 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
         const long long ck = pk < t_k ? pk : t_k, ek = pk + lk < t_k ? pk + lk : t_k;
         if (b < batch && (eq - cq != lq || ek - ck != lk)) bad = 1;
         const int lqc = static_cast<int>(eq - cq), lkc = static_cast<int>(ek - ck);
-        const long long nt = (b < batch) ? (lqc + kBM - 1) / kBM : 0;
-        long long tot_t;
-        const long long pt = carry_t + block_exclusive_scan(nt, tot_t, warp_sums);
+        const long long nu = (b < batch) ? (lqc + kUnitRows - 1) / kUnitRows : 0;
+        long long tot_u;
+        const long long pu = carry_u + block_exclusive_scan(nu, tot_u, warp_sums);
         if (b < batch) {
             seq_info[b] = make_int4(static_cast<int>(cq), static_cast<int>(ck), lqc, lkc);
-            tile_off[b] = static_cast<int>(pt);
+            unit_off[b] = static_cast<int>(pu);
         }
         carry_q += tot_q;
         carry_k += tot_k;
-        carry_t += tot_t;
+        carry_u += tot_u;
     }
-    const int total_tiles = static_cast<int>(carry_t);
-    if (threadIdx.x == 0) tile_off[batch] = total_tiles;
+    const int total = static_cast<int>(carry_u);
+    if (threadIdx.x == 0) unit_off[batch] = total;
     for (int c = threadIdx.x; c < hist_len; c += blockDim.x) hist[c] = 0;
     __syncthreads();
 
     // 2. histogram of key-tile counts
-    for (int t = threadIdx.x; t < total_tiles; t += blockDim.x) {
-        int lo = 0, hi = batch - 1;  // last b with tile_off[b] <= t
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (tile_off[mid] <= t) lo = mid; else hi = mid - 1;
-        }
-        const int4 s = seq_info[lo];
-        const int m = t - tile_off[lo];
-        const int q0 = m * kBM;
-        const int cost = kv_tiles_for(q0, min(kBM, s.z - q0), s.z, s.w, causal != 0);
+    for (int t = threadIdx.x; t < total; t += blockDim.x) {
+        const int b = seq_of_unit(unit_off, batch, t);
+        const int4 s = seq_info[b];
+        const int cost = unit_cost((t - unit_off[b]) * kUnitRows, s.z, s.w, causal != 0);
         atomicAdd(&hist[min(cost, hist_len - 1)], 1);
     }
     __syncthreads();
@@ -270,21 +297,16 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
     __syncthreads();
 
     // 4. scatter
-    for (int t = threadIdx.x; t < total_tiles; t += blockDim.x) {
-        int lo = 0, hi = batch - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (tile_off[mid] <= t) lo = mid; else hi = mid - 1;
-        }
-        const int4 s = seq_info[lo];
-        const int m = t - tile_off[lo];
-        const int q0 = m * kBM;
-        const int cost = kv_tiles_for(q0, min(kBM, s.z - q0), s.z, s.w, causal != 0);
+    for (int t = threadIdx.x; t < total; t += blockDim.x) {
+        const int b = seq_of_unit(unit_off, batch, t);
+        const int4 s = seq_info[b];
+        const int m = t - unit_off[b];
+        const int cost = unit_cost(m * kUnitRows, s.z, s.w, causal != 0);
         const int pos = atomicAdd(&hist[min(cost, hist_len - 1)], 1);
-        tiles[pos] = make_int2(lo, m);
+        units[pos] = make_int2(b, m);
     }
     if (threadIdx.x == 0) {
-        *num_tiles = total_tiles;
+        *num_units = total;
         if (bad) atomicCAS(status, 0, kStatusSeqlen);
     }
 }
@@ -319,8 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Barriers *bars = reinterpret_cast<Barriers *>(smem + kSmemBar);
     const uint32_t sQ = ptx::smem_addr(smem + kSmemQ);
-    const uint32_t sK = ptx::smem_addr(smem + kSmemK);
-    const uint32_t sV = ptx::smem_addr(smem + kSmemV);
+    const uint32_t sRing = ptx::smem_addr(smem + kSmemRing);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -328,23 +349,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](uint64_t &b) { return ptx::smem_addr(&b); };
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(bar(bars->q_full), 1);
-        ptx::mbar_init(bar(bars->q_empty), 1);
-        for (int s = 0; s < kKStages; ++s) {
-            ptx::mbar_init(bar(bars->k_full[s]), 1);
-            ptx::mbar_init(bar(bars->k_empty[s]), 1);
+        for (int t = 0; t < 2; ++t) {
+            ptx::mbar_init(bar(bars->q_full[t]), 1);
+            ptx::mbar_init(bar(bars->q_empty[t]), 1);
+            ptx::mbar_init(bar(bars->s_full[t]), 1);
+            ptx::mbar_init(bar(bars->p_full[t]), kBM);
+            ptx::mbar_init(bar(bars->o_full[t]), 1);
+            ptx::mbar_init(bar(bars->o_empty[t]), kBM);
         }
-        for (int s = 0; s < kVStages; ++s) {
-            ptx::mbar_init(bar(bars->v_full[s]), 1);
-            ptx::mbar_init(bar(bars->v_empty[s]), 1);
+        for (int c = 0; c < kRing; ++c) {
+            ptx::mbar_init(bar(bars->ch_full[c]), 1);
+            ptx::mbar_init(bar(bars->ch_empty[c]), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(bar(bars->s_full[s]), 1);
-            ptx::mbar_init(bar(bars->s_empty[s]), kBM);
-            ptx::mbar_init(bar(bars->p_full[s]), kBM);
-        }
-        ptx::mbar_init(bar(bars->o_done), 1);
-        ptx::mbar_init(bar(bars->o_empty), kBM);
         ptx::mbar_init(bar(bars->drain), 1);
         bars->abort = 0;
         ptx::fence_mbar_init();
@@ -358,11 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    const int n_items = *p.num_tiles * p.head_num;
+    const int n_items = *p.num_units * p.head_num;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (warp < 4) {
+        ptx::regs_dec<kRegsLow>();
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------- TMA producer
             ptx::tma_prefetch_desc(&tm_q);
             ptx::tma_prefetch_desc(&tm_qr);
             ptx::tma_prefetch_desc(&tm_k);
@@ -370,166 +387,210 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tma_prefetch_desc(&tm_v);
             const uint64_t pol_q = ptx::policy_evict_first();
             const uint64_t pol_kv = ptx::policy_evict_last();
-            uint32_t qc = 0, kc = 0, vc = 0;
+            uint32_t rc = 0;                // ring chunks filled
+            uint32_t ql0 = 0, ql1 = 0;      // Q tiles loaded per tile slot
             bool ok = true;
+            auto next_chunk = [&](uint32_t &dst, uint32_t &fb) -> bool {
+                const uint32_t slot = rc % kRing;
+                if (!wait_bar(bar(bars->ch_empty[slot]), ((rc / kRing) & 1) ^ 1, bars, p.status)) return false;
+                dst = sRing + slot * kChunkBytes;
+                fb = bar(bars->ch_full[slot]);
+                ptx::mbar_arrive_expect_tx(fb, kChunkBytes);
+                ++rc;
+                return true;
+            };
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const WorkItem x = decode_item(p, it, kCausal);
-                if (x.n_kv == 0) continue;
-                ok = wait_bar(bar(bars->q_empty), (qc & 1) ^ 1, bars, p.status);
-                if (!ok) break;
-                ptx::mbar_arrive_expect_tx(bar(bars->q_full), kQBytes);
-                ptx::tma_load_3d(sQ, &tm_q, bar(bars->q_full), 0, x.h, x.q_tok0, pol_q);
-                ptx::tma_load_3d(sQ + kChunkBytes, &tm_q, bar(bars->q_full), 64, x.h, x.q_tok0, pol_q);
-                ptx::tma_load_3d(sQ + 2 * kChunkBytes, &tm_qr, bar(bars->q_full), 0, x.h, x.q_tok0, pol_q);
-                ++qc;
-                auto load_k = [&](int j) -> bool {
-                    const int s = kc % kKStages;
-                    if (!wait_bar(bar(bars->k_empty[s]), ((kc / kKStages) & 1) ^ 1, bars, p.status)) return false;
-                    const uint32_t dst = sK + s * kKBytes;
+                if (x.n_max == 0) continue;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (!ok || x.n[t] == 0) continue;
+                    uint32_t &ql = t ? ql1 : ql0;
+                    // Q_t of the previous unit is free once its last S_t MMA has completed.
+                    ok = wait_bar(bar(bars->q_empty[t]), (ql & 1) ^ 1, bars, p.status);
+                    if (!ok) continue;
+                    const uint32_t fb = bar(bars->q_full[t]);
+                    const uint32_t dst = sQ + t * kQTileBytes;
+                    const int tok = x.q_tok0 + t * kBM;
+                    ptx::mbar_arrive_expect_tx(fb, kQTileBytes);
+                    ptx::tma_load_3d(dst, &tm_q, fb, 0, x.h, tok, pol_q);
+                    ptx::tma_load_3d(dst + kChunkBytes, &tm_q, fb, 64, x.h, tok, pol_q);
+                    ptx::tma_load_3d(dst + 2 * kChunkBytes, &tm_qr, fb, 0, x.h, tok, pol_q);
+                    ++ql;
+                }
+                for (int j = 0; j < x.n_max && ok; ++j) {
                     const int tok = x.k_tok0 + j * kBN;
-                    ptx::mbar_arrive_expect_tx(bar(bars->k_full[s]), kKBytes);
-                    ptx::tma_load_3d(dst, &tm_k, bar(bars->k_full[s]), 0, x.kh, tok, pol_kv);
-                    ptx::tma_load_3d(dst + kChunkBytes, &tm_k, bar(bars->k_full[s]), 64, x.kh, tok, pol_kv);
-                    ptx::tma_load_3d(dst + 2 * kChunkBytes, &tm_kr, bar(bars->k_full[s]), 0, x.kh, tok, pol_kv);
-                    ++kc;
-                    return true;
-                };
-                auto load_v = [&](int j) -> bool {
-                    const int s = vc % kVStages;
-                    if (!wait_bar(bar(bars->v_empty[s]), ((vc / kVStages) & 1) ^ 1, bars, p.status)) return false;
-                    const uint32_t dst = sV + s * kVBytes;
-                    const int tok = x.k_tok0 + j * kBN;
-                    ptx::mbar_arrive_expect_tx(bar(bars->v_full[s]), kVBytes);
-                    ptx::tma_load_3d(dst, &tm_v, bar(bars->v_full[s]), 0, x.kh, tok, pol_kv);
-                    ptx::tma_load_3d(dst + kChunkBytes, &tm_v, bar(bars->v_full[s]), 64, x.kh, tok, pol_kv);
-                    ++vc;
-                    return true;
-                };
-                ok = load_k(0);
-                for (int j = 0; j < x.n_kv && ok; ++j) {
-                    if (j + 1 < x.n_kv) ok = load_k(j + 1);
-                    if (ok) ok = load_v(j);
+                    uint32_t dst, fb;
+                    // K_j: nope cols 0-63, nope cols 64-127, rope
+                    if (!(ok = next_chunk(dst, fb))) break;
+                    ptx::tma_load_3d(dst, &tm_k, fb, 0, x.kh, tok, pol_kv);
+                    if (!(ok = next_chunk(dst, fb))) break;
+                    ptx::tma_load_3d(dst, &tm_k, fb, 64, x.kh, tok, pol_kv);
+                    if (!(ok = next_chunk(dst, fb))) break;
+                    ptx::tma_load_3d(dst, &tm_kr, fb, 0, x.kh, tok, pol_kv);
+                    // V_j: keys 0-63, keys 64-127; each chunk holds V cols 0-63 then 64-127
+                    for (int hh = 0; hh < kVChunks && ok; ++hh) {
+                        if (!(ok = next_chunk(dst, fb))) break;
+                        ptx::tma_load_3d(dst, &tm_v, fb, 0, x.kh, tok + hh * 64, pol_kv);
+                        ptx::tma_load_3d(dst + kVHalfBytes, &tm_v, fb, 64, x.kh, tok + hh * 64, pol_kv);
+                    }
                 }
             }
             // Let every copy this thread started land before the block can exit.
-            if (qc) wait_bar(bar(bars->q_full), (qc - 1) & 1, bars, p.status);
-            for (uint32_t s = 0; s < kKStages; ++s) {
-                const uint32_t n = kc / kKStages + (s < kc % kKStages ? 1 : 0);
-                if (n) wait_bar(bar(bars->k_full[s]), (n - 1) & 1, bars, p.status);
+            if (ql0) wait_bar(bar(bars->q_full[0]), (ql0 - 1) & 1, bars, p.status);
+            if (ql1) wait_bar(bar(bars->q_full[1]), (ql1 - 1) & 1, bars, p.status);
+            for (uint32_t s = 0; s < kRing; ++s) {
+                const uint32_t n = rc / kRing + (s < rc % kRing ? 1 : 0);
+                if (n) wait_bar(bar(bars->ch_full[s]), (n - 1) & 1, bars, p.status);
             }
-            for (uint32_t s = 0; s < kVStages; ++s) {
-                const uint32_t n = vc / kVStages + (s < vc % kVStages ? 1 : 0);
-                if (n) wait_bar(bar(bars->v_full[s]), (n - 1) & 1, bars, p.status);
-            }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        } else if (warp == 1 && lane == 0) {
+            // -------------------------------------------------------- MMA issuer
             constexpr bool kBf16 = DType<T>::kBf16;
             constexpr uint32_t idesc_qk = ptx::instr_desc_f16(kBf16, kBM, kBN, false);
             constexpr uint32_t idesc_pv = ptx::instr_desc_f16(kBf16, kBM, kDn, true);
-            uint32_t qc = 0, kc = 0, vc = 0, sc = 0, oe = 0;
+            uint32_t rc = 0;
+            uint32_t qf0 = 0, qf1 = 0, pf0 = 0, pf1 = 0, oe0 = 0, oe1 = 0;
             bool ok = true;
+            auto wait_chunk = [&](uint32_t c) -> bool {
+                return wait_bar(bar(bars->ch_full[c % kRing]), (c / kRing) & 1, bars, p.status);
+            };
+            auto release_chunk = [&](uint32_t c) { ptx::mma_commit(bar(bars->ch_empty[c % kRing])); };
+            // Descriptor low words: K-major Q / K blocks (leading offset unused: 16 B) and
+            // MN-major V blocks (leading offset = distance between the two 64-column halves).
+            constexpr uint32_t kHi = ptx::desc_hi_sw128(1024);
+            const uint32_t q_lo = ptx::desc_lo(sQ, 16);
+            const uint32_t ring_k_lo = ptx::desc_lo(sRing, 16);
+            const uint32_t ring_v_lo = ptx::desc_lo(sRing, kVHalfBytes);
+            // S_t = Q_t K^T for the K chunks starting at ring index kc
+            auto issue_s = [&](int t, uint32_t kc) {
+                const uint32_t d = tmem + kTmemS + t * kBN;
+#pragma unroll
+                for (int c = 0; c < kKChunks; ++c) {
+                    const uint32_t a_lo = q_lo + ((t * kQTileBytes + c * kChunkBytes) >> 4);
+                    const uint32_t b_lo = ring_k_lo + ((((kc + c) % kRing) * kChunkBytes) >> 4);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)  // 16 elements = 32 bytes per k-step
+                        ptx::mma_ss_lo(d, a_lo + 2 * k, b_lo + 2 * k, kHi, idesc_qk, (c | k) != 0);
+                }
+                ptx::mma_commit(bar(bars->s_full[t]));
+            };
+            // O_t (+)= P_t V for the V chunks starting at ring index vc
+            auto issue_pv = [&](int t, uint32_t vc, bool accumulate) {
+                const uint32_t d = tmem + kTmemO + t * kDn;
+                const uint32_t pa = tmem + kTmemS + t * kBN + kTmemPOff;
+#pragma unroll
+                for (int c = 0; c < kVChunks; ++c) {
+                    const uint32_t b_lo = ring_v_lo + ((((vc + c) % kRing) * kChunkBytes) >> 4);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)  // 16 keys x 128 B = 2048 B per k-step
+                        ptx::mma_ts_lo(d, pa + (c * 4 + k) * 8, b_lo + k * 128, kHi, idesc_pv,
+                                       (accumulate || c > 0 || k > 0) ? 1u : 0u);
+                }
+            };
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const WorkItem x = decode_item(p, it, kCausal);
-                if (x.n_kv == 0) continue;
-                ok = wait_bar(bar(bars->q_full), qc & 1, bars, p.status);
+                if (x.n_max == 0) continue;
+                if (x.n[0]) ok = wait_bar(bar(bars->q_full[0]), qf0++ & 1, bars, p.status);
+                if (ok && x.n[1]) ok = wait_bar(bar(bars->q_full[1]), qf1++ & 1, bars, p.status);
                 if (!ok) break;
-                ++qc;
+                // key tile j uses ring chunks K: rc + 5j + {0,1,2}, V: rc + 5j + {3,4}
+                ok = wait_chunk(rc) && wait_chunk(rc + 1) && wait_chunk(rc + 2);
+                if (!ok) break;
                 ptx::tc_fence_after();
-                for (int j = 0; j <= x.n_kv && ok; ++j) {
-                    if (j < x.n_kv) {
-                        // S_j = Q K_j^T over 192 channels: 2 nope chunks + 1 rope chunk, 4 k-steps each
-                        const int ks = kc % kKStages;
-                        const uint32_t sidx = sc + j, sb = sidx & 1;
-                        ok = wait_bar(bar(bars->k_full[ks]), (kc / kKStages) & 1, bars, p.status) &&
-                             wait_bar(bar(bars->s_empty[sb]), ((sidx >> 1) & 1) ^ 1, bars, p.status);
-                        if (!ok) break;
-                        ptx::tc_fence_after();
-                        const uint32_t d = tmem + kTmemS + sb * kBN;
-                        const uint32_t kbase = sK + ks * kKBytes;
 #pragma unroll
-                        for (int c = 0; c < 3; ++c) {
+                for (int t = 0; t < 2; ++t)
+                    if (x.n[t] > 0) {
+                        issue_s(t, rc);
+                        if (x.n[t] == 1) ptx::mma_commit(bar(bars->q_empty[t]));
+                    }
+                for (int c = 0; c < kKChunks; ++c) release_chunk(rc + c);
+                for (int j = 0; j < x.n_max && ok; ++j) {
+                    const uint32_t kc = rc + 5 * j, vc = kc + 3, kn = kc + 5;
+                    bool v_ready = false, k_next_ready = false;
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const uint64_t a = ptx::smem_desc_sw128(sQ + c * kChunkBytes + k * 32, 16, 1024);
-                                const uint64_t b = ptx::smem_desc_sw128(kbase + c * kChunkBytes + k * 32, 16, 1024);
-                                ptx::mma_ss(d, a, b, idesc_qk, (c | k) != 0);
+                    for (int t = 0; t < 2; ++t) {
+                        if (ok && j < x.n[t]) {
+                            uint32_t &pf = t ? pf1 : pf0;
+                            uint32_t &oe = t ? oe1 : oe0;
+                            ok = wait_bar(bar(bars->p_full[t]), pf++ & 1, bars, p.status);
+                            if (ok && !v_ready) {
+                                ok = wait_chunk(vc) && wait_chunk(vc + 1);
+                                v_ready = true;
+                            }
+                            if (ok && j == 0) ok = wait_bar(bar(bars->o_empty[t]), (oe++ & 1) ^ 1, bars, p.status);
+                            if (ok) {
+                                ptx::tc_fence_after();
+                                issue_pv(t, vc, j > 0);
+                                if (j == x.n[t] - 1) ptx::mma_commit(bar(bars->o_full[t]));
                             }
                         }
-                        ptx::mma_commit(bar(bars->k_empty[ks]));
-                        ++kc;
-                        ptx::mma_commit(bar(bars->s_full[sb]));
-                        if (j == x.n_kv - 1) ptx::mma_commit(bar(bars->q_empty));
-                    }
-                    if (j >= 1) {
-                        // O += P_{j-1} V_{j-1}: P from TMEM (A operand), V from shared memory (MN-major B)
-                        const int t = j - 1;
-                        const uint32_t pidx = sc + t, pb = pidx & 1;
-                        const int vs = vc % kVStages;
-                        ok = wait_bar(bar(bars->p_full[pb]), (pidx >> 1) & 1, bars, p.status) &&
-                             wait_bar(bar(bars->v_full[vs]), (vc / kVStages) & 1, bars, p.status);
-                        if (ok && t == 0) {
-                            ok = wait_bar(bar(bars->o_empty), (oe & 1) ^ 1, bars, p.status);
-                            ++oe;
+                        if (ok && j + 1 < x.n[t]) {
+                            if (!k_next_ready) {
+                                ok = wait_chunk(kn) && wait_chunk(kn + 1) && wait_chunk(kn + 2);
+                                k_next_ready = true;
+                                if (ok) ptx::tc_fence_after();
+                            }
+                            if (ok) {
+                                issue_s(t, kn);
+                                if (j + 2 == x.n[t]) ptx::mma_commit(bar(bars->q_empty[t]));  // last S_t of the unit
+                            }
                         }
-                        if (!ok) break;
-                        ptx::tc_fence_after();
-                        const uint32_t vbase = sV + vs * kVBytes;
-#pragma unroll
-                        for (int k = 0; k < kBN / 16; ++k) {
-                            const uint64_t b = ptx::smem_desc_sw128(vbase + k * 16 * 128, kChunkBytes, 1024);
-                            ptx::mma_ts(tmem + kTmemO, tmem + kTmemP + pb * (kBN / 2) + k * 8, b, idesc_pv,
-                                        (t > 0 || k > 0) ? 1u : 0u);
-                        }
-                        ptx::mma_commit(bar(bars->v_empty[vs]));
-                        ++vc;
-                        ptx::mma_commit(bar(bars->o_done));
                     }
+                    if (!ok) break;
+                    release_chunk(vc);
+                    release_chunk(vc + 1);
+                    if (j + 1 < x.n_max)
+                        for (int c = 0; c < kKChunks; ++c) release_chunk(kn + c);
                 }
-                sc += x.n_kv;
+                if (!ok) break;
+                rc += 5 * x.n_max;
             }
             // Drain: wait until every MMA this thread issued has completed.
             ptx::mma_commit(bar(bars->drain));
             wait_bar(bar(bars->drain), 0, bars, p.status);
         }
     } else {
+        ptx::regs_inc<kRegsHigh>();
         // ------------------------------------------------------------ softmax + epilogue
-        const int wq = warp & 3;           // TMEM lane quarter this warp may access
-        const int row = wq * 32 + lane;    // query row within the tile
+        const int t = (warp >> 2) - 1;   // query tile of this warpgroup
+        const int wq = warp & 3;         // TMEM lane quarter this warp may access
+        const int row = wq * 32 + lane;  // query row within the tile
         const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_addr + kTmemS + t * kBN;
+        const uint32_t tO = tmem + lane_addr + kTmemO + t * kDn;
         const float sl2 = p.scale_log2;
-        uint32_t sc = 0, od = 0;
+        uint32_t sf = 0, of = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
             const WorkItem x = decode_item(p, it, kCausal);
-            const bool row_valid = row < x.rows;
-            T *orow = reinterpret_cast<T *>(p.out) + (long long)(x.q_tok0 + row) * p.out_st +
+            const int n_t = t ? x.n[1] : x.n[0];
+            const bool row_valid = row < (t ? x.rows[1] : x.rows[0]);
+            const int i = x.u0 + t * kBM + row;  // query row within the sequence
+            T *orow = reinterpret_cast<T *>(p.out) + (long long)(x.q_tok0 + t * kBM + row) * p.out_st +
                       (long long)x.h * p.out_sh;
-            if (x.n_kv == 0) {
+            if (n_t == 0) {
                 if (row_valid) {
-                    uint4 z = make_uint4(0, 0, 0, 0);
+                    const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int c = 0; c < kDn * 2 / 16; ++c) reinterpret_cast<uint4 *>(orow)[c] = z;
                 }
                 continue;
             }
-            const int i = x.q0 + row;
             const int lim_row = kCausal ? min(i + x.off + 1, x.lk) : x.lk;  // keys [0, lim_row) visible
+            const int tile_q0 = x.u0 + t * kBM;
             float m_run = -INFINITY, l_run = 0.f;
-            for (int j = 0; j < x.n_kv; ++j) {
-                const uint32_t sidx = sc + j, sb = sidx & 1;
-                ok = wait_bar(bar(bars->s_full[sb]), (sidx >> 1) & 1, bars, p.status);
+            for (int j = 0; j < n_t; ++j) {
+                ok = wait_bar(bar(bars->s_full[t]), sf & 1, bars, p.status);
+                ++sf;
                 if (!ok) break;
                 ptx::tc_fence_after();
                 float s[kBN];
                 {
                     uint32_t r0[32], r1[32], r2[32], r3[32];
-                    const uint32_t sa = tmem + lane_addr + kTmemS + sb * kBN;
-                    ptx::tmem_ld32(sa, r0);
-                    ptx::tmem_ld32(sa + 32, r1);
-                    ptx::tmem_ld32(sa + 64, r2);
-                    ptx::tmem_ld32(sa + 96, r3);
+                    ptx::tmem_ld32(tS, r0);
+                    ptx::tmem_ld32(tS + 32, r1);
+                    ptx::tmem_ld32(tS + 64, r2);
+                    ptx::tmem_ld32(tS + 96, r3);
                     ptx::tmem_wait_ld_dep(r0);
                     ptx::tmem_wait_ld_dep(r1);
                     ptx::tmem_wait_ld_dep(r2);
@@ -542,12 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         s[96 + e] = __uint_as_float(r3[e]);
                     }
                 }
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(bar(bars->s_empty[sb]));
-
                 const int kv0 = j * kBN;
-                const bool tile_masked =
-                    (kv0 + kBN > x.lk) || (kCausal && kv0 + kBN - 1 > x.q0 + x.off);
+                const bool tile_masked = (kv0 + kBN > x.lk) || (kCausal && kv0 + kBN - 1 > tile_q0 + x.off);
                 float m_tile;
                 if (kPositiveScale) {
                     if (tile_masked) {
@@ -569,66 +626,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_run = m_tile;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                uint32_t pk[kBN / 2];
                 float psum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
-                for (int c = 0; c < kBN; c += 2) {
-                    float p0, p1;
-                    if (kPositiveScale) {
-                        p0 = ptx::ex2(fmaf(s[c], sl2, -m_use));
-                        p1 = ptx::ex2(fmaf(s[c + 1], sl2, -m_use));
-                    } else {
-                        p0 = ptx::ex2(s[c] - m_use);
-                        p1 = ptx::ex2(s[c + 1] - m_use);
-                    }
-                    psum[(c / 2) & 7] += p0 + p1;
-                    pk[c / 2] = DType<T>::pack(p0, p1);
-                }
-                if (j > 0) {
-                    // O holds P_{j-1} V_{j-1} once o_done completes; P buffer sb is free again.
-                    ok = wait_bar(bar(bars->o_done), od & 1, bars, p.status);
-                    ++od;
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t pk[32];
 #pragma unroll
-                        for (int c = 0; c < kDn / 32; ++c) {
-                            uint32_t r[32];
-                            const uint32_t taddr = tmem + lane_addr + kTmemO + c * 32;
-                            ptx::tmem_ld32(taddr, r);
-                            ptx::tmem_wait_ld_dep(r);
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                            ptx::tmem_st32(taddr, r);
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = h2 * 64 + 2 * e;
+                        float p0, p1;
+                        if (kPositiveScale) {
+                            p0 = ptx::ex2(fmaf(s[c], sl2, -m_use));
+                            p1 = ptx::ex2(fmaf(s[c + 1], sl2, -m_use));
+                        } else {
+                            p0 = ptx::ex2(s[c] - m_use);
+                            p1 = ptx::ex2(s[c + 1] - m_use);
                         }
+                        psum[e & 7] += p0 + p1;
+                        pk[e] = DType<T>::pack(p0, p1);
                     }
+                    ptx::tmem_st32(tS + kTmemPOff + h2 * 32, pk);
                 }
-                const float rowsum = ((psum[0] + psum[1]) + (psum[2] + psum[3])) +
-                                     ((psum[4] + psum[5]) + (psum[6] + psum[7]));
-                l_run = l_run * alpha + rowsum;
+                // O_t holds P(j-1) V(j-1) already (the MMAs behind S_t(j) have completed);
+                // rescale it before PV_t(j) may start (S is dead here: fewer live registers).
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                for (int c = 0; c < kBN / 2 / 32; ++c) {
-                    uint32_t r[32];
+                    for (int c = 0; c < kDn / 32; ++c) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(tO + c * 32, r);
+                        ptx::tmem_wait_ld_dep(r);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = pk[c * 32 + e];
-                    ptx::tmem_st32(tmem + lane_addr + kTmemP + sb * (kBN / 2) + c * 32, r);
+                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        ptx::tmem_st32(tO + c * 32, r);
+                    }
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(bar(bars->p_full[sb]));
+                ptx::mbar_arrive(bar(bars->p_full[t]));
+                const float rowsum = ((psum[0] + psum[1]) + (psum[2] + psum[3])) +
+                                     ((psum[4] + psum[5]) + (psum[6] + psum[7]));
+                l_run = l_run * alpha + rowsum;
             }
             if (!ok) break;
-            sc += x.n_kv;
             // Epilogue: O / l -> 16-bit, one 256-byte row per thread.
-            ok = wait_bar(bar(bars->o_done), od & 1, bars, p.status);
-            ++od;
+            ok = wait_bar(bar(bars->o_full[t]), of & 1, bars, p.status);
+            ++of;
             if (!ok) break;
             ptx::tc_fence_after();
             const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
             for (int c = 0; c < kDn / 32; ++c) {
                 uint32_t r[32];
-                ptx::tmem_ld32(tmem + lane_addr + kTmemO + c * 32, r);
+                ptx::tmem_ld32(tO + c * 32, r);
                 ptx::tmem_wait_ld_dep(r);
                 uint32_t w[16];
 #pragma unroll
@@ -641,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(bar(bars->o_empty));
+            ptx::mbar_arrive(bar(bars->o_empty[t]));
         }
     }
 
