@@ -65,8 +65,8 @@ constexpr uint32_t kTmemPOff = 64;  // P_t at S_t + 64
 constexpr uint32_t kTmemCols = 512;
 
 constexpr int kThreads = 384;  // warpgroup 0: TMA (warp 0), MMA (warp 1); warpgroups 1, 2: softmax of tiles 0, 1
-constexpr int kRegsLow = 56;
-constexpr int kRegsHigh = 224;
+constexpr int kRegsLow = 104;
+constexpr int kRegsHigh = 200;
 static_assert(kRegsLow * 128 + kRegsHigh * 256 <= 65536 / kThreads / 8 * 8 * kThreads,
               "register split exceeds the launch's register file share");
 
@@ -164,6 +164,13 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Barriers
             }
         }
     }
+}
+
+// The same wait for a whole warp: every lane polls, and the result is made
+// warp-uniform so that all lanes take the same path afterwards.
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, Barriers *bars, int *status) {
+    const bool ok = wait_bar(bar, parity, bars, status);
+    return __all_sync(0xffffffffu, ok);
 }
 
 template <typename T>
@@ -443,67 +450,93 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t n = rc / kRing + (s < rc % kRing ? 1 : 0);
                 if (n) wait_bar(bar(bars->ch_full[s]), (n - 1) & 1, bars, p.status);
             }
-        } else if (warp == 1 && lane == 0) {
+        } else if (warp == 1) {
             // -------------------------------------------------------- MMA issuer
+            // The whole warp runs this loop (all its state is warp-uniform); one
+            // elected lane issues each batch of MMAs and each commit.
             constexpr bool kBf16 = DType<T>::kBf16;
-            constexpr uint32_t idesc_qk = ptx::instr_desc_f16(kBf16, kBM, kBN, false);
-            constexpr uint32_t idesc_pv = ptx::instr_desc_f16(kBf16, kBM, kDn, true);
+            constexpr uint32_t kIdQK = ptx::instr_desc_f16(kBf16, kBM, kBN, false);
+            constexpr uint32_t kIdPV = ptx::instr_desc_f16(kBf16, kBM, kDn, true);
+            constexpr uint32_t kHi = ptx::desc_hi_sw128(1024);
+            // Descriptor low words: K-major Q / K blocks (leading offset unused: 16 B) and
+            // MN-major V blocks (leading offset = distance between the two 64-column halves).
+            const uint32_t q_lo = ptx::desc_lo(sQ, 16);
+            const uint32_t ring_k_lo = ptx::desc_lo(sRing, 16);
+            const uint32_t ring_v_lo = ptx::desc_lo(sRing, kVHalfBytes);
             uint32_t rc = 0;
             uint32_t qf0 = 0, qf1 = 0, pf0 = 0, pf1 = 0, oe0 = 0, oe1 = 0;
             bool ok = true;
             auto wait_chunk = [&](uint32_t c) -> bool {
-                return wait_bar(bar(bars->ch_full[c % kRing]), (c / kRing) & 1, bars, p.status);
+                return wait_bar_warp(bar(bars->ch_full[c % kRing]), (c / kRing) & 1, bars, p.status);
             };
-            auto release_chunk = [&](uint32_t c) { ptx::mma_commit(bar(bars->ch_empty[c % kRing])); };
-            // Descriptor low words: K-major Q / K blocks (leading offset unused: 16 B) and
-            // MN-major V blocks (leading offset = distance between the two 64-column halves).
-            constexpr uint32_t kHi = ptx::desc_hi_sw128(1024);
-            const uint32_t q_lo = ptx::desc_lo(sQ, 16);
-            const uint32_t ring_k_lo = ptx::desc_lo(sRing, 16);
-            const uint32_t ring_v_lo = ptx::desc_lo(sRing, kVHalfBytes);
+            auto commit = [&](uint64_t &b) {
+                if (ptx::elect_one()) ptx::mma_commit(bar(b));
+                __syncwarp();
+            };
             // S_t = Q_t K^T for the K chunks starting at ring index kc
             auto issue_s = [&](int t, uint32_t kc) {
                 const uint32_t d = tmem + kTmemS + t * kBN;
-#pragma unroll
-                for (int c = 0; c < kKChunks; ++c) {
-                    const uint32_t a_lo = q_lo + ((t * kQTileBytes + c * kChunkBytes) >> 4);
-                    const uint32_t b_lo = ring_k_lo + ((((kc + c) % kRing) * kChunkBytes) >> 4);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)  // 16 elements = 32 bytes per k-step
-                        ptx::mma_ss_lo(d, a_lo + 2 * k, b_lo + 2 * k, kHi, idesc_qk, (c | k) != 0);
+                const uint32_t a0 = q_lo + ((t * kQTileBytes) >> 4);
+                const uint32_t b0 = ring_k_lo + (((kc + 0) % kRing) * (kChunkBytes >> 4));
+                const uint32_t b1 = ring_k_lo + (((kc + 1) % kRing) * (kChunkBytes >> 4));
+                const uint32_t b2 = ring_k_lo + (((kc + 2) % kRing) * (kChunkBytes >> 4));
+                if (ptx::elect_one()) {
+                    constexpr uint32_t kC = kChunkBytes >> 4;  // one chunk, in descriptor units
+                    ptx::mma_ss_lo<kHi, kIdQK, 0>(d, a0 + 0, b0 + 0);  // 16 elements = 2 units per k-step
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + 2, b0 + 2);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + 4, b0 + 4);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + 6, b0 + 6);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + kC + 0, b1 + 0);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + kC + 2, b1 + 2);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + kC + 4, b1 + 4);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + kC + 6, b1 + 6);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + 2 * kC + 0, b2 + 0);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + 2 * kC + 2, b2 + 2);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + 2 * kC + 4, b2 + 4);
+                    ptx::mma_ss_lo<kHi, kIdQK, 1>(d, a0 + 2 * kC + 6, b2 + 6);
+                    ptx::mma_commit(bar(bars->s_full[t]));
                 }
-                ptx::mma_commit(bar(bars->s_full[t]));
+                __syncwarp();
             };
             // O_t (+)= P_t V for the V chunks starting at ring index vc
             auto issue_pv = [&](int t, uint32_t vc, bool accumulate) {
                 const uint32_t d = tmem + kTmemO + t * kDn;
                 const uint32_t pa = tmem + kTmemS + t * kBN + kTmemPOff;
-#pragma unroll
-                for (int c = 0; c < kVChunks; ++c) {
-                    const uint32_t b_lo = ring_v_lo + ((((vc + c) % kRing) * kChunkBytes) >> 4);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)  // 16 keys x 128 B = 2048 B per k-step
-                        ptx::mma_ts_lo(d, pa + (c * 4 + k) * 8, b_lo + k * 128, kHi, idesc_pv,
-                                       (accumulate || c > 0 || k > 0) ? 1u : 0u);
+                const uint32_t v0 = ring_v_lo + (((vc + 0) % kRing) * (kChunkBytes >> 4));
+                const uint32_t v1 = ring_v_lo + (((vc + 1) % kRing) * (kChunkBytes >> 4));
+                if (ptx::elect_one()) {
+                    // 16 keys x 128 B = 2048 B = 128 units per k-step; P advances 8 columns per k-step
+                    if (accumulate) ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa, v0);
+                    else ptx::mma_ts_lo<kHi, kIdPV, 0>(d, pa, v0);
+                    ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa + 8, v0 + 128);
+                    ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa + 16, v0 + 256);
+                    ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa + 24, v0 + 384);
+                    ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa + 32, v1);
+                    ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa + 40, v1 + 128);
+                    ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa + 48, v1 + 256);
+                    ptx::mma_ts_lo<kHi, kIdPV, 1>(d, pa + 56, v1 + 384);
                 }
+                __syncwarp();
             };
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const WorkItem x = decode_item(p, it, kCausal);
                 if (x.n_max == 0) continue;
-                if (x.n[0]) ok = wait_bar(bar(bars->q_full[0]), qf0++ & 1, bars, p.status);
-                if (ok && x.n[1]) ok = wait_bar(bar(bars->q_full[1]), qf1++ & 1, bars, p.status);
+                if (x.n[0]) ok = wait_bar_warp(bar(bars->q_full[0]), qf0++ & 1, bars, p.status);
+                if (ok && x.n[1]) ok = wait_bar_warp(bar(bars->q_full[1]), qf1++ & 1, bars, p.status);
                 if (!ok) break;
                 // key tile j uses ring chunks K: rc + 5j + {0,1,2}, V: rc + 5j + {3,4}
                 ok = wait_chunk(rc) && wait_chunk(rc + 1) && wait_chunk(rc + 2);
                 if (!ok) break;
                 ptx::tc_fence_after();
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-                    if (x.n[t] > 0) {
-                        issue_s(t, rc);
-                        if (x.n[t] == 1) ptx::mma_commit(bar(bars->q_empty[t]));
-                    }
-                for (int c = 0; c < kKChunks; ++c) release_chunk(rc + c);
+                if (x.n[0] > 0) {
+                    issue_s(0, rc);
+                    if (x.n[0] == 1) commit(bars->q_empty[0]);
+                }
+                if (x.n[1] > 0) {
+                    issue_s(1, rc);
+                    if (x.n[1] == 1) commit(bars->q_empty[1]);
+                }
+                for (int c = 0; c < kKChunks; ++c) commit(bars->ch_empty[(rc + c) % kRing]);
                 for (int j = 0; j < x.n_max && ok; ++j) {
                     const uint32_t kc = rc + 5 * j, vc = kc + 3, kn = kc + 5;
                     bool v_ready = false, k_next_ready = false;
@@ -512,16 +545,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (ok && j < x.n[t]) {
                             uint32_t &pf = t ? pf1 : pf0;
                             uint32_t &oe = t ? oe1 : oe0;
-                            ok = wait_bar(bar(bars->p_full[t]), pf++ & 1, bars, p.status);
+                            ok = wait_bar_warp(bar(bars->p_full[t]), pf++ & 1, bars, p.status);
                             if (ok && !v_ready) {
                                 ok = wait_chunk(vc) && wait_chunk(vc + 1);
                                 v_ready = true;
                             }
-                            if (ok && j == 0) ok = wait_bar(bar(bars->o_empty[t]), (oe++ & 1) ^ 1, bars, p.status);
+                            if (ok && j == 0) ok = wait_bar_warp(bar(bars->o_empty[t]), (oe++ & 1) ^ 1, bars, p.status);
                             if (ok) {
                                 ptx::tc_fence_after();
                                 issue_pv(t, vc, j > 0);
-                                if (j == x.n[t] - 1) ptx::mma_commit(bar(bars->o_full[t]));
+                                if (j == x.n[t] - 1) commit(bars->o_full[t]);
                             }
                         }
                         if (ok && j + 1 < x.n[t]) {
@@ -532,22 +565,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                             if (ok) {
                                 issue_s(t, kn);
-                                if (j + 2 == x.n[t]) ptx::mma_commit(bar(bars->q_empty[t]));  // last S_t of the unit
+                                if (j + 2 == x.n[t]) commit(bars->q_empty[t]);  // last S_t of the unit
                             }
                         }
                     }
                     if (!ok) break;
-                    release_chunk(vc);
-                    release_chunk(vc + 1);
+                    commit(bars->ch_empty[vc % kRing]);
+                    commit(bars->ch_empty[(vc + 1) % kRing]);
                     if (j + 1 < x.n_max)
-                        for (int c = 0; c < kKChunks; ++c) release_chunk(kn + c);
+                        for (int c = 0; c < kKChunks; ++c) commit(bars->ch_empty[(kn + c) % kRing]);
                 }
                 if (!ok) break;
                 rc += 5 * x.n_max;
             }
-            // Drain: wait until every MMA this thread issued has completed.
-            ptx::mma_commit(bar(bars->drain));
-            wait_bar(bar(bars->drain), 0, bars, p.status);
+            // Drain: wait until every MMA this warp issued has completed.
+            commit(bars->drain);
+            wait_bar_warp(bar(bars->drain), 0, bars, p.status);
         }
     } else {
         ptx::regs_inc<kRegsHigh>();

@@ -119,27 +119,41 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 }
 
 // Same MMAs with the two smem descriptors given as (low word, shared high
-// word): only the start address / leading offset change between k-steps.
-__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t desc_hi,
-                                          uint32_t idesc, uint32_t accumulate) {
+// word) -- only the start address / leading offset change between k-steps --
+// and the accumulate flag, high word and instruction descriptor as
+// compile-time immediates, so the issuing thread spends almost nothing
+// between consecutive MMAs.
+template <uint32_t kHi, uint32_t kIdesc, int kAcc>
+__device__ __forceinline__ void mma_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
         "mov.b64 da, {%1, %3};\n\t"
         "mov.b64 db, {%2, %3};\n\t"
         "setp.ne.b32 p, %5, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(desc_hi), "r"(idesc), "r"(accumulate)
+        "r"(a_lo), "r"(b_lo), "n"(kHi), "n"(kIdesc), "n"(kAcc)
         : "memory");
 }
-__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t desc_hi,
-                                          uint32_t idesc, uint32_t accumulate) {
+template <uint32_t kHi, uint32_t kIdesc, int kAcc>
+__device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
         "mov.b64 db, {%2, %3};\n\t"
         "setp.ne.b32 p, %5, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(desc_hi), "r"(idesc), "r"(accumulate)
+        "r"(a_tmem), "r"(b_lo), "n"(kHi), "n"(kIdesc), "n"(kAcc)
         : "memory");
+}
+
+// One lane of the (fully active) warp is chosen; true on that lane only.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, e;\n\t}"
+        : "=r"(p));
+    return p != 0;
 }
 
 // Arrive once on the mbarrier when every tcgen05 operation issued so far by
