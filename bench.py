@@ -297,6 +297,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling aid: scale head_num and kv_head_num down to this many query heads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -304,6 +306,10 @@ def main():
     from mla_prefill_attention_varlen_b200 import workloads as W
 
     wl = W.get(args.workload)
+    if args.heads:
+        g = wl.head_num // wl.kv_head_num
+        wl.head_num, wl.kv_head_num = args.heads, max(1, args.heads // g)
+        wl.name += "_h%d" % args.heads
     if args.impl == "reference":
         return reference_arm(args, wl)
 

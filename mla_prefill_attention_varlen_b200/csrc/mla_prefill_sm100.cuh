@@ -126,11 +126,17 @@ struct WorkItem {
     int n_max;
 };
 
-__device__ __forceinline__ WorkItem decode_item(const Params &p, int it, bool causal) {
-    const int u = it / p.head_num;
+// Work items are ordered kv-head-major: for each kv head, its units in the
+// sorted (longest-first) order, and for each unit the query heads of the group.
+// Concurrently running CTAs then read the same kv head's K/V (L2 reuse), and the
+// last items of the grid are the cheapest units.
+__device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num_units, bool causal) {
+    const int per_kh = num_units * p.group;
     WorkItem x;
-    x.h = it - u * p.head_num;
-    x.kh = x.h / p.group;
+    x.kh = it / per_kh;
+    const int rem = it - x.kh * per_kh;
+    const int u = rem / p.group;
+    x.h = x.kh * p.group + (rem - u * p.group);
     const int2 bm = p.units[u];
     const int4 s = p.seq_info[bm.x];
     x.u0 = bm.y * kUnitRows;
@@ -381,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    const int n_items = *p.num_units * p.head_num;
+    const int num_units = *p.num_units;
+    const int n_items = num_units * p.head_num;
 
     if (warp < 4) {
         ptx::regs_dec<kRegsLow>();
@@ -407,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                const WorkItem x = decode_item(p, it, kCausal);
+                const WorkItem x = decode_item(p, it, num_units, kCausal);
                 if (x.n_max == 0) continue;
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
@@ -519,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
             };
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                const WorkItem x = decode_item(p, it, kCausal);
+                const WorkItem x = decode_item(p, it, num_units, kCausal);
                 if (x.n_max == 0) continue;
                 if (x.n[0]) ok = wait_bar_warp(bar(bars->q_full[0]), qf0++ & 1, bars, p.status);
                 if (ok && x.n[1]) ok = wait_bar_warp(bar(bars->q_full[1]), qf1++ & 1, bars, p.status);
@@ -595,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sf = 0, of = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const WorkItem x = decode_item(p, it, kCausal);
+            const WorkItem x = decode_item(p, it, num_units, kCausal);
             const int n_t = t ? x.n[1] : x.n[0];
             const bool row_valid = row < (t ? x.rows[1] : x.rows[0]);
             const int i = x.u0 + t * kBM + row;  // query row within the sequence
