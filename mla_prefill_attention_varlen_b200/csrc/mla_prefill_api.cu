@@ -255,6 +255,7 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
 
     uint8_t *ws = static_cast<uint8_t *>(ds->ws);
     int *num_units = reinterpret_cast<int *>(ws + lay.num_units);
+    int *work_counter = num_units + 1;  // second word of the 16-byte header
     int4 *seq_info = reinterpret_cast<int4 *>(ws + lay.seq_info);
     int *unit_off = reinterpret_cast<int *>(ws + lay.unit_off);
     int *hist = reinterpret_cast<int *>(ws + lay.hist);
@@ -263,13 +264,15 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
 
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
         static_cast<const int *>(q_seqlen->data), static_cast<const int *>(kv_seqlen->data), static_cast<int>(batch),
-        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, ds->status);
+        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
+        ds->status);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
     mla::Params p;
     p.seq_info = seq_info;
     p.units = units;
     p.num_units = num_units;
+    p.work_counter = work_counter;
     p.status = ds->status;
     p.out = vo.data;
     p.out_st = vo.st_tok;

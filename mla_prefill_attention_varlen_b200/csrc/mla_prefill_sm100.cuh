@@ -52,6 +52,7 @@ constexpr int kRing = 8;                      // ring chunks
 constexpr int kKChunks = 3;                   // Kn lo | Kn hi | Kr            (128 keys each)
 constexpr int kVChunks = 2;                   // keys 0-63 | keys 64-127      (V cols 0-63 then 64-127 inside)
 constexpr int kVHalfBytes = 8192;             // 64 keys x 64 V columns
+constexpr int kSched = 4;                     // depth of the work-item hand-off ring
 
 constexpr int kSmemQ = 0;
 constexpr int kSmemRing = kSmemQ + 2 * kQTileBytes;
@@ -80,6 +81,7 @@ struct Params {
     const int4 *seq_info;  // per sequence {cq, ck, lq, lk} after clamping
     const int2 *units;     // (sequence, 256-row unit) pairs, most key tiles first
     const int *num_units;  // number of valid entries in units
+    int *work_counter;     // dynamic work counter (zeroed by the plan kernel)
     int *status;           // sticky device status word
     void *out;
     long long out_st, out_sh;  // token / head strides of out, elements
@@ -93,7 +95,9 @@ struct Barriers {
     uint64_t ch_full[kRing], ch_empty[kRing];
     uint64_t s_full[2], p_full[2];
     uint64_t o_full[2], o_empty[2];
+    uint64_t sched_full[kSched], sched_empty[kSched];
     uint64_t drain;
+    int sched_item[kSched];
     uint32_t tmem_base;
     int abort;
 };
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
                                                                 long long t_q, long long t_k, int causal,
                                                                 int4 *seq_info, int *unit_off, int *hist,
                                                                 int hist_len, int2 *units, int *num_units,
-                                                                int *status) {
+                                                                int *work_counter, int *status) {
     __shared__ long long warp_sums[32];
     __shared__ int bad;
     if (threadIdx.x == 0) bad = 0;
@@ -320,6 +324,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
     }
     if (threadIdx.x == 0) {
         *num_units = total;
+        *work_counter = 0;
         if (bad) atomicCAS(status, 0, kStatusSeqlen);
     }
 }
@@ -374,6 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(bars->ch_full[c]), 1);
             ptx::mbar_init(bar(bars->ch_empty[c]), 1);
         }
+        for (int i = 0; i < kSched; ++i) {
+            ptx::mbar_init(bar(bars->sched_full[i]), 1);
+            ptx::mbar_init(bar(bars->sched_empty[i]), 1 + 8);  // the MMA warp + each softmax warp
+        }
         ptx::mbar_init(bar(bars->drain), 1);
         bars->abort = 0;
         ptx::fence_mbar_init();
@@ -413,7 +422,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++rc;
                 return true;
             };
-            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            // Dynamic scheduling: the first item is blockIdx.x, later ones come from a global
+            // counter; each claimed item index (or -1 at the end) is handed to the MMA and
+            // softmax warps through a small ring in shared memory.
+            uint32_t sc = 0;
+            int next = blockIdx.x < n_items ? (int)blockIdx.x : -1;
+            while (ok) {
+                const int it = next;
+                const uint32_t slot = sc % kSched;
+                ok = wait_bar(bar(bars->sched_empty[slot]), ((sc / kSched) & 1) ^ 1, bars, p.status);
+                if (!ok) break;
+                *reinterpret_cast<volatile int *>(&bars->sched_item[slot]) = it;
+                ptx::mbar_arrive(bar(bars->sched_full[slot]));
+                ++sc;
+                if (it < 0) break;
+                next = (int)gridDim.x + atomicAdd(p.work_counter, 1);
+                if (next >= n_items) next = -1;
                 const WorkItem x = decode_item(p, it, num_units, kCausal);
                 if (x.n_max == 0) continue;
 #pragma unroll
@@ -525,7 +549,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             };
-            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            uint32_t ss = 0;
+            while (ok) {
+                const uint32_t slot = ss % kSched;
+                ok = wait_bar_warp(bar(bars->sched_full[slot]), (ss / kSched) & 1, bars, p.status);
+                if (!ok) break;
+                const int it = *reinterpret_cast<volatile int *>(&bars->sched_item[slot]);
+                __syncwarp();
+                if (ptx::elect_one()) ptx::mbar_arrive(bar(bars->sched_empty[slot]));
+                __syncwarp();
+                ++ss;
+                if (it < 0) break;
                 const WorkItem x = decode_item(p, it, num_units, kCausal);
                 if (x.n_max == 0) continue;
                 if (x.n[0]) ok = wait_bar_warp(bar(bars->q_full[0]), qf0++ & 1, bars, p.status);
@@ -601,7 +635,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl2 = p.scale_log2;
         uint32_t sf = 0, of = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        uint32_t ss = 0;
+        while (ok) {
+            const uint32_t slot = ss % kSched;
+            ok = wait_bar_warp(bar(bars->sched_full[slot]), (ss / kSched) & 1, bars, p.status);
+            if (!ok) break;
+            const int it = *reinterpret_cast<volatile int *>(&bars->sched_item[slot]);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(bars->sched_empty[slot]));
+            ++ss;
+            if (it < 0) break;
             const WorkItem x = decode_item(p, it, num_units, kCausal);
             const int n_t = t ? x.n[1] : x.n[0];
             const bool row_valid = row < (t ? x.rows[1] : x.rows[0]);
@@ -620,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int tile_q0 = x.u0 + t * kBM;
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < n_t; ++j) {
-                ok = wait_bar(bar(bars->s_full[t]), sf & 1, bars, p.status);
+                ok = wait_bar_warp(bar(bars->s_full[t]), sf & 1, bars, p.status);
                 ++sf;
                 if (!ok) break;
                 ptx::tc_fence_after();
@@ -708,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             // Epilogue: O / l -> 16-bit, one 256-byte row per thread.
-            ok = wait_bar(bar(bars->o_full[t]), of & 1, bars, p.status);
+            ok = wait_bar_warp(bar(bars->o_full[t]), of & 1, bars, p.status);
             ++of;
             if (!ok) break;
             ptx::tc_fence_after();
