@@ -125,6 +125,46 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
  */
 int mla_prefill_device_status(mla_stream_t stream, int *status);
 
+/*
+ * mla_prefill_noalloc -- the same operation, arguments, validation, layouts
+ * and results as mla_prefill, for callers that cannot allocate device memory.
+ * (The MLA Prefill page has no counterpart: its two-phase API hands the
+ * operator a caller-allocated workspace; this entry point needs none.)
+ *
+ * Who needs it: a caller that has already reserved (nearly) all of the GPU's
+ * memory for its own pool, as serving engines do at start-up, so that a
+ * cudaMalloc from a library would fail or eat into that pool; and a caller
+ * on a latency-critical path that must never call cudaMalloc, because a first
+ * allocation or a workspace growth can stall on the driver at an arbitrary
+ * moment.  mla_prefill allocates its per-GPU workspace and status word on first
+ * use (and grows the workspace when a larger problem arrives); this entry point
+ * calls no cudaMalloc / cudaFree or other allocating routine.
+ *
+ * Scratch: one static 1 MiB device array per GPU that loads the library
+ * (reserved for the life of the process).  The problem must fit in it: the
+ * plan workspace, 16 + 16*batch + 4*(batch+1) + 4*(ceil(T_k/128)+2) +
+ * 8*(ceil(T_q/256)+batch) bytes with each part rounded up to 256 bytes, must
+ * not exceed 1 MiB - 256 bytes (for example batch <= 8192 with T_q, T_k <= 1M
+ * tokens fits).  A larger problem is rejected on the host with
+ * MLA_ERR_UNSUPPORTED before anything is launched.
+ *
+ * The first call on a GPU does a one-time set-up with that GPU current (it
+ * looks up the array's device address, the SM count and the tensor-map
+ * encoder); make that first call before any stream capture.  All calls on a
+ * GPU share the one array: calls whose work overlaps on that GPU (different
+ * streams, or host threads without ordering) race and may produce wrong
+ * results; order them on one stream.  Nothing in the array needs clearing
+ * between calls: each call rewrites every entry it later reads.
+ * Inconsistent seqlens are clamped exactly as in mla_prefill (no out-of-bounds
+ * access), but the status word they set lives in the static array and is not
+ * reported: mla_prefill_device_status() covers mla_prefill calls only.
+ * Returns MLA_OK or an mla_status error code, like mla_prefill.
+ */
+int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
+                        const mla_tensor *k_rope, const mla_tensor *v, const mla_tensor *q_seqlen,
+                        const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num, float qk_scale,
+                        mla_tensor *out, mla_stream_t stream);
+
 /* A static, human-readable name for a status code (never NULL). */
 const char *mla_status_string(int status);
 

@@ -59,6 +59,9 @@ def load_library(path=None):
     lib.mla_prefill_device_status.restype = ctypes.c_int
     lib.mla_status_string.argtypes = [ctypes.c_int]
     lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_prefill_noalloc.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_float, T, ctypes.c_void_p]
+    lib.mla_prefill_noalloc.restype = ctypes.c_int
     lib.mla_prefill_set_profile_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.mla_prefill_set_profile_events.restype = ctypes.c_int
     lib.mla_prefill_version.argtypes = []
@@ -119,6 +122,21 @@ def mla_prefill(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_nu
                          float(qk_scale), ctypes.byref(descs[7]), _stream_handle(stream, q.device))
     if rc != 0:
         raise MlaError(rc)
+    return out
+
+
+def mla_prefill_noalloc(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num,
+                        qk_scale, out, stream=None):
+    """Call the C ABI ``mla_prefill_noalloc``: same as ``mla_prefill`` but the
+    library allocates no device memory (its scratch is a fixed static array;
+    see include/mla_prefill.h for the size limit and the sharing rules)."""
+    lib = load_library()
+    descs = [as_mla_tensor(t) for t in (q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, out)]
+    rc = lib.mla_prefill_noalloc(*(ctypes.byref(d) for d in descs[:7]), int(mask_type), int(head_num),
+                                 int(kv_head_num), float(qk_scale), ctypes.byref(descs[7]),
+                                 _stream_handle(stream, q.device))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_noalloc")
     return out
 
 

@@ -346,3 +346,157 @@ int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *
 int mla_prefill_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.  Same validation and the same two kernels as
+// mla_prefill, but the plan workspace and the status word live in one static
+// device array of fixed size instead of library-allocated device memory.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;               // 1 MiB on every GPU that loads the library
+constexpr size_t kNoAllocStatusOffset = kNoAllocScratchBytes - 256;    // last 256 bytes: status word
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocDevice {
+    bool ready = false;
+    int sm_count = 0;
+    uint8_t *scratch = nullptr;  // device address of g_noalloc_scratch on this GPU
+    DeviceState launch;          // only its dynamic-shared-memory opt-in flags are used
+};
+
+NoAllocDevice g_noalloc[kMaxDevices];
+
+// One-time set-up per GPU, with that GPU current: the array's device address
+// (the host-side symbol is only a stand-in), the SM count, the arch check.
+int noalloc_setup(int dev, NoAllocDevice **out) {
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    NoAllocDevice &d = g_noalloc[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MLA_ERR_CUDA;
+        d.scratch = static_cast<uint8_t *>(ptr);
+        d.ready = true;
+    }
+    *out = &d;
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
+                                   const mla_tensor *k_rope, const mla_tensor *v, const mla_tensor *q_seqlen,
+                                   const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num,
+                                   float qk_scale, mla_tensor *out, mla_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!q || !q_rope || !k || !k_rope || !v || !q_seqlen || !kv_seqlen || !out) return MLA_ERR_NULL;
+    if (head_num < 1 || kv_head_num < 1 || head_num % kv_head_num != 0) return MLA_ERR_HEADS;
+    if (mask_type != MLA_MASK_CAUSAL && mask_type != MLA_MASK_NONE) return MLA_ERR_UNSUPPORTED;
+    if (!std::isfinite(qk_scale)) return MLA_ERR_UNSUPPORTED;
+    const int dt = q->dtype;
+    if (dt != MLA_BF16 && dt != MLA_F16) return MLA_ERR_DTYPE;
+    if (is_padded_kv(k, kv_head_num, mla::kDn) || is_padded_kv(v, kv_head_num, mla::kDn) ||
+        is_padded_kv(k_rope, kv_head_num, mla::kDr))
+        return MLA_ERR_UNSUPPORTED;
+
+    View3 vq, vqr, vk, vkr, vv, vo;
+    int rc;
+    if ((rc = view3(q, dt, head_num, mla::kDn, &vq)) != MLA_OK) return rc;
+    if ((rc = view3(q_rope, dt, head_num, mla::kDr, &vqr)) != MLA_OK) return rc;
+    if ((rc = view3(k, dt, kv_head_num, mla::kDn, &vk)) != MLA_OK) return rc;
+    if ((rc = view3(k_rope, dt, kv_head_num, mla::kDr, &vkr)) != MLA_OK) return rc;
+    if ((rc = view3(v, dt, kv_head_num, mla::kDn, &vv)) != MLA_OK) return rc;
+    if ((rc = view3(out, dt, head_num, mla::kDn, &vo)) != MLA_OK) return rc;
+    if (vqr.tokens != vq.tokens || vo.tokens != vq.tokens || vkr.tokens != vk.tokens || vv.tokens != vk.tokens)
+        return MLA_ERR_SHAPE;
+
+    if (q_seqlen->dtype != MLA_I32 || kv_seqlen->dtype != MLA_I32) return MLA_ERR_DTYPE;
+    if (q_seqlen->ndim != 1 || kv_seqlen->ndim != 1 || q_seqlen->shape[0] != kv_seqlen->shape[0])
+        return MLA_ERR_SHAPE;
+    if (q_seqlen->shape[0] > 0 && (!q_seqlen->data || !kv_seqlen->data)) return MLA_ERR_NULL;
+    if (q_seqlen->shape[0] > 1 && (q_seqlen->stride[0] != 1 || kv_seqlen->stride[0] != 1)) return MLA_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(q_seqlen->data) & 3u) || (reinterpret_cast<uintptr_t>(kv_seqlen->data) & 3u))
+        return MLA_ERR_ALIGN;
+    const int64_t batch = q_seqlen->shape[0];
+    if (batch < 0 || batch > INT32_MAX / 2) return MLA_ERR_SHAPE;
+
+    for (const View3 *in : {&vq, &vqr, &vk, &vkr, &vv})
+        if (overlaps(vo, *in)) return MLA_ERR_UNSUPPORTED;
+
+    // The whole plan workspace must fit in the static array, ahead of the status word.
+    const WsLayout lay = ws_layout(batch, vq.tokens, vk.tokens);
+    if (lay.total > kNoAllocStatusOffset) return MLA_ERR_UNSUPPORTED;
+
+    if (batch == 0 || vq.tokens == 0) return MLA_OK;  // nothing to compute
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    NoAllocDevice *nd = nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((rc = noalloc_setup(dev, &nd)) != MLA_OK) return rc;
+    if ((rc = ensure_encode()) != MLA_OK) return rc;
+
+    const bool bf16 = dt == MLA_BF16;
+    CUtensorMap maps[5];
+    if ((rc = encode_map(&maps[0], vq, bf16, nd->scratch, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[1], vqr, bf16, nd->scratch, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[2], vk, bf16, nd->scratch, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[3], vkr, bf16, nd->scratch, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[4], vv, bf16, nd->scratch, 64)) != MLA_OK) return rc;
+
+    // Every entry the kernels read is rewritten by the plan kernel on each call
+    // (including the zeroed histogram and work counter), so the array's previous
+    // contents never leak into a result.
+    uint8_t *ws = nd->scratch;
+    int *num_units = reinterpret_cast<int *>(ws + lay.num_units);
+    int *work_counter = num_units + 1;
+    int4 *seq_info = reinterpret_cast<int4 *>(ws + lay.seq_info);
+    int *unit_off = reinterpret_cast<int *>(ws + lay.unit_off);
+    int *hist = reinterpret_cast<int *>(ws + lay.hist);
+    int2 *units = reinterpret_cast<int2 *>(ws + lay.units);
+    int *status = reinterpret_cast<int *>(ws + kNoAllocStatusOffset);
+    const bool causal = mask_type == MLA_MASK_CAUSAL;
+
+    mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
+        static_cast<const int *>(q_seqlen->data), static_cast<const int *>(kv_seqlen->data), static_cast<int>(batch),
+        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
+        status);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+
+    mla::Params p;
+    p.seq_info = seq_info;
+    p.units = units;
+    p.num_units = num_units;
+    p.work_counter = work_counter;
+    p.status = status;
+    p.out = vo.data;
+    p.out_st = vo.st_tok;
+    p.out_sh = vo.st_head;
+    p.head_num = head_num;
+    p.group = head_num / kv_head_num;
+    p.scale_log2 = qk_scale * 1.4426950408889634f;
+
+    const int64_t max_items = ((vq.tokens + mla::kUnitRows - 1) / mla::kUnitRows + batch) * head_num;
+    const int grid = static_cast<int>(max_items < nd->sm_count ? max_items : nd->sm_count);
+    const bool pos = qk_scale > 0.f;
+    DeviceState *ls = &nd->launch;
+    if (bf16) {
+        if (causal)
+            return pos ? launch_attention<__nv_bfloat16, true, true>(ls, 0, grid, stream, maps, p)
+                       : launch_attention<__nv_bfloat16, true, false>(ls, 1, grid, stream, maps, p);
+        return pos ? launch_attention<__nv_bfloat16, false, true>(ls, 2, grid, stream, maps, p)
+                   : launch_attention<__nv_bfloat16, false, false>(ls, 3, grid, stream, maps, p);
+    }
+    if (causal)
+        return pos ? launch_attention<__half, true, true>(ls, 4, grid, stream, maps, p)
+                   : launch_attention<__half, true, false>(ls, 5, grid, stream, maps, p);
+    return pos ? launch_attention<__half, false, true>(ls, 6, grid, stream, maps, p)
+               : launch_attention<__half, false, false>(ls, 7, grid, stream, maps, p);
+}
