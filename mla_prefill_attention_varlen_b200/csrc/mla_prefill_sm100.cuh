@@ -329,22 +329,21 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
     }
 }
 
-// Max of a 128-element row as a balanced tree (short dependency chains).
+// Max of a 128-element row: eight independent chains of three-input max
+// (two new elements per instruction), then a short tree.
 __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
-    float m[16];
+    static_assert(kBN == 128, "the block split below assumes 128 keys per tile");
+    float m[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m[i] = fmaxf(s[i], s[i + 16]);
+    for (int i = 0; i < 8; ++i) m[i] = ptx::fmax3(s[i], s[i + 8], s[i + 16]);  // s[0..23]
 #pragma unroll
-    for (int c = 32; c < kBN; c += 16) {
+    for (int c = 24; c + 16 <= kBN; c += 16) {                                 // s[24..119]
 #pragma unroll
-        for (int i = 0; i < 16; ++i) m[i] = fmaxf(m[i], s[c + i]);
+        for (int i = 0; i < 8; ++i) m[i] = ptx::fmax3(m[i], s[c + i], s[c + 8 + i]);
     }
 #pragma unroll
-    for (int w = 8; w >= 1; w >>= 1) {
-#pragma unroll
-        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
-    }
-    return m[0];
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], s[120 + i]);                // s[120..127]
+    return ptx::fmax3(ptx::fmax3(m[0], m[1], m[2]), ptx::fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // ---------------------------------------------------------------------------
@@ -669,21 +668,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after();
                 float s[kBN];
                 {
-                    uint32_t r0[32], r1[32], r2[32], r3[32];
-                    ptx::tmem_ld32(tS, r0);
-                    ptx::tmem_ld32(tS + 32, r1);
-                    ptx::tmem_ld32(tS + 64, r2);
-                    ptx::tmem_ld32(tS + 96, r3);
-                    ptx::tmem_wait_ld_dep(r0);
-                    ptx::tmem_wait_ld_dep(r1);
-                    ptx::tmem_wait_ld_dep(r2);
-                    ptx::tmem_wait_ld_dep(r3);
+                    uint32_t r0[64], r1[64];
+                    ptx::tmem_ld64(tS, r0);
+                    ptx::tmem_ld64(tS + 64, r1);
+                    ptx::tmem_wait_ld_dep64(r0);
+                    ptx::tmem_wait_ld_dep64(r1);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 64; ++e) {
                         s[e] = __uint_as_float(r0[e]);
-                        s[32 + e] = __uint_as_float(r1[e]);
-                        s[64 + e] = __uint_as_float(r2[e]);
-                        s[96 + e] = __uint_as_float(r3[e]);
+                        s[64 + e] = __uint_as_float(r1[e]);
                     }
                 }
                 const int kv0 = j * kBN;
@@ -709,44 +702,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_run = m_tile;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                float psum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
+                // p = 2^(s * scale * log2 e - m): one packed FMA per pair, one MUFU op per element,
+                // packed partial sums, one 16-bit pair conversion per pair.
+                const float2 sc2 = kPositiveScale ? make_float2(sl2, sl2) : make_float2(1.f, 1.f);
+                const float2 nm2 = make_float2(-m_use, -m_use);
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f)};
+                uint32_t pk[64];
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = h2 * 64 + 2 * e;
-                        float p0, p1;
-                        if (kPositiveScale) {
-                            p0 = ptx::ex2(fmaf(s[c], sl2, -m_use));
-                            p1 = ptx::ex2(fmaf(s[c + 1], sl2, -m_use));
-                        } else {
-                            p0 = ptx::ex2(s[c] - m_use);
-                            p1 = ptx::ex2(s[c + 1] - m_use);
-                        }
-                        psum[e & 7] += p0 + p1;
-                        pk[e] = DType<T>::pack(p0, p1);
-                    }
-                    ptx::tmem_st32(tS + kTmemPOff + h2 * 32, pk);
+                for (int e = 0; e < 64; ++e) {
+                    const float2 x2 = ptx::ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+                    const float2 p2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
+                    acc[e & 3] = ptx::fadd2(acc[e & 3], p2);
+                    pk[e] = DType<T>::pack(p2.x, p2.y);
                 }
+                ptx::tmem_st64(tS + kTmemPOff, pk);
                 // O_t holds P(j-1) V(j-1) already (the MMAs behind S_t(j) have completed);
-                // rescale it before PV_t(j) may start (S is dead here: fewer live registers).
+                // rescale it before PV_t(j) may start.
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-                    for (int c = 0; c < kDn / 32; ++c) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(tO + c * 32, r);
-                        ptx::tmem_wait_ld_dep(r);
+                    for (int c = 0; c < kDn / 64; ++c) {
+                        uint32_t r[64];
+                        ptx::tmem_ld64(tO + c * 64, r);
+                        ptx::tmem_wait_ld_dep64(r);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                        ptx::tmem_st32(tO + c * 32, r);
+                        for (int e = 0; e < 32; ++e) {
+                            const float2 v2 = ptx::fmul2(
+                                make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), a2);
+                            r[2 * e] = __float_as_uint(v2.x);
+                            r[2 * e + 1] = __float_as_uint(v2.y);
+                        }
+                        ptx::tmem_st64(tO + c * 64, r);
                     }
                 }
+                const float2 acc01 = ptx::fadd2(acc[0], acc[1]), acc23 = ptx::fadd2(acc[2], acc[3]);
+                const float2 acc2 = ptx::fadd2(acc01, acc23);
+                const float rowsum = acc2.x + acc2.y;
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(bar(bars->p_full[t]));
-                const float rowsum = ((psum[0] + psum[1]) + (psum[2] + psum[3])) +
-                                     ((psum[4] + psum[5]) + (psum[6] + psum[7]));
                 l_run = l_run * alpha + rowsum;
             }
             if (!ok) break;
