@@ -48,6 +48,41 @@ def algorithmic_bytes(wl):
         wl.d_nope + wl.d_rope + wl.d_nope) + wl.t_q * wl.head_num * wl.d_nope)
 
 
+KERNEL_SOURCES = ["mla_prefill_attention_varlen_b200/csrc/mla_prefill_sm100.cuh",
+                  "mla_prefill_attention_varlen_b200/csrc/sm100_ptx.cuh"]
+
+
+def kernel_sources_hash():
+    """sha256 over the device-code sources (a measured traffic figure is only valid for this code)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "mla_prefill_sm100_kernel_%s_dram.md" % workload)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        line = line.strip().strip("`")
+        if line.startswith("traffic_bytes_per_launch=") or line.startswith("kernel_sources_sha256="):
+            k, v = line.split("=", 1)
+            fields[k] = v.strip()
+    if fields.get("kernel_sources_sha256") != kernel_sources_hash():
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -439,7 +474,7 @@ def main():
         "tokens_per_s": tokens_per_s,
         "north_star_literal_tflops": 2 * value,
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": kern_tflops / peak, "traffic": None, "peak_source": peak_src,
+                     "frac": kern_tflops / peak, "traffic": measured_traffic(wl.name), "peak_source": peak_src,
                      "peak_kind": "burst", "frac_of_sustained": kern_tflops / peak_sus,
                      "kernel": "mla_prefill_sm100_kernel", "kernel_ms": kms,
                      "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": algorithmic_bytes(wl)},

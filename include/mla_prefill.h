@@ -81,6 +81,11 @@ typedef enum {
  *   k       [T_k, G, 128] or [T_k, G*128]   K "nope" part        (page: K row, packed form)
  *   k_rope  [T_k, G, 64]  or [T_k, G*64]    K rotary part, per kv head (page: kRope row)
  *   v       [T_k, G, 128] or [T_k, G*128]   values               (page: V row, packed form)
+ *     or all three in the page's padded form [batch, max_seq, G*128] / [batch,
+ *     max_seq, G*64] / [batch, max_seq, G*128]: sequence b's keys are rows
+ *     0 .. Lk_b-1 of batch entry b (Lk_b <= max_seq); the batch rows must be
+ *     dense (batch stride = max_seq * token stride).  A [batch, 1, G*W]
+ *     tensor reads the same either way and is taken as packed.
  *   q_seqlen, kv_seqlen  [batch] MLA_I32 in DEVICE memory (page: qSeqLen / kvSeqLen rows).
  *     Sequence b owns query tokens [sum_{b'<b} Lq_b', + Lq_b) and key tokens
  *     [sum_{b'<b} Lk_b', + Lk_b) of the packed tensors.
@@ -95,9 +100,9 @@ typedef enum {
  *
  * Layout rules: the last dimension is contiguous (stride 1); token and head
  * strides are positive multiples of 8 elements (so q_rope / k_rope may be views
- * into wider buffers); every base pointer is 16-byte aligned.  The padded
- * [batch, max_seq, G*128] K/V form of the page is rejected with
- * MLA_ERR_UNSUPPORTED.  `out` must not overlap any input.
+ * into wider buffers); every base pointer is 16-byte aligned.  K, K_rope and V
+ * are either all packed or all padded (else MLA_ERR_UNSUPPORTED).  `out` must
+ * not overlap any input.
  *
  * Ownership and errors: the caller owns every buffer.  Argument errors are
  * detected on the host and returned before anything is launched; `out` is then
@@ -106,7 +111,8 @@ typedef enum {
  * that GPU, grown when a call needs more; a call that grows it allocates
  * device memory).  Calls that share a GPU must be ordered on one stream, or
  * otherwise serialised, because they share that workspace.
- * Inconsistent seqlens (negative, or summing past T_q / T_k) are detected on
+ * Inconsistent seqlens (negative, summing past T_q / T_k, or Lk_b > max_seq in
+ * the padded form) are detected on
  * the device: the kernel clamps to the tensor extents -- it never reads or
  * writes out of bounds -- and records MLA_ERR_SEQLEN in a sticky status word
  * that mla_prefill_device_status() returns.

@@ -73,10 +73,33 @@ int view3(const mla_tensor *t, int dtype, int64_t heads, int64_t width, View3 *v
     return MLA_OK;
 }
 
-// The padded [batch, max_seq, G*128] K/V form: 3-D with a last dim of G*W (G > 1),
-// or with a middle extent other than G when G == 1.
+// The padded [batch, max_seq, G*W] K/V form of the page: 3-D with a last dim of
+// G*W and a middle extent other than G (G == 1 and max_seq == 1 read the same
+// either way).
 bool is_padded_kv(const mla_tensor *t, int64_t heads, int64_t width) {
     return t && t->ndim == 3 && t->shape[2] == heads * width && !(t->shape[1] == heads && t->shape[2] == width);
+}
+
+// A dense padded tensor [batch, max_seq, G*W] viewed as packed tokens
+// [batch*max_seq, G, W]: sequence b's keys start at token b*max_seq.
+int padded_view(const mla_tensor *t, int dtype, int64_t heads, int64_t width, int64_t batch, int64_t max_seq,
+                View3 *v) {
+    if (!t || (!t->data && t->shape[0] * t->shape[1] != 0)) return MLA_ERR_NULL;
+    if (t->dtype != dtype) return MLA_ERR_DTYPE;
+    if (t->shape[0] != batch || t->shape[1] != max_seq || t->shape[2] != heads * width) return MLA_ERR_SHAPE;
+    if (t->stride[2] != 1) return MLA_ERR_ALIGN;
+    if (batch > 1 && t->stride[0] != max_seq * t->stride[1]) return MLA_ERR_UNSUPPORTED;  // batch rows must be dense
+    v->data = t->data;
+    v->tokens = batch * max_seq;
+    v->heads = heads;
+    v->width = width;
+    v->st_tok = t->stride[1];
+    v->st_head = width;
+    if (v->tokens > INT32_MAX) return MLA_ERR_SHAPE;
+    if (v->data && !aligned16(v->data)) return MLA_ERR_ALIGN;
+    if (v->st_tok % 8 != 0 || (v->tokens > 1 && v->st_tok < heads * width)) return MLA_ERR_ALIGN;
+    if (v->st_tok * 2 >= (int64_t(1) << 40)) return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
 }
 
 // [lo, hi) byte range a view touches (for the no-alias check).
@@ -193,34 +216,26 @@ int launch_attention(DeviceState *ds, int slot, int grid, cudaStream_t stream, c
     return MLA_OK;
 }
 
-}  // namespace
+// Everything a call needs after host-side validation.
+struct Problem {
+    View3 q, qr, k, kr, v, o;
+    const int *q_seqlen, *kv_seqlen;
+    int64_t batch;
+    int64_t kv_pad;  // 0: packed K/V; else the padded layout's max_seq
+    bool bf16, causal;
+    int head_num, kv_head_num;
+    float qk_scale;
+};
 
-extern "C" {
-
-int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
-                const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
-                int head_num, int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+int validate(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+             const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+             int head_num, int kv_head_num, float qk_scale, const mla_tensor *out, Problem *pr) {
     if (!q || !q_rope || !k || !k_rope || !v || !q_seqlen || !kv_seqlen || !out) return MLA_ERR_NULL;
     if (head_num < 1 || kv_head_num < 1 || head_num % kv_head_num != 0) return MLA_ERR_HEADS;
     if (mask_type != MLA_MASK_CAUSAL && mask_type != MLA_MASK_NONE) return MLA_ERR_UNSUPPORTED;
     if (!std::isfinite(qk_scale)) return MLA_ERR_UNSUPPORTED;
     const int dt = q->dtype;
     if (dt != MLA_BF16 && dt != MLA_F16) return MLA_ERR_DTYPE;
-    if (is_padded_kv(k, kv_head_num, mla::kDn) || is_padded_kv(v, kv_head_num, mla::kDn) ||
-        is_padded_kv(k_rope, kv_head_num, mla::kDr))
-        return MLA_ERR_UNSUPPORTED;
-
-    View3 vq, vqr, vk, vkr, vv, vo;
-    int rc;
-    if ((rc = view3(q, dt, head_num, mla::kDn, &vq)) != MLA_OK) return rc;
-    if ((rc = view3(q_rope, dt, head_num, mla::kDr, &vqr)) != MLA_OK) return rc;
-    if ((rc = view3(k, dt, kv_head_num, mla::kDn, &vk)) != MLA_OK) return rc;
-    if ((rc = view3(k_rope, dt, kv_head_num, mla::kDr, &vkr)) != MLA_OK) return rc;
-    if ((rc = view3(v, dt, kv_head_num, mla::kDn, &vv)) != MLA_OK) return rc;
-    if ((rc = view3(out, dt, head_num, mla::kDn, &vo)) != MLA_OK) return rc;
-    if (vqr.tokens != vq.tokens || vo.tokens != vq.tokens || vkr.tokens != vk.tokens || vv.tokens != vk.tokens)
-        return MLA_ERR_SHAPE;
 
     if (q_seqlen->dtype != MLA_I32 || kv_seqlen->dtype != MLA_I32) return MLA_ERR_DTYPE;
     if (q_seqlen->ndim != 1 || kv_seqlen->ndim != 1 || q_seqlen->shape[0] != kv_seqlen->shape[0])
@@ -232,40 +247,67 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
     const int64_t batch = q_seqlen->shape[0];
     if (batch < 0 || batch > INT32_MAX / 2) return MLA_ERR_SHAPE;
 
-    for (const View3 *in : {&vq, &vqr, &vk, &vkr, &vv})
-        if (overlaps(vo, *in)) return MLA_ERR_UNSUPPORTED;
+    int rc;
+    if ((rc = view3(q, dt, head_num, mla::kDn, &pr->q)) != MLA_OK) return rc;
+    if ((rc = view3(q_rope, dt, head_num, mla::kDr, &pr->qr)) != MLA_OK) return rc;
+    if ((rc = view3(out, dt, head_num, mla::kDn, &pr->o)) != MLA_OK) return rc;
+    const bool pk = is_padded_kv(k, kv_head_num, mla::kDn), pkr = is_padded_kv(k_rope, kv_head_num, mla::kDr),
+               pv = is_padded_kv(v, kv_head_num, mla::kDn);
+    pr->kv_pad = 0;
+    if (pk || pkr || pv) {
+        if (!(pk && pkr && pv)) return MLA_ERR_UNSUPPORTED;  // all three padded, or none
+        const int64_t max_seq = k->shape[1];
+        if (max_seq < 1 || max_seq > INT32_MAX) return MLA_ERR_SHAPE;
+        if ((rc = padded_view(k, dt, kv_head_num, mla::kDn, batch, max_seq, &pr->k)) != MLA_OK) return rc;
+        if ((rc = padded_view(k_rope, dt, kv_head_num, mla::kDr, batch, max_seq, &pr->kr)) != MLA_OK) return rc;
+        if ((rc = padded_view(v, dt, kv_head_num, mla::kDn, batch, max_seq, &pr->v)) != MLA_OK) return rc;
+        pr->kv_pad = max_seq;
+    } else {
+        if ((rc = view3(k, dt, kv_head_num, mla::kDn, &pr->k)) != MLA_OK) return rc;
+        if ((rc = view3(k_rope, dt, kv_head_num, mla::kDr, &pr->kr)) != MLA_OK) return rc;
+        if ((rc = view3(v, dt, kv_head_num, mla::kDn, &pr->v)) != MLA_OK) return rc;
+    }
+    if (pr->qr.tokens != pr->q.tokens || pr->o.tokens != pr->q.tokens || pr->kr.tokens != pr->k.tokens ||
+        pr->v.tokens != pr->k.tokens)
+        return MLA_ERR_SHAPE;
+    for (const View3 *in : {&pr->q, &pr->qr, &pr->k, &pr->kr, &pr->v})
+        if (overlaps(pr->o, *in)) return MLA_ERR_UNSUPPORTED;
 
-    if (batch == 0 || vq.tokens == 0) return MLA_OK;  // nothing to compute
+    pr->q_seqlen = static_cast<const int *>(q_seqlen->data);
+    pr->kv_seqlen = static_cast<const int *>(kv_seqlen->data);
+    pr->batch = batch;
+    pr->bf16 = dt == MLA_BF16;
+    pr->causal = mask_type == MLA_MASK_CAUSAL;
+    pr->head_num = head_num;
+    pr->kv_head_num = kv_head_num;
+    pr->qk_scale = qk_scale;
+    return MLA_OK;
+}
 
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-    const WsLayout lay = ws_layout(batch, vq.tokens, vk.tokens);
-    DeviceState *ds = nullptr;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if ((rc = device_state(dev, stream, lay.total, &ds)) != MLA_OK) return rc;
+// Encodes the tensor maps and enqueues the plan and attention kernels.  `ws`
+// holds the workspace described by `lay`; `launch_flags` records the
+// per-instantiation shared-memory opt-in for the current GPU.
+int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, int sm_count, DeviceState *launch_flags,
+            cudaStream_t stream) {
+    int rc;
     if ((rc = ensure_encode()) != MLA_OK) return rc;
-
-    const bool bf16 = dt == MLA_BF16;
     CUtensorMap maps[5];
-    if ((rc = encode_map(&maps[0], vq, bf16, ds->ws, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[1], vqr, bf16, ds->ws, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[2], vk, bf16, ds->ws, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[3], vkr, bf16, ds->ws, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[4], vv, bf16, ds->ws, 64)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[0], pr.q, pr.bf16, ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[1], pr.qr, pr.bf16, ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[2], pr.k, pr.bf16, ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[3], pr.kr, pr.bf16, ws, 128)) != MLA_OK) return rc;
+    if ((rc = encode_map(&maps[4], pr.v, pr.bf16, ws, 64)) != MLA_OK) return rc;
 
-    uint8_t *ws = static_cast<uint8_t *>(ds->ws);
     int *num_units = reinterpret_cast<int *>(ws + lay.num_units);
     int *work_counter = num_units + 1;  // second word of the 16-byte header
     int4 *seq_info = reinterpret_cast<int4 *>(ws + lay.seq_info);
     int *unit_off = reinterpret_cast<int *>(ws + lay.unit_off);
     int *hist = reinterpret_cast<int *>(ws + lay.hist);
     int2 *units = reinterpret_cast<int2 *>(ws + lay.units);
-    const bool causal = mask_type == MLA_MASK_CAUSAL;
 
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
-        static_cast<const int *>(q_seqlen->data), static_cast<const int *>(kv_seqlen->data), static_cast<int>(batch),
-        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
-        ds->status);
+        pr.q_seqlen, pr.kv_seqlen, static_cast<int>(pr.batch), pr.q.tokens, pr.k.tokens, pr.kv_pad,
+        pr.causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter, status);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
     mla::Params p;
@@ -273,29 +315,53 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
     p.units = units;
     p.num_units = num_units;
     p.work_counter = work_counter;
-    p.status = ds->status;
-    p.out = vo.data;
-    p.out_st = vo.st_tok;
-    p.out_sh = vo.st_head;
-    p.head_num = head_num;
-    p.group = head_num / kv_head_num;
-    p.scale_log2 = qk_scale * 1.4426950408889634f;
+    p.status = status;
+    p.out = pr.o.data;
+    p.out_st = pr.o.st_tok;
+    p.out_sh = pr.o.st_head;
+    p.head_num = pr.head_num;
+    p.group = pr.head_num / pr.kv_head_num;
+    p.scale_log2 = pr.qk_scale * 1.4426950408889634f;
 
-    const int64_t max_items = ((vq.tokens + mla::kUnitRows - 1) / mla::kUnitRows + batch) * head_num;
-    const int grid = static_cast<int>(max_items < ds->sm_count ? max_items : ds->sm_count);
-    const bool pos = qk_scale > 0.f;
-    if (bf16) {
-        if (causal)
-            return pos ? launch_attention<__nv_bfloat16, true, true>(ds, 0, grid, stream, maps, p)
-                       : launch_attention<__nv_bfloat16, true, false>(ds, 1, grid, stream, maps, p);
-        return pos ? launch_attention<__nv_bfloat16, false, true>(ds, 2, grid, stream, maps, p)
-                   : launch_attention<__nv_bfloat16, false, false>(ds, 3, grid, stream, maps, p);
+    const int64_t max_items = ((pr.q.tokens + mla::kUnitRows - 1) / mla::kUnitRows + pr.batch) * pr.head_num;
+    const int grid = static_cast<int>(max_items < sm_count ? max_items : sm_count);
+    const bool pos = pr.qk_scale > 0.f;
+    DeviceState *ls = launch_flags;
+    if (pr.bf16) {
+        if (pr.causal)
+            return pos ? launch_attention<__nv_bfloat16, true, true>(ls, 0, grid, stream, maps, p)
+                       : launch_attention<__nv_bfloat16, true, false>(ls, 1, grid, stream, maps, p);
+        return pos ? launch_attention<__nv_bfloat16, false, true>(ls, 2, grid, stream, maps, p)
+                   : launch_attention<__nv_bfloat16, false, false>(ls, 3, grid, stream, maps, p);
     }
-    if (causal)
-        return pos ? launch_attention<__half, true, true>(ds, 4, grid, stream, maps, p)
-                   : launch_attention<__half, true, false>(ds, 5, grid, stream, maps, p);
-    return pos ? launch_attention<__half, false, true>(ds, 6, grid, stream, maps, p)
-               : launch_attention<__half, false, false>(ds, 7, grid, stream, maps, p);
+    if (pr.causal)
+        return pos ? launch_attention<__half, true, true>(ls, 4, grid, stream, maps, p)
+                   : launch_attention<__half, true, false>(ls, 5, grid, stream, maps, p);
+    return pos ? launch_attention<__half, false, true>(ls, 6, grid, stream, maps, p)
+               : launch_attention<__half, false, false>(ls, 7, grid, stream, maps, p);
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+                const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+                int head_num, int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    Problem pr;
+    int rc = validate(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
+                      &pr);
+    if (rc != MLA_OK) return rc;
+    if (pr.batch == 0 || pr.q.tokens == 0) return MLA_OK;  // nothing to compute
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const WsLayout lay = ws_layout(pr.batch, pr.q.tokens, pr.k.tokens);
+    DeviceState *ds = nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((rc = device_state(dev, stream, lay.total, &ds)) != MLA_OK) return rc;
+    return enqueue(pr, lay, static_cast<uint8_t *>(ds->ws), ds->status, ds->sm_count, ds, stream);
 }
 
 int mla_prefill_device_status(mla_stream_t stream_, int *status) {
@@ -396,107 +462,23 @@ extern "C" int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope
                                    const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num,
                                    float qk_scale, mla_tensor *out, mla_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (!q || !q_rope || !k || !k_rope || !v || !q_seqlen || !kv_seqlen || !out) return MLA_ERR_NULL;
-    if (head_num < 1 || kv_head_num < 1 || head_num % kv_head_num != 0) return MLA_ERR_HEADS;
-    if (mask_type != MLA_MASK_CAUSAL && mask_type != MLA_MASK_NONE) return MLA_ERR_UNSUPPORTED;
-    if (!std::isfinite(qk_scale)) return MLA_ERR_UNSUPPORTED;
-    const int dt = q->dtype;
-    if (dt != MLA_BF16 && dt != MLA_F16) return MLA_ERR_DTYPE;
-    if (is_padded_kv(k, kv_head_num, mla::kDn) || is_padded_kv(v, kv_head_num, mla::kDn) ||
-        is_padded_kv(k_rope, kv_head_num, mla::kDr))
-        return MLA_ERR_UNSUPPORTED;
-
-    View3 vq, vqr, vk, vkr, vv, vo;
-    int rc;
-    if ((rc = view3(q, dt, head_num, mla::kDn, &vq)) != MLA_OK) return rc;
-    if ((rc = view3(q_rope, dt, head_num, mla::kDr, &vqr)) != MLA_OK) return rc;
-    if ((rc = view3(k, dt, kv_head_num, mla::kDn, &vk)) != MLA_OK) return rc;
-    if ((rc = view3(k_rope, dt, kv_head_num, mla::kDr, &vkr)) != MLA_OK) return rc;
-    if ((rc = view3(v, dt, kv_head_num, mla::kDn, &vv)) != MLA_OK) return rc;
-    if ((rc = view3(out, dt, head_num, mla::kDn, &vo)) != MLA_OK) return rc;
-    if (vqr.tokens != vq.tokens || vo.tokens != vq.tokens || vkr.tokens != vk.tokens || vv.tokens != vk.tokens)
-        return MLA_ERR_SHAPE;
-
-    if (q_seqlen->dtype != MLA_I32 || kv_seqlen->dtype != MLA_I32) return MLA_ERR_DTYPE;
-    if (q_seqlen->ndim != 1 || kv_seqlen->ndim != 1 || q_seqlen->shape[0] != kv_seqlen->shape[0])
-        return MLA_ERR_SHAPE;
-    if (q_seqlen->shape[0] > 0 && (!q_seqlen->data || !kv_seqlen->data)) return MLA_ERR_NULL;
-    if (q_seqlen->shape[0] > 1 && (q_seqlen->stride[0] != 1 || kv_seqlen->stride[0] != 1)) return MLA_ERR_ALIGN;
-    if ((reinterpret_cast<uintptr_t>(q_seqlen->data) & 3u) || (reinterpret_cast<uintptr_t>(kv_seqlen->data) & 3u))
-        return MLA_ERR_ALIGN;
-    const int64_t batch = q_seqlen->shape[0];
-    if (batch < 0 || batch > INT32_MAX / 2) return MLA_ERR_SHAPE;
-
-    for (const View3 *in : {&vq, &vqr, &vk, &vkr, &vv})
-        if (overlaps(vo, *in)) return MLA_ERR_UNSUPPORTED;
-
+    Problem pr;
+    int rc = validate(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
+                      &pr);
+    if (rc != MLA_OK) return rc;
     // The whole plan workspace must fit in the static array, ahead of the status word.
-    const WsLayout lay = ws_layout(batch, vq.tokens, vk.tokens);
+    const WsLayout lay = ws_layout(pr.batch, pr.q.tokens, pr.k.tokens);
     if (lay.total > kNoAllocStatusOffset) return MLA_ERR_UNSUPPORTED;
-
-    if (batch == 0 || vq.tokens == 0) return MLA_OK;  // nothing to compute
+    if (pr.batch == 0 || pr.q.tokens == 0) return MLA_OK;  // nothing to compute
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     NoAllocDevice *nd = nullptr;
     std::lock_guard<std::mutex> lock(g_mu);
     if ((rc = noalloc_setup(dev, &nd)) != MLA_OK) return rc;
-    if ((rc = ensure_encode()) != MLA_OK) return rc;
-
-    const bool bf16 = dt == MLA_BF16;
-    CUtensorMap maps[5];
-    if ((rc = encode_map(&maps[0], vq, bf16, nd->scratch, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[1], vqr, bf16, nd->scratch, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[2], vk, bf16, nd->scratch, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[3], vkr, bf16, nd->scratch, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[4], vv, bf16, nd->scratch, 64)) != MLA_OK) return rc;
-
     // Every entry the kernels read is rewritten by the plan kernel on each call
     // (including the zeroed histogram and work counter), so the array's previous
     // contents never leak into a result.
-    uint8_t *ws = nd->scratch;
-    int *num_units = reinterpret_cast<int *>(ws + lay.num_units);
-    int *work_counter = num_units + 1;
-    int4 *seq_info = reinterpret_cast<int4 *>(ws + lay.seq_info);
-    int *unit_off = reinterpret_cast<int *>(ws + lay.unit_off);
-    int *hist = reinterpret_cast<int *>(ws + lay.hist);
-    int2 *units = reinterpret_cast<int2 *>(ws + lay.units);
-    int *status = reinterpret_cast<int *>(ws + kNoAllocStatusOffset);
-    const bool causal = mask_type == MLA_MASK_CAUSAL;
-
-    mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
-        static_cast<const int *>(q_seqlen->data), static_cast<const int *>(kv_seqlen->data), static_cast<int>(batch),
-        vq.tokens, vk.tokens, causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
-        status);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-
-    mla::Params p;
-    p.seq_info = seq_info;
-    p.units = units;
-    p.num_units = num_units;
-    p.work_counter = work_counter;
-    p.status = status;
-    p.out = vo.data;
-    p.out_st = vo.st_tok;
-    p.out_sh = vo.st_head;
-    p.head_num = head_num;
-    p.group = head_num / kv_head_num;
-    p.scale_log2 = qk_scale * 1.4426950408889634f;
-
-    const int64_t max_items = ((vq.tokens + mla::kUnitRows - 1) / mla::kUnitRows + batch) * head_num;
-    const int grid = static_cast<int>(max_items < nd->sm_count ? max_items : nd->sm_count);
-    const bool pos = qk_scale > 0.f;
-    DeviceState *ls = &nd->launch;
-    if (bf16) {
-        if (causal)
-            return pos ? launch_attention<__nv_bfloat16, true, true>(ls, 0, grid, stream, maps, p)
-                       : launch_attention<__nv_bfloat16, true, false>(ls, 1, grid, stream, maps, p);
-        return pos ? launch_attention<__nv_bfloat16, false, true>(ls, 2, grid, stream, maps, p)
-                   : launch_attention<__nv_bfloat16, false, false>(ls, 3, grid, stream, maps, p);
-    }
-    if (causal)
-        return pos ? launch_attention<__half, true, true>(ls, 4, grid, stream, maps, p)
-                   : launch_attention<__half, true, false>(ls, 5, grid, stream, maps, p);
-    return pos ? launch_attention<__half, false, true>(ls, 6, grid, stream, maps, p)
-               : launch_attention<__half, false, false>(ls, 7, grid, stream, maps, p);
+    return enqueue(pr, lay, nd->scratch, reinterpret_cast<int *>(nd->scratch + kNoAllocStatusOffset), nd->sm_count,
+                   &nd->launch, stream);
 }

@@ -247,7 +247,8 @@ __device__ __forceinline__ int seq_of_unit(const int *unit_off, int batch, int t
 
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__restrict__ q_seqlen,
                                                                 const int *__restrict__ kv_seqlen, int batch,
-                                                                long long t_q, long long t_k, int causal,
+                                                                long long t_q, long long t_k, long long kv_pad,
+                                                                int causal,
                                                                 int4 *seq_info, int *unit_off, int *hist,
                                                                 int hist_len, int2 *units, int *num_units,
                                                                 int *work_counter, int *status) {
@@ -272,7 +273,10 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
         const long long pq = carry_q + block_exclusive_scan(lq, tot_q, warp_sums);
         const long long pk = carry_k + block_exclusive_scan(lk, tot_k, warp_sums);
         const long long cq = pq < t_q ? pq : t_q, eq = pq + lq < t_q ? pq + lq : t_q;
-        const long long ck = pk < t_k ? pk : t_k, ek = pk + lk < t_k ? pk + lk : t_k;
+        // packed K/V: sequences follow each other; padded K/V: sequence b starts at b * kv_pad
+        const long long kb = kv_pad ? (long long)b * kv_pad : pk;
+        const long long kcap = kv_pad ? kb + kv_pad : t_k;
+        const long long ck = kb < t_k ? kb : t_k, ek = kb + lk < kcap ? (kb + lk < t_k ? kb + lk : t_k) : (kcap < t_k ? kcap : t_k);
         if (b < batch && (eq - cq != lq || ek - ck != lk)) bad = 1;
         const int lqc = static_cast<int>(eq - cq), lkc = static_cast<int>(ek - ck);
         const long long nu = (b < batch) ? (lqc + kUnitRows - 1) / kUnitRows : 0;

@@ -130,11 +130,25 @@ def test_rejects_shapes(lib):
     assert call(lib, t, H, G) == 3
 
 
-def test_rejects_padded_kv_layout(lib):
-    # the page's [batch, max_seq, kv_head*embeddimV] form is not supported
-    t, H, G = make_args()
+def test_padded_kv_layout_checks(lib):
+    # the page's padded [batch, max_seq, kv_head*embeddimV] form: all of K, K_rope, V or none
+    t, H, G = make_args(batch=2)
     t["k"] = torch.zeros(2, 128, G * 128, dtype=torch.bfloat16)
+    assert call(lib, t, H, G) == 6  # K padded, K_rope / V packed
+    t["k_rope"] = torch.zeros(2, 128, G * 64, dtype=torch.bfloat16)
+    t["v"] = torch.zeros(2, 128, G * 128, dtype=torch.bfloat16)
+    if not torch.cuda.is_available():
+        assert call(lib, t, H, G) == 7  # valid: passes host validation, then needs CUDA
+    t["v"] = torch.zeros(2, 100, G * 128, dtype=torch.bfloat16)
+    assert call(lib, t, H, G) == 3  # max_seq differs between K and V
+    wide = torch.zeros(2, 256, G * 128, dtype=torch.bfloat16)
+    t["v"] = wide[:, :128]  # batch rows not dense
     assert call(lib, t, H, G) == 6
+    t, H, G = make_args(batch=3)
+    t["k"] = torch.zeros(2, 128, G * 128, dtype=torch.bfloat16)
+    t["k_rope"] = torch.zeros(2, 128, G * 64, dtype=torch.bfloat16)
+    t["v"] = torch.zeros(2, 128, G * 128, dtype=torch.bfloat16)
+    assert call(lib, t, H, G) == 3  # padded batch differs from len(q_seqlen)
 
 
 def test_rejects_misalignment(lib):

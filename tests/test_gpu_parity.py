@@ -280,3 +280,48 @@ def test_inconsistent_seqlens_are_clamped_and_reported(bad):
     assert torch.all(buf[:guard] == 5.0) and torch.all(buf[guard + T:] == 5.0)
     assert torch.isfinite(out.float()).all() or bad == "negative"
     assert status() == 0  # reading clears it
+
+
+# ---------------------------------------------------------------------------
+# the page's padded K/V layout [batch, max_seq, kv_head * dim]
+# ---------------------------------------------------------------------------
+
+def _to_padded(x, lens_k, max_seq, G):
+    """Packed K/K_rope/V -> dense padded [batch, max_seq, G*W] tensors (rows past Lk_b filled with 9)."""
+    out = {}
+    for key, w in (("k", 128), ("k_rope", 64), ("v", 128)):
+        buf = torch.full((len(lens_k), max_seq, G * w), 9.0, dtype=x[key].dtype, device=DEV)
+        start = 0
+        for b, L in enumerate(lens_k):
+            buf[b, :L] = x[key][start:start + L].reshape(L, G * w)
+            start += L
+        out[key] = buf
+    return out
+
+
+@pytest.mark.parametrize("case", [
+    ([100, 7, 260], [100, 7, 260], 300, 4, 2, torch.bfloat16),
+    ([64, 200], [700, 200], 768, 2, 2, torch.float16),
+])
+def test_padded_kv_layout_matches_packed(case):
+    lq, lk, max_seq, H, G, dtype = case
+    _, x = problem(lq, lk, H, G, dtype=dtype, seed=501)
+    packed = run(x, H, G, 0.07).clone()
+    y = dict(x, **_to_padded(x, lk, max_seq, G))
+    padded = run(y, H, G, 0.07)
+    torch.cuda.synchronize()
+    assert torch.equal(packed, padded)  # same keys, same tiles: bit-identical
+    check_against_oracle(x, padded, H, G, 0.07)
+    assert status() == 0
+
+
+def test_padded_kv_longer_than_max_seq_is_clamped_and_reported():
+    lq, lk, H, G = [50, 40], [50, 40], 2, 1
+    _, x = problem(lq, lk, H, G, seed=502)
+    y = dict(x, **_to_padded(x, lk, 64, G))
+    y["kv_seqlen"] = torch.tensor([50, 90], dtype=torch.int32, device=DEV)  # 90 > max_seq = 64
+    y["q_seqlen"] = torch.tensor([50, 40], dtype=torch.int32, device=DEV)
+    assert status() == 0
+    out = run(y, H, G, 0.07)
+    assert status() == 8
+    assert torch.isfinite(out[:90].float()).all()
