@@ -322,6 +322,99 @@ def reference_arm(args, wl):
     return 0
 
 
+def paged_inputs(wl, block_size, device, seed=7):
+    """A paged K/V cache holding the workload's keys: K rows [nope | rope] (192), V rows (128),
+    blocks assigned to the sequences in a seeded random order (a fragmented cache)."""
+    import torch
+
+    from mla_prefill_attention_varlen_b200 import workloads as W
+
+    x = W.make_inputs(wl, device=device)
+    G = wl.kv_head_num
+    kcat = torch.cat([x["k"], x["k_rope"]], dim=2)
+    need = [(L + block_size - 1) // block_size for L in wl.kv_seqlens]
+    nb = sum(need)
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(seed))
+    kc = torch.zeros(nb, block_size, G, wl.d_nope + wl.d_rope, dtype=wl.dtype, device=device)
+    vc = torch.zeros(nb, block_size, G, wl.d_nope, dtype=wl.dtype, device=device)
+    table = torch.zeros(len(need), max(need), dtype=torch.int32)
+    used = start = 0
+    for b, L in enumerate(wl.kv_seqlens):
+        idx = perm[used:used + need[b]]
+        table[b, :need[b]] = idx.to(torch.int32)
+        pad = need[b] * block_size - L
+        src_k = torch.nn.functional.pad(kcat[start:start + L], (0, 0, 0, 0, 0, pad))
+        src_v = torch.nn.functional.pad(x["v"][start:start + L], (0, 0, 0, 0, 0, pad))
+        kc[idx.to(device)] = src_k.view(need[b], block_size, G, -1)
+        vc[idx.to(device)] = src_v.view(need[b], block_size, G, -1)
+        used += need[b]
+        start += L
+    return kc, vc, table.to(device), x["kv_seqlen"]
+
+
+def bench_paged(args):
+    """mla_paged_cache_load on the cached prefix of a workload: GB/s of bytes read + written."""
+    import torch
+
+    import mla_prefill_attention_varlen_b200 as mla
+    from mla_prefill_attention_varlen_b200 import workloads as W
+
+    rank, world, local = dist_setup(args.gpus)
+    wl = W.get(args.workload)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    mla.load_library()
+    kc, vc, table, lens = paged_inputs(wl, args.block_size, dev)
+    T, G = wl.t_k, wl.kv_head_num
+    key = torch.empty(T, G, kc.shape[3], dtype=kc.dtype, device=dev)
+    value = torch.empty(T, G, vc.shape[3], dtype=vc.dtype, device=dev)
+    moved = 2 * (key.numel() + value.numel()) * key.element_size()  # each byte read once and written once
+    stream = torch.cuda.current_stream()
+
+    def step():
+        mla.mla_paged_cache_load(kc, vc, table, lens, key, value, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    smi = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    with smi:
+        time.sleep(0.1)
+        smi.mark_start()
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            stops[i].record(stream)
+        torch.cuda.synchronize()
+        smi.mark_stop()
+    barrier(world)
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)])), world)
+    st = mla.mla_prefill_device_status()
+    if st != 0:
+        raise RuntimeError("device status: %s" % mla.mla_status_string(st))
+    gbs = job_throughput(world, moved, ms) / 1e9
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    line = {
+        "metric": "paged KV-cache gather GB/s (bytes read + written)", "value": gbs, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16" if kc.dtype == torch.float16 else "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name + "_paged_prefix", "tokens": T, "kv_heads": G, "key_dim": kc.shape[3],
+                   "value_dim": vc.shape[3], "block_size": args.block_size, "blocks": kc.shape[0],
+                   "l2": "cache %.2f GB > 126 MB L2" % (moved / 2e9)},
+        "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / world / peak, "traffic": None, "peak_source": peak_src,
+                     "kernel": "paged_gather_kernel", "algorithmic_bytes_per_launch": moved},
+        "gpu_launches": 2 * args.steps, "clocks": smi.summary(), "cpu_baseline": None, "e2e": None,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -332,6 +425,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--op", default="prefill", choices=["prefill", "paged_cache_load"])
+    ap.add_argument("--block-size", type=int, default=64, help="paged_cache_load: tokens per cache block")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: scale head_num and kv_head_num down to this many query heads")
     args = ap.parse_args()
@@ -347,6 +442,8 @@ def main():
         wl.name += "_h%d" % args.heads
     if args.impl == "reference":
         return reference_arm(args, wl)
+    if args.op == "paged_cache_load":
+        return bench_paged(args)
 
     import torch
 

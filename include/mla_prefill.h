@@ -38,8 +38,8 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st *mla_stream_t;
 
-/* Element types (the page's float16 / bf16 data types, int32 seqlens). */
-typedef enum { MLA_F16 = 0, MLA_BF16 = 1, MLA_I32 = 2 } mla_dtype;
+/* Element types (the pages' float16 / bf16 / int8 data types, int32 lengths and tables). */
+typedef enum { MLA_F16 = 0, MLA_BF16 = 1, MLA_I32 = 2, MLA_I8 = 3 } mla_dtype;
 
 /*
  * A strided view of device memory, in the spirit of the page's aclTensor.
@@ -69,7 +69,8 @@ typedef enum {
     MLA_ERR_UNSUPPORTED = 6,   /* unsupported mask type, layout or argument value */
     MLA_ERR_CUDA = 7,          /* a CUDA runtime/driver call failed */
     MLA_ERR_SEQLEN = 8,        /* device-detected: a negative seqlen, or sum(seqlen) above the tensor extent */
-    MLA_ERR_DEVICE_TIMEOUT = 9 /* device-detected: a pipeline wait gave up (never expected) */
+    MLA_ERR_DEVICE_TIMEOUT = 9, /* device-detected: a pipeline wait gave up (never expected) */
+    MLA_ERR_INDEX = 10          /* device-detected: a paged-cache block index out of range (row zeroed) */
 } mla_status;
 
 /*
@@ -124,8 +125,9 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
 
 /*
  * mla_prefill_device_status -- synchronises `stream`, then reads and clears the
- * device status word of the current GPU (MLA_OK, MLA_ERR_SEQLEN or
- * MLA_ERR_DEVICE_TIMEOUT; the first error recorded since the last read).
+ * device status word of the current GPU (MLA_OK, MLA_ERR_SEQLEN,
+ * MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_INDEX; the first error recorded since the
+ * last read by mla_prefill or mla_paged_cache_load).
  * Writes it to *status and returns MLA_OK, or returns MLA_ERR_NULL /
  * MLA_ERR_CUDA.
  */
@@ -170,6 +172,43 @@ int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope, const mla
                         const mla_tensor *k_rope, const mla_tensor *v, const mla_tensor *q_seqlen,
                         const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num, float qk_scale,
                         mla_tensor *out, mla_stream_t stream);
+
+/*
+ * mla_paged_cache_load -- gathers a block-paged key / value cache into packed
+ * key / value tensors, asynchronously on `stream` (the PagedCacheLoadOperation
+ * page: AtbPagedCacheLoadGetWorkspaceSize / AtbPagedCacheLoad, ND cache format).
+ * Its key output, viewed as K_nope / K_rope columns, feeds mla_prefill.
+ *
+ *   key_cache    [num_blocks, block_size, H, Dk]  (page: keyCache, ND)
+ *   value_cache  [num_blocks, block_size, H, Dv]  (page: valueCache, ND)
+ *                MLA_F16, MLA_BF16 or MLA_I8 (bytes are copied, never converted);
+ *                each slot's H x D block contiguous; block / slot strides free
+ *                (multiples of 16 bytes); H*D*element size a multiple of 16 bytes.
+ *   block_tables [batch, W] MLA_I32: logical block i of batch entry b is physical
+ *                block block_tables[b][i] (page: blockTables).
+ *   context_lens MLA_I32 [batch] lengths, or with context_lens_cumsum != 0,
+ *                [batch + 1] running sums c with len_b = c[b+1] - c[b]
+ *                (page: contextLens, isSeqLensCumsumType).
+ *   seq_starts   MLA_I32 [batch] token offset of each entry's first token in
+ *                its block-table row, or NULL for 0 (page: seqStarts /
+ *                hasSeqStarts).
+ *   key, value   [T, H, Dk] / [T, H, Dv] (or [T, H*D]) outputs, dtypes of their
+ *                caches (page: key / value).  Entry b's tokens go to rows
+ *                len_0 + ... + len_{b-1} onwards.
+ * Token t of entry b is read from slot p % block_size of block
+ * block_tables[b][p / block_size], p = seq_starts[b] + t.
+ *
+ * All tensors are caller-owned device memory; the outputs must not overlap
+ * the caches or each other.  Argument errors return before any launch.
+ * Device-detected: lengths summing past T (clamped, MLA_ERR_SEQLEN) and rows
+ * whose logical block is past W or whose block id is outside [0, num_blocks)
+ * (written as zeros, MLA_ERR_INDEX); read them with mla_prefill_device_status.
+ * Shares the per-GPU workspace with mla_prefill: order both on one stream.
+ * Returns MLA_OK or an mla_status error code.
+ */
+int mla_paged_cache_load(const mla_tensor *key_cache, const mla_tensor *value_cache, const mla_tensor *block_tables,
+                         const mla_tensor *context_lens, const mla_tensor *seq_starts, int context_lens_cumsum,
+                         mla_tensor *key, mla_tensor *value, mla_stream_t stream);
 
 /* A static, human-readable name for a status code (never NULL). */
 const char *mla_status_string(int status);

@@ -12,16 +12,16 @@ import os
 from . import workloads  # noqa: F401  (seeded synthetic inputs)
 
 __all__ = [
-    "MLA_MASK_NONE", "MLA_MASK_CAUSAL", "MlaError", "load_library", "mla_prefill", "mla_prefill_device_status",
-    "mla_status_string", "prefill", "workloads",
+    "MLA_MASK_NONE", "MLA_MASK_CAUSAL", "MlaError", "load_library", "mla_prefill", "mla_prefill_noalloc",
+    "mla_paged_cache_load", "mla_prefill_device_status", "mla_status_string", "prefill", "workloads",
 ]
 
-MLA_F16, MLA_BF16, MLA_I32 = 0, 1, 2
+MLA_F16, MLA_BF16, MLA_I32, MLA_I8 = 0, 1, 2, 3
 MLA_MASK_NONE, MLA_MASK_CAUSAL = 0, 1
 STATUS_NAMES = {
     0: "MLA_OK", 1: "MLA_ERR_NULL", 2: "MLA_ERR_DTYPE", 3: "MLA_ERR_SHAPE", 4: "MLA_ERR_ALIGN",
     5: "MLA_ERR_HEADS", 6: "MLA_ERR_UNSUPPORTED", 7: "MLA_ERR_CUDA", 8: "MLA_ERR_SEQLEN",
-    9: "MLA_ERR_DEVICE_TIMEOUT",
+    9: "MLA_ERR_DEVICE_TIMEOUT", 10: "MLA_ERR_INDEX",
 }
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +62,8 @@ def load_library(path=None):
     lib.mla_prefill_noalloc.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_float, T, ctypes.c_void_p]
     lib.mla_prefill_noalloc.restype = ctypes.c_int
+    lib.mla_paged_cache_load.argtypes = [T, T, T, T, T, ctypes.c_int, T, T, ctypes.c_void_p]
+    lib.mla_paged_cache_load.restype = ctypes.c_int
     lib.mla_prefill_set_profile_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.mla_prefill_set_profile_events.restype = ctypes.c_int
     lib.mla_prefill_version.argtypes = []
@@ -81,7 +83,8 @@ def mla_status_string(code):
 def _dtype_code(t):
     import torch
 
-    return {torch.float16: MLA_F16, torch.bfloat16: MLA_BF16, torch.int32: MLA_I32}.get(t.dtype, -1)
+    return {torch.float16: MLA_F16, torch.bfloat16: MLA_BF16, torch.int32: MLA_I32, torch.int8: MLA_I8}.get(t.dtype,
+                                                                                                        -1)
 
 
 def as_mla_tensor(t):
@@ -150,6 +153,20 @@ def prefill(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, head_num, kv_head_num,
                           device=q.device)
     return mla_prefill(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale,
                        out, stream)
+
+
+def mla_paged_cache_load(key_cache, value_cache, block_tables, context_lens, key, value, seq_starts=None,
+                         cumsum=False, stream=None):
+    """Call the C ABI ``mla_paged_cache_load`` (gather a paged K/V cache into packed key / value)."""
+    lib = load_library()
+    d = [as_mla_tensor(t) for t in (key_cache, value_cache, block_tables, context_lens, key, value)]
+    ss = ctypes.byref(as_mla_tensor(seq_starts)) if seq_starts is not None else None
+    rc = lib.mla_paged_cache_load(ctypes.byref(d[0]), ctypes.byref(d[1]), ctypes.byref(d[2]), ctypes.byref(d[3]),
+                                  ss, 1 if cumsum else 0, ctypes.byref(d[4]), ctypes.byref(d[5]),
+                                  _stream_handle(stream, key.device))
+    if rc != 0:
+        raise MlaError(rc, "mla_paged_cache_load")
+    return key, value
 
 
 def set_profile_events(start=None, stop=None):

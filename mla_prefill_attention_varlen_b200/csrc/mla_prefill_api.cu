@@ -12,6 +12,7 @@
 
 #include "../../include/mla_prefill.h"
 #include "mla_prefill_sm100.cuh"
+#include "paged_cache_load.cuh"
 
 namespace {
 
@@ -395,6 +396,7 @@ const char *mla_status_string(int status) {
         case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA call failed";
         case MLA_ERR_SEQLEN: return "MLA_ERR_SEQLEN: seqlens inconsistent with tensor extents (clamped)";
         case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT: a device pipeline wait gave up";
+        case MLA_ERR_INDEX: return "MLA_ERR_INDEX: a paged-cache block index was out of range (row zeroed)";
         default: return "unknown mla_status";
     }
 }
@@ -481,4 +483,163 @@ extern "C" int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope
     // contents never leak into a result.
     return enqueue(pr, lay, nd->scratch, reinterpret_cast<int *>(nd->scratch + kNoAllocStatusOffset), nd->sm_count,
                    &nd->launch, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Paged KV-cache gather
+// ---------------------------------------------------------------------------
+namespace {
+
+int elem_bytes(int dtype) {
+    if (dtype == MLA_I8) return 1;
+    if (dtype == MLA_F16 || dtype == MLA_BF16) return 2;
+    return 0;
+}
+
+// A token-rows view: rows of `row_bytes` contiguous bytes, `stride` bytes apart.
+struct Rows {
+    uint8_t *data;
+    int64_t count, row_bytes, stride;
+};
+
+// Output [T, H, D] or [T, H*D] with each token's H x D block contiguous.
+int paged_output(const mla_tensor *t, int dtype, int64_t heads, int64_t dim, Rows *r) {
+    if (!t) return MLA_ERR_NULL;
+    if (t->dtype != dtype) return MLA_ERR_DTYPE;
+    const int es = elem_bytes(dtype);
+    if (t->ndim == 3) {
+        if (t->shape[1] != heads || t->shape[2] != dim) return MLA_ERR_SHAPE;
+        if (t->stride[2] != 1 || (heads > 1 && t->stride[1] != dim)) return MLA_ERR_ALIGN;
+    } else if (t->ndim == 2) {
+        if (t->shape[1] != heads * dim) return MLA_ERR_SHAPE;
+        if (t->stride[1] != 1) return MLA_ERR_ALIGN;
+    } else {
+        return MLA_ERR_SHAPE;
+    }
+    r->count = t->shape[0];
+    r->row_bytes = heads * dim * es;
+    r->stride = t->stride[0] * es;
+    r->data = static_cast<uint8_t *>(t->data);
+    if (r->count < 0 || r->count > INT32_MAX) return MLA_ERR_SHAPE;
+    if (r->count > 0 && !r->data) return MLA_ERR_NULL;
+    if ((r->data && !aligned16(r->data)) || r->row_bytes % 16 != 0) return MLA_ERR_ALIGN;
+    if (r->count > 1 && (r->stride % 16 != 0 || r->stride < r->row_bytes)) return MLA_ERR_ALIGN;
+    return MLA_OK;
+}
+
+// Cache [num_blocks, block_size, H, D] with each slot's H x D block contiguous.
+int paged_cache(const mla_tensor *t, int *dtype, int64_t *heads, int64_t *dim, int64_t *block_bytes,
+                int64_t *slot_bytes) {
+    if (!t || !t->data) return MLA_ERR_NULL;
+    if (t->ndim != 4) return MLA_ERR_SHAPE;
+    const int es = elem_bytes(t->dtype);
+    if (!es) return MLA_ERR_DTYPE;
+    *dtype = t->dtype;
+    *heads = t->shape[2];
+    *dim = t->shape[3];
+    if (t->shape[0] < 1 || t->shape[1] < 1 || *heads < 1 || *dim < 1) return MLA_ERR_SHAPE;
+    if (t->shape[0] > INT32_MAX) return MLA_ERR_SHAPE;
+    if (t->stride[3] != 1 || (*heads > 1 && t->stride[2] != *dim)) return MLA_ERR_ALIGN;
+    *block_bytes = t->stride[0] * es;
+    *slot_bytes = t->stride[1] * es;
+    const int64_t row = *heads * *dim * es;
+    if (!aligned16(t->data) || row % 16 != 0 || *block_bytes % 16 != 0 || *slot_bytes % 16 != 0)
+        return MLA_ERR_ALIGN;
+    if (*slot_bytes < row || *block_bytes <= 0) return MLA_ERR_ALIGN;
+    return MLA_OK;
+}
+
+bool rows_overlap(const Rows &r, const void *base, int64_t bytes) {
+    if (r.count == 0 || bytes <= 0) return false;
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(r.data), hi = lo + (r.count - 1) * r.stride + r.row_bytes;
+    const uintptr_t blo = reinterpret_cast<uintptr_t>(base), bhi = blo + bytes;
+    return lo < bhi && blo < hi;
+}
+
+}  // namespace
+
+extern "C" int mla_paged_cache_load(const mla_tensor *key_cache, const mla_tensor *value_cache,
+                                    const mla_tensor *block_tables, const mla_tensor *context_lens,
+                                    const mla_tensor *seq_starts, int context_lens_cumsum, mla_tensor *key,
+                                    mla_tensor *value, mla_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!key_cache || !value_cache || !block_tables || !context_lens || !key || !value) return MLA_ERR_NULL;
+    int kdt, vdt, rc;
+    int64_t H, Dk, Hv, Dv, kc_block, kc_slot, vc_block, vc_slot;
+    if ((rc = paged_cache(key_cache, &kdt, &H, &Dk, &kc_block, &kc_slot)) != MLA_OK) return rc;
+    if ((rc = paged_cache(value_cache, &vdt, &Hv, &Dv, &vc_block, &vc_slot)) != MLA_OK) return rc;
+    if (value_cache->shape[0] != key_cache->shape[0] || value_cache->shape[1] != key_cache->shape[1] || Hv != H)
+        return MLA_ERR_SHAPE;
+    Rows ko, vo;
+    if ((rc = paged_output(key, kdt, H, Dk, &ko)) != MLA_OK) return rc;
+    if ((rc = paged_output(value, vdt, H, Dv, &vo)) != MLA_OK) return rc;
+    if (ko.count != vo.count) return MLA_ERR_SHAPE;
+
+    if (block_tables->dtype != MLA_I32 || context_lens->dtype != MLA_I32) return MLA_ERR_DTYPE;
+    if (block_tables->ndim != 2 || context_lens->ndim != 1) return MLA_ERR_SHAPE;
+    const int64_t batch = block_tables->shape[0], width = block_tables->shape[1];
+    if (batch < 0 || batch > INT32_MAX / 2 || width < 0 || width > INT32_MAX) return MLA_ERR_SHAPE;
+    if (context_lens->shape[0] != batch + (context_lens_cumsum ? 1 : 0)) return MLA_ERR_SHAPE;
+    if (batch > 0 && (!block_tables->data || !context_lens->data)) return MLA_ERR_NULL;
+    if (width > 1 && block_tables->stride[1] != 1) return MLA_ERR_ALIGN;
+    if (batch > 1 && block_tables->stride[0] < width) return MLA_ERR_ALIGN;
+    if (context_lens->shape[0] > 1 && context_lens->stride[0] != 1) return MLA_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(block_tables->data) & 3u) || (reinterpret_cast<uintptr_t>(context_lens->data) & 3u))
+        return MLA_ERR_ALIGN;
+    if (seq_starts) {
+        if (seq_starts->dtype != MLA_I32) return MLA_ERR_DTYPE;
+        if (seq_starts->ndim != 1 || seq_starts->shape[0] != batch) return MLA_ERR_SHAPE;
+        if (batch > 0 && !seq_starts->data) return MLA_ERR_NULL;
+        if (batch > 1 && seq_starts->stride[0] != 1) return MLA_ERR_ALIGN;
+        if (reinterpret_cast<uintptr_t>(seq_starts->data) & 3u) return MLA_ERR_ALIGN;
+    }
+    const int64_t kc_bytes = (key_cache->shape[0] - 1) * kc_block + (key_cache->shape[1] - 1) * kc_slot + H * Dk *
+                             elem_bytes(kdt);
+    const int64_t vc_bytes = (value_cache->shape[0] - 1) * vc_block + (value_cache->shape[1] - 1) * vc_slot + H * Dv *
+                             elem_bytes(vdt);
+    if (rows_overlap(ko, key_cache->data, kc_bytes) || rows_overlap(ko, value_cache->data, vc_bytes) ||
+        rows_overlap(vo, key_cache->data, kc_bytes) || rows_overlap(vo, value_cache->data, vc_bytes) ||
+        rows_overlap(ko, vo.data, vo.count > 0 ? (vo.count - 1) * vo.stride + vo.row_bytes : 0))
+        return MLA_ERR_UNSUPPORTED;
+    if (batch == 0 || ko.count == 0) return MLA_OK;  // nothing to copy
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    DeviceState *ds = nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((rc = device_state(dev, stream, align_up(sizeof(int) * (batch + 1), 256), &ds)) != MLA_OK) return rc;
+    int *offs = static_cast<int *>(ds->ws);
+    mla::paged_plan_kernel<<<1, mla::kPagedPlanThreads, 0, stream>>>(
+        static_cast<const int *>(context_lens->data), static_cast<int>(batch), context_lens_cumsum ? 1 : 0, ko.count,
+        offs, ds->status);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+
+    mla::GatherParams p;
+    p.key_cache = static_cast<const uint8_t *>(key_cache->data);
+    p.value_cache = static_cast<const uint8_t *>(value_cache->data);
+    p.kc_block = kc_block;
+    p.kc_slot = kc_slot;
+    p.vc_block = vc_block;
+    p.vc_slot = vc_slot;
+    p.key_row = static_cast<int>(ko.row_bytes);
+    p.value_row = static_cast<int>(vo.row_bytes);
+    p.key = ko.data;
+    p.value = vo.data;
+    p.key_tok = ko.stride;
+    p.value_tok = vo.stride;
+    p.tables = static_cast<const int *>(block_tables->data);
+    p.table_stride = batch > 1 ? block_tables->stride[0] : width;
+    p.width = static_cast<int>(width);
+    p.num_blocks = static_cast<int>(key_cache->shape[0]);
+    p.block_size = static_cast<int>(key_cache->shape[1]);
+    p.starts = seq_starts ? static_cast<const int *>(seq_starts->data) : nullptr;
+    p.offs = offs;
+    p.batch = static_cast<int>(batch);
+    p.status = ds->status;
+    const int64_t rows = ko.count;
+    const int64_t want = (rows + mla::kGatherThreads / 32 - 1) / (mla::kGatherThreads / 32);
+    const int64_t cap = static_cast<int64_t>(ds->sm_count) * 8;
+    const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+    mla::paged_gather_kernel<<<grid, mla::kGatherThreads, 0, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

@@ -192,3 +192,41 @@ def test_accepts_2d_and_strided_views_on_host(lib):
 def test_empty_batch_is_a_no_op(lib):
     t, H, G = make_args(batch=0)
     assert call(lib, t, H, G) == 0
+
+
+# ---------------------------------------------------------------------------
+# mla_paged_cache_load host-side validation (descriptors are never dereferenced)
+# ---------------------------------------------------------------------------
+
+def paged_args(nb=6, bs=16, H=2, Dk=64, Dv=64, batch=2, W=4, T=40, dtype=torch.bfloat16):
+    return dict(kc=torch.zeros(nb, bs, H, Dk, dtype=dtype), vc=torch.zeros(nb, bs, H, Dv, dtype=dtype),
+                table=torch.zeros(batch, W, dtype=torch.int32), lens=torch.zeros(batch, dtype=torch.int32),
+                key=torch.zeros(T, H, Dk, dtype=dtype), value=torch.zeros(T, H, Dv, dtype=dtype))
+
+
+def paged_call(lib, a, starts=None, cumsum=0):
+    d = {k: mla.as_mla_tensor(v) for k, v in a.items()}
+    s = ctypes.byref(mla.as_mla_tensor(starts)) if starts is not None else None
+    return lib.mla_paged_cache_load(ctypes.byref(d["kc"]), ctypes.byref(d["vc"]), ctypes.byref(d["table"]),
+                                    ctypes.byref(d["lens"]), s, cumsum, ctypes.byref(d["key"]),
+                                    ctypes.byref(d["value"]), None)
+
+
+def test_paged_rejects_bad_arguments(lib):
+    a = paged_args()
+    if not torch.cuda.is_available():
+        assert paged_call(lib, a) == 7  # well formed: reaches CUDA
+    b = dict(a, key=torch.zeros(40, 2, 64, dtype=torch.float16))
+    assert paged_call(lib, b) == 2  # output dtype differs from its cache
+    b = dict(a, lens=torch.zeros(3, dtype=torch.int32))
+    assert paged_call(lib, b) == 3  # plain lengths must be [batch]
+    assert paged_call(lib, dict(a, lens=torch.zeros(3, dtype=torch.int32)), cumsum=1) in (0, 7)  # [batch+1] ok
+    b = dict(a, kc=torch.zeros(6, 16, 1, 64, dtype=torch.bfloat16), key=torch.zeros(40, 1, 64, dtype=torch.bfloat16))
+    assert paged_call(lib, b) == 3  # value cache heads differ from key cache heads
+    b = dict(a, kc=torch.zeros(6, 16, 2, 3, dtype=torch.bfloat16), key=torch.zeros(40, 2, 3, dtype=torch.bfloat16))
+    assert paged_call(lib, b) == 4  # 12-byte rows are not whole 16-byte vectors
+    b = dict(a, table=torch.zeros(2, 4, dtype=torch.int64))
+    assert paged_call(lib, b) == 2
+    assert paged_call(lib, a, starts=torch.zeros(3, dtype=torch.int32)) == 3
+    b = dict(a, value=a["key"])
+    assert paged_call(lib, b) == 6  # outputs overlap
