@@ -325,31 +325,11 @@ def reference_arm(args, wl):
 def paged_inputs(wl, block_size, device, seed=7):
     """A paged K/V cache holding the workload's keys: K rows [nope | rope] (192), V rows (128),
     blocks assigned to the sequences in a seeded random order (a fragmented cache)."""
-    import torch
-
     from mla_prefill_attention_varlen_b200 import workloads as W
 
     x = W.make_inputs(wl, device=device)
-    G = wl.kv_head_num
-    kcat = torch.cat([x["k"], x["k_rope"]], dim=2)
-    need = [(L + block_size - 1) // block_size for L in wl.kv_seqlens]
-    nb = sum(need)
-    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(seed))
-    kc = torch.zeros(nb, block_size, G, wl.d_nope + wl.d_rope, dtype=wl.dtype, device=device)
-    vc = torch.zeros(nb, block_size, G, wl.d_nope, dtype=wl.dtype, device=device)
-    table = torch.zeros(len(need), max(need), dtype=torch.int32)
-    used = start = 0
-    for b, L in enumerate(wl.kv_seqlens):
-        idx = perm[used:used + need[b]]
-        table[b, :need[b]] = idx.to(torch.int32)
-        pad = need[b] * block_size - L
-        src_k = torch.nn.functional.pad(kcat[start:start + L], (0, 0, 0, 0, 0, pad))
-        src_v = torch.nn.functional.pad(x["v"][start:start + L], (0, 0, 0, 0, 0, pad))
-        kc[idx.to(device)] = src_k.view(need[b], block_size, G, -1)
-        vc[idx.to(device)] = src_v.view(need[b], block_size, G, -1)
-        used += need[b]
-        start += L
-    return kc, vc, table.to(device), x["kv_seqlen"]
+    kc, vc, table = W.paged_cache(x["k"], x["k_rope"], x["v"], wl.kv_seqlens, block_size, seed=seed)
+    return kc, vc, table, x["kv_seqlen"]
 
 
 def bench_paged(args):
@@ -425,8 +405,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--op", default="prefill", choices=["prefill", "paged_cache_load"])
-    ap.add_argument("--block-size", type=int, default=64, help="paged_cache_load: tokens per cache block")
+    ap.add_argument("--op", default="prefill", choices=["prefill", "prefill_paged", "paged_cache_load"],
+                    help="prefill: mla_prefill on packed K/V; prefill_paged: mla_prefill_paged reading a "
+                         "paged cache in place; paged_cache_load: the gather alone")
+    ap.add_argument("--block-size", type=int, default=64, help="paged ops: tokens per cache block")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: scale head_num and kv_head_num down to this many query heads")
     args = ap.parse_args()
@@ -456,10 +438,23 @@ def main():
     out = torch.empty(wl.t_q, wl.head_num, wl.d_nope, dtype=wl.dtype, device=dev)
     H, G, scale = wl.head_num, wl.kv_head_num, wl.qk_scale
     stream = torch.cuda.current_stream()
+    paged = args.op == "prefill_paged"
+    packed_x = x
+    if paged:
+        kc, vc, table = W.paged_cache(x["k"], x["k_rope"], x["v"], wl.kv_seqlens, args.block_size, seed=7)
+        x = {"q": x["q"], "q_rope": x["q_rope"], "key_cache": kc, "value_cache": vc, "block_tables": table,
+             "q_seqlen": x["q_seqlen"], "kv_seqlen": x["kv_seqlen"]}
+
+    def call(d, o):
+        if paged:
+            mla.mla_prefill_paged(d["q"], d["q_rope"], d["key_cache"], d["value_cache"], d["block_tables"],
+                                  d["q_seqlen"], d["kv_seqlen"], mla.MLA_MASK_CAUSAL, H, G, scale, o, stream)
+        else:
+            mla.mla_prefill(d["q"], d["q_rope"], d["k"], d["k_rope"], d["v"], d["q_seqlen"], d["kv_seqlen"],
+                            mla.MLA_MASK_CAUSAL, H, G, scale, o, stream)
 
     def step(o=out):
-        mla.mla_prefill(x["q"], x["q_rope"], x["k"], x["k_rope"], x["v"], x["q_seqlen"], x["kv_seqlen"],
-                        mla.MLA_MASK_CAUSAL, H, G, scale, o, stream)
+        call(x, o)
 
     in_bytes = sum(t.numel() * t.element_size() for t in x.values())
     flush = None
@@ -523,8 +518,7 @@ def main():
         def e2e_step():
             for k in dx:
                 dx[k].copy_(hx[k], non_blocking=True)
-            mla.mla_prefill(dx["q"], dx["q_rope"], dx["k"], dx["k_rope"], dx["v"], dx["q_seqlen"], dx["kv_seqlen"],
-                            mla.MLA_MASK_CAUSAL, H, G, scale, out, stream)
+            call(dx, out)
             hout.copy_(out, non_blocking=True)
 
         for _ in range(args.warmup):
@@ -548,7 +542,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
 
-        xc = to_numpy_f64({k: v.cpu() for k, v in x.items()})
+        xc = to_numpy_f64({k: v.cpu() for k, v in packed_x.items()})
         dt, trip, desc = time_oracle_sample(wl, xc, args.cpu_seconds)
         cpu_baseline = {"value": trip * FLOPS_PER_TRIPLE / dt / 1e12, "unit": "TFLOP/s",
                         "cores": oracle.core_count(), "kind": "oracle", "sample": desc}
@@ -557,7 +551,8 @@ def main():
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     clocks = smi.summary()
     line = {
-        "metric": "causal MLA prefill TFLOP/s (visible pairs x 640 FLOPs), % of B200 dense bf16 peak, tokens/s",
+        "metric": "causal MLA prefill TFLOP/s (visible pairs x 640 FLOPs), % of B200 dense bf16 peak, tokens/s"
+                  + (" (K/V read in place from a paged cache)" if paged else ""),
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f16", "data": "synthetic",
@@ -566,12 +561,15 @@ def main():
                    "parallelism": "replicas" if world > 1 else "single", "l2": (
                        "flushed between steps (512 MB write)" if flush is not None else
                        "inputs %.2f GB > 126 MB L2" % (in_bytes / 1e9)),
-                   "visible_triples": triples},
+                   "visible_triples": triples,
+                   **({"kv_layout": "paged", "block_size": args.block_size, "blocks": int(x["key_cache"].shape[0])}
+                      if paged else {"kv_layout": "packed"})},
         "pct_of_peak": 100.0 * value / world / peak,
         "tokens_per_s": tokens_per_s,
         "north_star_literal_tflops": 2 * value,
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": kern_tflops / peak, "traffic": measured_traffic(wl.name), "peak_source": peak_src,
+                     "frac": kern_tflops / peak, "traffic": None if paged else measured_traffic(wl.name),
+                     "peak_source": peak_src,
                      "peak_kind": "burst", "frac_of_sustained": kern_tflops / peak_sus,
                      "kernel": "mla_prefill_sm100_kernel", "kernel_ms": kms,
                      "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": algorithmic_bytes(wl)},

@@ -85,8 +85,9 @@ typedef enum {
  *     or all three in the page's padded form [batch, max_seq, G*128] / [batch,
  *     max_seq, G*64] / [batch, max_seq, G*128]: sequence b's keys are rows
  *     0 .. Lk_b-1 of batch entry b (Lk_b <= max_seq); the batch rows must be
- *     dense (batch stride = max_seq * token stride).  A [batch, 1, G*W]
- *     tensor reads the same either way and is taken as packed.
+ *     dense (batch stride = max_seq * token stride).  Rows Lk_b .. max_seq-1
+ *     never reach the result, whatever they hold (NaN and Inf included).
+ *     A [batch, 1, G*W] tensor reads the same either way and is taken as packed.
  *   q_seqlen, kv_seqlen  [batch] MLA_I32 in DEVICE memory (page: qSeqLen / kvSeqLen rows).
  *     Sequence b owns query tokens [sum_{b'<b} Lq_b', + Lq_b) and key tokens
  *     [sum_{b'<b} Lk_b', + Lk_b) of the packed tensors.
@@ -127,7 +128,7 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
  * mla_prefill_device_status -- synchronises `stream`, then reads and clears the
  * device status word of the current GPU (MLA_OK, MLA_ERR_SEQLEN,
  * MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_INDEX; the first error recorded since the
- * last read by mla_prefill or mla_paged_cache_load).
+ * last read by mla_prefill, mla_prefill_paged or mla_paged_cache_load).
  * Writes it to *status and returns MLA_OK, or returns MLA_ERR_NULL /
  * MLA_ERR_CUDA.
  */
@@ -209,6 +210,46 @@ int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope, const mla
 int mla_paged_cache_load(const mla_tensor *key_cache, const mla_tensor *value_cache, const mla_tensor *block_tables,
                          const mla_tensor *context_lens, const mla_tensor *seq_starts, int context_lens_cumsum,
                          mla_tensor *key, mla_tensor *value, mla_stream_t stream);
+
+/*
+ * mla_prefill_paged -- mla_prefill with K, K_rope and V read in place from
+ * block-paged caches through a block table: the composition of the
+ * PagedCacheLoadOperation page's gather (ND format, plain lengths, no
+ * seqStarts) with the MLA Prefill page's attention, without the packed copy.
+ * Its result is bit-identical to mla_paged_cache_load into packed key / value
+ * tensors followed by mla_prefill on them.
+ *
+ *   q, q_rope, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num,
+ *   qk_scale, out   exactly as in mla_prefill.
+ *   key_cache    [num_blocks, block_size, G, 192]: per slot and kv head the
+ *                128 K_nope channels followed by the 64 K_rope channels
+ *                (page: keyCache, ND).
+ *   value_cache  [num_blocks, block_size, G, 128] (page: valueCache, ND).
+ *                Both of q's dtype; last dimension contiguous; block, slot
+ *                and head strides positive multiples of 8 elements; base
+ *                pointers 16-byte aligned; the two caches agree in
+ *                num_blocks and block_size.
+ *   block_size   a multiple of 8 that divides 128, or a multiple of 128
+ *                (8, 16, 32, 64, 128, 256, ...); else MLA_ERR_UNSUPPORTED.
+ *   block_tables [batch, W] MLA_I32 (page: blockTables): key j < Lk_b of
+ *                sequence b is slot j % block_size of physical block
+ *                block_tables[b][j / block_size].  Lk_b <= W * block_size
+ *                (else clamped, MLA_ERR_SEQLEN).  Entries for blocks wholly
+ *                past Lk_b are never read; slots past Lk_b in the last block
+ *                may hold anything (NaN and Inf included).
+ *
+ * All tensors are caller-owned device memory; `out` must not overlap the
+ * queries or the caches.  Argument errors return before any launch.
+ * Device-detected: MLA_ERR_SEQLEN as in mla_prefill, and a visible key whose
+ * block id lies outside [0, num_blocks) (its K and V rows read as zeros,
+ * MLA_ERR_INDEX); read them with mla_prefill_device_status.  Shares the
+ * per-GPU workspace with mla_prefill: order both on one stream.
+ * Returns MLA_OK or an mla_status error code.
+ */
+int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *key_cache,
+                      const mla_tensor *value_cache, const mla_tensor *block_tables, const mla_tensor *q_seqlen,
+                      const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num, float qk_scale,
+                      mla_tensor *out, mla_stream_t stream);
 
 /* A static, human-readable name for a status code (never NULL). */
 const char *mla_status_string(int status);

@@ -13,7 +13,8 @@ from . import workloads  # noqa: F401  (seeded synthetic inputs)
 
 __all__ = [
     "MLA_MASK_NONE", "MLA_MASK_CAUSAL", "MlaError", "load_library", "mla_prefill", "mla_prefill_noalloc",
-    "mla_paged_cache_load", "mla_prefill_device_status", "mla_status_string", "prefill", "workloads",
+    "mla_paged_cache_load", "mla_prefill_paged", "mla_prefill_device_status", "mla_status_string", "prefill",
+    "workloads",
 ]
 
 MLA_F16, MLA_BF16, MLA_I32, MLA_I8 = 0, 1, 2, 3
@@ -64,6 +65,9 @@ def load_library(path=None):
     lib.mla_prefill_noalloc.restype = ctypes.c_int
     lib.mla_paged_cache_load.argtypes = [T, T, T, T, T, ctypes.c_int, T, T, ctypes.c_void_p]
     lib.mla_paged_cache_load.restype = ctypes.c_int
+    lib.mla_prefill_paged.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                      T, ctypes.c_void_p]
+    lib.mla_prefill_paged.restype = ctypes.c_int
     lib.mla_prefill_set_profile_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.mla_prefill_set_profile_events.restype = ctypes.c_int
     lib.mla_prefill_version.argtypes = []
@@ -167,6 +171,20 @@ def mla_paged_cache_load(key_cache, value_cache, block_tables, context_lens, key
     if rc != 0:
         raise MlaError(rc, "mla_paged_cache_load")
     return key, value
+
+
+def mla_prefill_paged(q, q_rope, key_cache, value_cache, block_tables, q_seqlen, kv_seqlen, mask_type, head_num,
+                      kv_head_num, qk_scale, out, stream=None):
+    """Call the C ABI ``mla_prefill_paged``: prefill attention reading K / K_rope / V in place from
+    paged caches (key_cache [blocks, block_size, G, 192] = K_nope | K_rope, value_cache
+    [blocks, block_size, G, 128]) through block_tables [batch, W]."""
+    lib = load_library()
+    d = [as_mla_tensor(t) for t in (q, q_rope, key_cache, value_cache, block_tables, q_seqlen, kv_seqlen, out)]
+    rc = lib.mla_prefill_paged(*(ctypes.byref(x) for x in d[:7]), int(mask_type), int(head_num), int(kv_head_num),
+                               float(qk_scale), ctypes.byref(d[7]), _stream_handle(stream, q.device))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_paged")
+    return out
 
 
 def set_profile_events(start=None, stop=None):

@@ -25,7 +25,7 @@ struct DeviceState {
     int *status = nullptr;  // sticky device status word (own 256-byte allocation)
     void *ws = nullptr;     // plan workspace
     size_t ws_bytes = 0;
-    bool attr_set[8] = {};  // dynamic shared memory opt-in done, per kernel instantiation
+    bool attr_set[16] = {};  // dynamic shared memory opt-in done, per kernel instantiation
 };
 
 std::mutex g_mu;
@@ -146,6 +146,23 @@ int encode_map(CUtensorMap *m, const View3 &v, bool bf16, void *dummy, int box_t
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_UNSUPPORTED;
 }
 
+// 4-D map over a paged cache {channels, heads, slots, blocks} with a
+// {64, 1, box_rows, 1} box and 128-byte swizzle.
+int encode_cache_map(CUtensorMap *m, const void *data, int64_t blocks, int64_t slots, int64_t heads, int64_t channels,
+                     int64_t block_bytes, int64_t slot_bytes, int64_t head_bytes, bool bf16, int box_rows) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(channels), static_cast<cuuint64_t>(heads),
+                                static_cast<cuuint64_t>(slots), static_cast<cuuint64_t>(blocks)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(head_bytes), static_cast<cuuint64_t>(slot_bytes),
+                                   static_cast<cuuint64_t>(block_bytes)};
+    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                          const_cast<void *>(data), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_UNSUPPORTED;
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
@@ -201,10 +218,10 @@ int device_state(int dev, cudaStream_t stream, size_t ws_need, DeviceState **out
     return MLA_OK;
 }
 
-template <typename T, bool kCausal, bool kPos>
+template <typename T, bool kCausal, bool kPos, bool kKvAny>
 int launch_attention(DeviceState *ds, int slot, int grid, cudaStream_t stream, const CUtensorMap (&maps)[5],
                      const mla::Params &p) {
-    auto kern = mla::mla_prefill_sm100_kernel<T, kCausal, kPos>;
+    auto kern = mla::mla_prefill_sm100_kernel<T, kCausal, kPos, kKvAny>;
     if (!ds->attr_set[slot]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kSmemAlloc) != cudaSuccess)
             return MLA_ERR_CUDA;
@@ -223,15 +240,22 @@ struct Problem {
     const int *q_seqlen, *kv_seqlen;
     int64_t batch;
     int64_t kv_pad;  // 0: packed K/V; else the padded layout's max_seq
+    // paged K/V (mla_prefill_paged): caches [blocks, block_size, G, 192 | 128] and the block table
+    bool paged = false;
+    const void *key_cache = nullptr, *value_cache = nullptr;
+    int64_t num_blocks = 0, block_size = 0, table_width = 0, table_stride = 0;
+    int64_t kc_block = 0, kc_slot = 0, kc_head = 0, vc_block = 0, vc_slot = 0, vc_head = 0;
+    const int *tables = nullptr;
     bool bf16, causal;
     int head_num, kv_head_num;
     float qk_scale;
 };
 
-int validate(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
-             const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
-             int head_num, int kv_head_num, float qk_scale, const mla_tensor *out, Problem *pr) {
-    if (!q || !q_rope || !k || !k_rope || !v || !q_seqlen || !kv_seqlen || !out) return MLA_ERR_NULL;
+// Arguments every prefill entry point shares: queries, output, seqlens, scalars.
+int validate_common(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *q_seqlen,
+                    const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num, float qk_scale,
+                    const mla_tensor *out, Problem *pr) {
+    if (!q || !q_rope || !q_seqlen || !kv_seqlen || !out) return MLA_ERR_NULL;
     if (head_num < 1 || kv_head_num < 1 || head_num % kv_head_num != 0) return MLA_ERR_HEADS;
     if (mask_type != MLA_MASK_CAUSAL && mask_type != MLA_MASK_NONE) return MLA_ERR_UNSUPPORTED;
     if (!std::isfinite(qk_scale)) return MLA_ERR_UNSUPPORTED;
@@ -252,6 +276,28 @@ int validate(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
     if ((rc = view3(q, dt, head_num, mla::kDn, &pr->q)) != MLA_OK) return rc;
     if ((rc = view3(q_rope, dt, head_num, mla::kDr, &pr->qr)) != MLA_OK) return rc;
     if ((rc = view3(out, dt, head_num, mla::kDn, &pr->o)) != MLA_OK) return rc;
+    if (pr->qr.tokens != pr->q.tokens || pr->o.tokens != pr->q.tokens) return MLA_ERR_SHAPE;
+    for (const View3 *in : {&pr->q, &pr->qr})
+        if (overlaps(pr->o, *in)) return MLA_ERR_UNSUPPORTED;
+    pr->q_seqlen = static_cast<const int *>(q_seqlen->data);
+    pr->kv_seqlen = static_cast<const int *>(kv_seqlen->data);
+    pr->batch = batch;
+    pr->bf16 = dt == MLA_BF16;
+    pr->causal = mask_type == MLA_MASK_CAUSAL;
+    pr->head_num = head_num;
+    pr->kv_head_num = kv_head_num;
+    pr->qk_scale = qk_scale;
+    return MLA_OK;
+}
+
+int validate(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+             const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+             int head_num, int kv_head_num, float qk_scale, const mla_tensor *out, Problem *pr) {
+    if (!k || !k_rope || !v) return MLA_ERR_NULL;
+    int rc = validate_common(q, q_rope, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out, pr);
+    if (rc != MLA_OK) return rc;
+    const int dt = q->dtype;
+    const int64_t batch = pr->batch;
     const bool pk = is_padded_kv(k, kv_head_num, mla::kDn), pkr = is_padded_kv(k_rope, kv_head_num, mla::kDr),
                pv = is_padded_kv(v, kv_head_num, mla::kDn);
     pr->kv_pad = 0;
@@ -268,20 +314,9 @@ int validate(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
         if ((rc = view3(k_rope, dt, kv_head_num, mla::kDr, &pr->kr)) != MLA_OK) return rc;
         if ((rc = view3(v, dt, kv_head_num, mla::kDn, &pr->v)) != MLA_OK) return rc;
     }
-    if (pr->qr.tokens != pr->q.tokens || pr->o.tokens != pr->q.tokens || pr->kr.tokens != pr->k.tokens ||
-        pr->v.tokens != pr->k.tokens)
-        return MLA_ERR_SHAPE;
-    for (const View3 *in : {&pr->q, &pr->qr, &pr->k, &pr->kr, &pr->v})
+    if (pr->kr.tokens != pr->k.tokens || pr->v.tokens != pr->k.tokens) return MLA_ERR_SHAPE;
+    for (const View3 *in : {&pr->k, &pr->kr, &pr->v})
         if (overlaps(pr->o, *in)) return MLA_ERR_UNSUPPORTED;
-
-    pr->q_seqlen = static_cast<const int *>(q_seqlen->data);
-    pr->kv_seqlen = static_cast<const int *>(kv_seqlen->data);
-    pr->batch = batch;
-    pr->bf16 = dt == MLA_BF16;
-    pr->causal = mask_type == MLA_MASK_CAUSAL;
-    pr->head_num = head_num;
-    pr->kv_head_num = kv_head_num;
-    pr->qk_scale = qk_scale;
     return MLA_OK;
 }
 
@@ -295,9 +330,22 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     CUtensorMap maps[5];
     if ((rc = encode_map(&maps[0], pr.q, pr.bf16, ws, 128)) != MLA_OK) return rc;
     if ((rc = encode_map(&maps[1], pr.qr, pr.bf16, ws, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[2], pr.k, pr.bf16, ws, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[3], pr.kr, pr.bf16, ws, 128)) != MLA_OK) return rc;
-    if ((rc = encode_map(&maps[4], pr.v, pr.bf16, ws, 64)) != MLA_OK) return rc;
+    const int rows_k = static_cast<int>(pr.block_size < mla::kBN ? pr.block_size : mla::kBN);
+    const int rows_v = static_cast<int>(pr.block_size < 64 ? pr.block_size : 64);
+    if (pr.paged) {
+        const int64_t G = pr.kv_head_num;
+        if ((rc = encode_cache_map(&maps[2], pr.key_cache, pr.num_blocks, pr.block_size, G, mla::kDn + mla::kDr,
+                                   pr.kc_block, pr.kc_slot, pr.kc_head, pr.bf16, rows_k)) != MLA_OK)
+            return rc;
+        maps[3] = maps[2];
+        if ((rc = encode_cache_map(&maps[4], pr.value_cache, pr.num_blocks, pr.block_size, G, mla::kDn,
+                                   pr.vc_block, pr.vc_slot, pr.vc_head, pr.bf16, rows_v)) != MLA_OK)
+            return rc;
+    } else {
+        if ((rc = encode_map(&maps[2], pr.k, pr.bf16, ws, 128)) != MLA_OK) return rc;
+        if ((rc = encode_map(&maps[3], pr.kr, pr.bf16, ws, 128)) != MLA_OK) return rc;
+        if ((rc = encode_map(&maps[4], pr.v, pr.bf16, ws, 64)) != MLA_OK) return rc;
+    }
 
     int *num_units = reinterpret_cast<int *>(ws + lay.num_units);
     int *work_counter = num_units + 1;  // second word of the 16-byte header
@@ -308,7 +356,8 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
 
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
         pr.q_seqlen, pr.kv_seqlen, static_cast<int>(pr.batch), pr.q.tokens, pr.k.tokens, pr.kv_pad,
-        pr.causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter, status);
+        pr.paged ? 1 : 0, pr.causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
+        status);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
     mla::Params p;
@@ -323,23 +372,31 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     p.head_num = pr.head_num;
     p.group = pr.head_num / pr.kv_head_num;
     p.scale_log2 = pr.qk_scale * 1.4426950408889634f;
+    p.tables = pr.tables;
+    p.table_stride = pr.table_stride;
+    p.table_width = static_cast<int>(pr.table_width);
+    p.num_blocks = static_cast<int>(pr.num_blocks);
+    p.block_size = static_cast<int>(pr.block_size > 0 ? pr.block_size : 1);
+    p.rows_k = rows_k > 0 ? rows_k : 1;
+    p.rows_v = rows_v > 0 ? rows_v : 1;
+    p.paged = pr.paged ? 1 : 0;
+    const bool kv_any = pr.paged || pr.kv_pad > 0;  // padded or paged K/V
 
     const int64_t max_items = ((pr.q.tokens + mla::kUnitRows - 1) / mla::kUnitRows + pr.batch) * pr.head_num;
     const int grid = static_cast<int>(max_items < sm_count ? max_items : sm_count);
     const bool pos = pr.qk_scale > 0.f;
     DeviceState *ls = launch_flags;
+    const int slot = (pr.bf16 ? 0 : 4) + (pr.causal ? 0 : 2) + (pos ? 0 : 1) + (kv_any ? 8 : 0);
+#define MLA_LAUNCH(T, C, P, G) launch_attention<T, C, P, G>(ls, slot, grid, stream, maps, p)
+#define MLA_PICK(T, C, P) (kv_any ? MLA_LAUNCH(T, C, P, true) : MLA_LAUNCH(T, C, P, false))
     if (pr.bf16) {
-        if (pr.causal)
-            return pos ? launch_attention<__nv_bfloat16, true, true>(ls, 0, grid, stream, maps, p)
-                       : launch_attention<__nv_bfloat16, true, false>(ls, 1, grid, stream, maps, p);
-        return pos ? launch_attention<__nv_bfloat16, false, true>(ls, 2, grid, stream, maps, p)
-                   : launch_attention<__nv_bfloat16, false, false>(ls, 3, grid, stream, maps, p);
+        if (pr.causal) return pos ? MLA_PICK(__nv_bfloat16, true, true) : MLA_PICK(__nv_bfloat16, true, false);
+        return pos ? MLA_PICK(__nv_bfloat16, false, true) : MLA_PICK(__nv_bfloat16, false, false);
     }
-    if (pr.causal)
-        return pos ? launch_attention<__half, true, true>(ls, 4, grid, stream, maps, p)
-                   : launch_attention<__half, true, false>(ls, 5, grid, stream, maps, p);
-    return pos ? launch_attention<__half, false, true>(ls, 6, grid, stream, maps, p)
-               : launch_attention<__half, false, false>(ls, 7, grid, stream, maps, p);
+    if (pr.causal) return pos ? MLA_PICK(__half, true, true) : MLA_PICK(__half, true, false);
+    return pos ? MLA_PICK(__half, false, true) : MLA_PICK(__half, false, false);
+#undef MLA_PICK
+#undef MLA_LAUNCH
 }
 
 }  // namespace
@@ -642,4 +699,89 @@ extern "C" int mla_paged_cache_load(const mla_tensor *key_cache, const mla_tenso
     const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
     mla::paged_gather_kernel<<<grid, mla::kGatherThreads, 0, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Prefill reading K / K_rope / V in place from paged caches
+// ---------------------------------------------------------------------------
+namespace {
+
+// A [blocks, block_size, G, W] cache of the query dtype, read by 4-D TMA maps.
+int attention_cache(const mla_tensor *t, int dtype, int64_t heads, int64_t width, int64_t *blocks,
+                    int64_t *block_size, int64_t *bb, int64_t *sb, int64_t *hb) {
+    if (!t || !t->data) return MLA_ERR_NULL;
+    if (t->dtype != dtype) return MLA_ERR_DTYPE;
+    if (t->ndim != 4 || t->shape[2] != heads || t->shape[3] != width) return MLA_ERR_SHAPE;
+    if (t->shape[0] < 1 || t->shape[0] > INT32_MAX || t->shape[1] < 1) return MLA_ERR_SHAPE;
+    if (t->stride[3] != 1) return MLA_ERR_ALIGN;
+    *blocks = t->shape[0];
+    *block_size = t->shape[1];
+    *bb = t->stride[0] * 2;
+    *sb = t->stride[1] * 2;
+    *hb = (heads > 1 ? t->stride[2] : width) * 2;
+    if (!aligned16(t->data) || *bb % 16 || *sb % 16 || *hb % 16 || *bb <= 0 || *sb <= 0 || *hb <= 0)
+        return MLA_ERR_ALIGN;
+    if (*bb >= (int64_t(1) << 40) || *sb >= (int64_t(1) << 40) || *hb >= (int64_t(1) << 40))
+        return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *key_cache,
+                                 const mla_tensor *value_cache, const mla_tensor *block_tables,
+                                 const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type, int head_num,
+                                 int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!key_cache || !value_cache || !block_tables) return MLA_ERR_NULL;
+    Problem pr;
+    int rc = validate_common(q, q_rope, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out, &pr);
+    if (rc != MLA_OK) return rc;
+    const int dt = q->dtype;
+    int64_t nb, bs, nbv, bsv;
+    if ((rc = attention_cache(key_cache, dt, kv_head_num, mla::kDn + mla::kDr, &nb, &bs, &pr.kc_block, &pr.kc_slot,
+                              &pr.kc_head)) != MLA_OK)
+        return rc;
+    if ((rc = attention_cache(value_cache, dt, kv_head_num, mla::kDn, &nbv, &bsv, &pr.vc_block, &pr.vc_slot,
+                              &pr.vc_head)) != MLA_OK)
+        return rc;
+    if (nbv != nb || bsv != bs) return MLA_ERR_SHAPE;
+    // a block holds whole 8-row swizzle atoms, and a 128-key tile covers whole blocks (or lies in one)
+    if (bs % 8 != 0 || (bs <= mla::kBN ? mla::kBN % bs != 0 : bs % mla::kBN != 0)) return MLA_ERR_UNSUPPORTED;
+    if (block_tables->dtype != MLA_I32) return MLA_ERR_DTYPE;
+    if (block_tables->ndim != 2 || block_tables->shape[0] != pr.batch) return MLA_ERR_SHAPE;
+    const int64_t width = block_tables->shape[1];
+    if (width < 0 || width * bs > INT32_MAX) return MLA_ERR_SHAPE;
+    if (pr.batch > 0 && width > 0 && !block_tables->data) return MLA_ERR_NULL;
+    if (width > 1 && block_tables->stride[1] != 1) return MLA_ERR_ALIGN;
+    if (pr.batch > 1 && block_tables->stride[0] < width) return MLA_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(block_tables->data) & 3u) return MLA_ERR_ALIGN;
+    // out must not overlap the caches
+    uintptr_t olo, ohi;
+    byte_range(pr.o, &olo, &ohi);
+    const uintptr_t klo = reinterpret_cast<uintptr_t>(key_cache->data),
+                    khi = klo + (nb - 1) * pr.kc_block + (bs - 1) * pr.kc_slot + (kv_head_num - 1) * pr.kc_head + 384;
+    const uintptr_t vlo = reinterpret_cast<uintptr_t>(value_cache->data),
+                    vhi = vlo + (nb - 1) * pr.vc_block + (bs - 1) * pr.vc_slot + (kv_head_num - 1) * pr.vc_head + 256;
+    if ((olo < khi && klo < ohi) || (olo < vhi && vlo < ohi)) return MLA_ERR_UNSUPPORTED;
+
+    pr.paged = true;
+    pr.key_cache = key_cache->data;
+    pr.value_cache = value_cache->data;
+    pr.num_blocks = nb;
+    pr.block_size = bs;
+    pr.table_width = width;
+    pr.table_stride = pr.batch > 1 ? block_tables->stride[0] : width;
+    pr.tables = static_cast<const int *>(block_tables->data);
+    pr.kv_pad = width * bs;  // per-sequence key capacity of the table
+    pr.k.tokens = width * bs;
+    if (pr.batch == 0 || pr.q.tokens == 0) return MLA_OK;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const WsLayout lay = ws_layout(pr.batch, pr.q.tokens, pr.k.tokens);
+    DeviceState *ds = nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if ((rc = device_state(dev, stream, lay.total, &ds)) != MLA_OK) return rc;
+    return enqueue(pr, lay, static_cast<uint8_t *>(ds->ws), ds->status, ds->sm_count, ds, stream);
 }

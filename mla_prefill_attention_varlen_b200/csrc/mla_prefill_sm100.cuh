@@ -35,6 +35,7 @@
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "sm100_ptx.cuh"
 
@@ -76,6 +77,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a pipeline wait gives up af
 // Status codes the device writes (mirror mla_status in include/mla_prefill.h).
 constexpr int kStatusSeqlen = 8;
 constexpr int kStatusTimeout = 9;
+constexpr int kStatusIndex = 10;
 
 struct Params {
     const int4 *seq_info;  // per sequence {cq, ck, lq, lk} after clamping
@@ -88,6 +90,12 @@ struct Params {
     int head_num;
     int group;         // head_num / kv_head_num
     float scale_log2;  // qk_scale * log2(e)
+    // paged K/V only: logical block i of sequence b is physical block tables[b * table_stride + i]
+    const int *tables;
+    long long table_stride;
+    int table_width, num_blocks, block_size;
+    int rows_k, rows_v;  // tokens per TMA box: min(128, block_size), min(64, block_size)
+    int paged;  // K/V read from paged caches through the block table (kKvAny kernels only)
 };
 
 struct Barriers {
@@ -121,6 +129,7 @@ __host__ __device__ __forceinline__ int unit_cost(int u0, int lq, int lk, bool c
 }
 
 struct WorkItem {
+    int b;  // sequence
     int h, kh;
     int u0;              // first query row of the unit within its sequence
     int q_tok0, k_tok0;  // first packed token of the unit / of the sequence's keys
@@ -142,6 +151,7 @@ __device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num
     const int u = rem / p.group;
     x.h = x.kh * p.group + (rem - u * p.group);
     const int2 bm = p.units[u];
+    x.b = bm.x;
     const int4 s = p.seq_info[bm.x];
     x.u0 = bm.y * kUnitRows;
     x.q_tok0 = s.x + x.u0;
@@ -248,7 +258,7 @@ __device__ __forceinline__ int seq_of_unit(const int *unit_off, int batch, int t
 __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__restrict__ q_seqlen,
                                                                 const int *__restrict__ kv_seqlen, int batch,
                                                                 long long t_q, long long t_k, long long kv_pad,
-                                                                int causal,
+                                                                int paged, int causal,
                                                                 int4 *seq_info, int *unit_off, int *hist,
                                                                 int hist_len, int2 *units, int *num_units,
                                                                 int *work_counter, int *status) {
@@ -274,7 +284,8 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
         const long long pk = carry_k + block_exclusive_scan(lk, tot_k, warp_sums);
         const long long cq = pq < t_q ? pq : t_q, eq = pq + lq < t_q ? pq + lq : t_q;
         // packed K/V: sequences follow each other; padded K/V: sequence b starts at b * kv_pad
-        const long long kb = kv_pad ? (long long)b * kv_pad : pk;
+        // paged K/V: keys are addressed through the block table; kv_pad is the table's capacity
+        const long long kb = paged ? 0 : (kv_pad ? (long long)b * kv_pad : pk);
         const long long kcap = kv_pad ? kb + kv_pad : t_k;
         const long long ck = kb < t_k ? kb : t_k, ek = kb + lk < kcap ? (kb + lk < t_k ? kb + lk : t_k) : (kcap < t_k ? kcap : t_k);
         if (b < batch && (eq - cq != lq || ek - ck != lk)) bad = 1;
@@ -353,7 +364,10 @@ __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
 // ---------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------
-template <typename T, bool kCausal, bool kPositiveScale>
+// kKvAny: padded or paged K/V, where rows of the last key tile past Lk may hold anything
+// (padding, unwritten cache slots).  Packed K/V (kKvAny = false) has only real keys or
+// TMA's zero fill there.
+template <typename T, bool kCausal, bool kPositiveScale, bool kKvAny>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
@@ -404,85 +418,159 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 4) {
         ptx::regs_dec<kRegsLow>();
-        if (warp == 0 && lane == 0) {
+        if (warp == 0) {
             // -------------------------------------------------------- TMA producer
-            ptx::tma_prefetch_desc(&tm_q);
-            ptx::tma_prefetch_desc(&tm_qr);
-            ptx::tma_prefetch_desc(&tm_k);
-            ptx::tma_prefetch_desc(&tm_kr);
-            ptx::tma_prefetch_desc(&tm_v);
-            const uint64_t pol_q = ptx::policy_evict_first();
-            const uint64_t pol_kv = ptx::policy_evict_last();
-            uint32_t rc = 0;                // ring chunks filled
-            uint32_t ql0 = 0, ql1 = 0;      // Q tiles loaded per tile slot
-            bool ok = true;
-            auto next_chunk = [&](uint32_t &dst, uint32_t &fb) -> bool {
-                const uint32_t slot = rc % kRing;
-                if (!wait_bar(bar(bars->ch_empty[slot]), ((rc / kRing) & 1) ^ 1, bars, p.status)) return false;
-                dst = sRing + slot * kChunkBytes;
-                fb = bar(bars->ch_full[slot]);
-                ptx::mbar_arrive_expect_tx(fb, kChunkBytes);
-                ++rc;
-                return true;
-            };
-            // Dynamic scheduling: the first item is blockIdx.x, later ones come from a global
-            // counter; each claimed item index (or -1 at the end) is handed to the MMA and
-            // softmax warps through a small ring in shared memory.
-            uint32_t sc = 0;
-            int next = blockIdx.x < n_items ? (int)blockIdx.x : -1;
-            while (ok) {
-                const int it = next;
-                const uint32_t slot = sc % kSched;
-                ok = wait_bar(bar(bars->sched_empty[slot]), ((sc / kSched) & 1) ^ 1, bars, p.status);
-                if (!ok) break;
-                *reinterpret_cast<volatile int *>(&bars->sched_item[slot]) = it;
-                ptx::mbar_arrive(bar(bars->sched_full[slot]));
-                ++sc;
-                if (it < 0) break;
-                next = (int)gridDim.x + atomicAdd(p.work_counter, 1);
-                if (next >= n_items) next = -1;
-                const WorkItem x = decode_item(p, it, num_units, kCausal);
-                if (x.n_max == 0) continue;
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (!ok || x.n[t] == 0) continue;
-                    uint32_t &ql = t ? ql1 : ql0;
-                    // Q_t of the previous unit is free once its last S_t MMA has completed.
-                    ok = wait_bar(bar(bars->q_empty[t]), (ql & 1) ^ 1, bars, p.status);
-                    if (!ok) continue;
-                    const uint32_t fb = bar(bars->q_full[t]);
-                    const uint32_t dst = sQ + t * kQTileBytes;
-                    const int tok = x.q_tok0 + t * kBM;
-                    ptx::mbar_arrive_expect_tx(fb, kQTileBytes);
-                    ptx::tma_load_3d(dst, &tm_q, fb, 0, x.h, tok, pol_q);
-                    ptx::tma_load_3d(dst + kChunkBytes, &tm_q, fb, 64, x.h, tok, pol_q);
-                    ptx::tma_load_3d(dst + 2 * kChunkBytes, &tm_qr, fb, 0, x.h, tok, pol_q);
-                    ++ql;
+            // Lane 0 alone for packed and padded K/V.  For paged K/V the whole warp runs the
+            // loop (its state is warp-uniform): lane e looks up physical block e of a key tile
+            // (one tile ahead), and lane r issues the r-th TMA box of a chunk, so the work per
+            // tile does not grow as the blocks get smaller.
+            auto producer = [&](auto warp_wide) {
+                constexpr bool kW = decltype(warp_wide)::value;
+                const bool lead = !kW || lane == 0;
+                auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+                    return kW ? wait_bar_warp(b, parity, bars, p.status) : wait_bar(b, parity, bars, p.status);
+                };
+                if (lead) {
+                    ptx::tma_prefetch_desc(&tm_q);
+                    ptx::tma_prefetch_desc(&tm_qr);
+                    ptx::tma_prefetch_desc(&tm_k);
+                    ptx::tma_prefetch_desc(&tm_kr);
+                    ptx::tma_prefetch_desc(&tm_v);
                 }
-                for (int j = 0; j < x.n_max && ok; ++j) {
-                    const int tok = x.k_tok0 + j * kBN;
-                    uint32_t dst, fb;
-                    // K_j: nope cols 0-63, nope cols 64-127, rope
-                    if (!(ok = next_chunk(dst, fb))) break;
-                    ptx::tma_load_3d(dst, &tm_k, fb, 0, x.kh, tok, pol_kv);
-                    if (!(ok = next_chunk(dst, fb))) break;
-                    ptx::tma_load_3d(dst, &tm_k, fb, 64, x.kh, tok, pol_kv);
-                    if (!(ok = next_chunk(dst, fb))) break;
-                    ptx::tma_load_3d(dst, &tm_kr, fb, 0, x.kh, tok, pol_kv);
-                    // V_j: keys 0-63, keys 64-127; each chunk holds V cols 0-63 then 64-127
-                    for (int hh = 0; hh < kVChunks && ok; ++hh) {
-                        if (!(ok = next_chunk(dst, fb))) break;
-                        ptx::tma_load_3d(dst, &tm_v, fb, 0, x.kh, tok + hh * 64, pol_kv);
-                        ptx::tma_load_3d(dst + kVHalfBytes, &tm_v, fb, 64, x.kh, tok + hh * 64, pol_kv);
+                const uint64_t pol_q = ptx::policy_evict_first();
+                const uint64_t pol_kv = ptx::policy_evict_last();
+                uint32_t rc = 0;            // ring chunks filled
+                uint32_t ql0 = 0, ql1 = 0;  // Q tiles loaded per tile slot
+                bool ok = true;
+                auto next_chunk = [&](uint32_t &dst, uint32_t &fb) -> bool {
+                    const uint32_t slot = rc % kRing;
+                    if (!wait(bar(bars->ch_empty[slot]), ((rc / kRing) & 1) ^ 1)) return false;
+                    dst = sRing + slot * kChunkBytes;
+                    fb = bar(bars->ch_full[slot]);
+                    if (lead) ptx::mbar_arrive_expect_tx(fb, kChunkBytes);
+                    ++rc;
+                    return true;
+                };
+                // Dynamic scheduling: the first item is blockIdx.x, later ones come from a global
+                // counter; each claimed item index (or -1 at the end) is handed to the MMA and
+                // softmax warps through a small ring in shared memory.
+                uint32_t sc = 0;
+                int next = blockIdx.x < n_items ? (int)blockIdx.x : -1;
+                while (ok) {
+                    const int it = next;
+                    const uint32_t slot = sc % kSched;
+                    ok = wait(bar(bars->sched_empty[slot]), ((sc / kSched) & 1) ^ 1);
+                    if (!ok) break;
+                    if (lead) {
+                        *reinterpret_cast<volatile int *>(&bars->sched_item[slot]) = it;
+                        ptx::mbar_arrive(bar(bars->sched_full[slot]));
+                    }
+                    ++sc;
+                    if (it < 0) break;
+                    if (lead) {
+                        next = (int)gridDim.x + atomicAdd(p.work_counter, 1);
+                        if (next >= n_items) next = -1;
+                    }
+                    if (kW) next = __shfl_sync(0xffffffffu, next, 0);
+                    const WorkItem x = decode_item(p, it, num_units, kCausal);
+                    if (x.n_max == 0) continue;
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (!ok || x.n[t] == 0) continue;
+                        uint32_t &ql = t ? ql1 : ql0;
+                        // Q_t of the previous unit is free once its last S_t MMA has completed.
+                        ok = wait(bar(bars->q_empty[t]), (ql & 1) ^ 1);
+                        if (!ok) continue;
+                        const uint32_t fb = bar(bars->q_full[t]);
+                        const uint32_t dst = sQ + t * kQTileBytes;
+                        const int tok = x.q_tok0 + t * kBM;
+                        if (lead) {
+                            ptx::mbar_arrive_expect_tx(fb, kQTileBytes);
+                            ptx::tma_load_3d(dst, &tm_q, fb, 0, x.h, tok, pol_q);
+                            ptx::tma_load_3d(dst + kChunkBytes, &tm_q, fb, 64, x.h, tok, pol_q);
+                            ptx::tma_load_3d(dst + 2 * kChunkBytes, &tm_qr, fb, 0, x.h, tok, pol_q);
+                        }
+                        ++ql;
+                    }
+                    if constexpr (kW) {
+                        // Paged caches.  Key tile j spans `per` logical blocks (128 / block_size, or 1
+                        // for blocks of 128 keys or more); lane e < per holds the physical id of block
+                        // e.  A block wholly past Lk, or one without a valid id, becomes block
+                        // num_blocks: out of the map, so TMA fills its boxes with zeros and reads nothing.
+                        const int bs = p.block_size;
+                        const int per = bs < kBN ? kBN / bs : 1;
+                        auto first_key = [&](int j) { return max((j * kBN / bs + lane) * bs, j * kBN); };
+                        auto raw_id = [&](int j) -> int {  // issues the table load; checked when used
+                            const int lb = j * kBN / bs + lane;
+                            if (lane >= per || first_key(j) >= x.lk) return p.num_blocks;
+                            return lb < p.table_width ? __ldg(p.tables + (long long)x.b * p.table_stride + lb) : -1;
+                        };
+                        // `count` TMA boxes of `rows` keys each, from logical position pos0 (a multiple
+                        // of rows); box r comes from one block and lands on whole 1 KB swizzle atoms.
+                        auto boxes = [&](int id, int j, uint32_t dst, const void *map, uint32_t fb, int c0, int pos0,
+                                         int rows, int count) {
+                            const int r = lane < count ? lane : 0;
+                            const int pos = pos0 + r * rows;
+                            const int lb = pos / bs;
+                            const int blk = __shfl_sync(0xffffffffu, id, lb - j * kBN / bs);
+                            if (lane < count)
+                                ptx::tma_load_4d(dst + r * rows * 128, map, fb, c0, x.kh, pos - lb * bs, blk, pol_kv);
+                        };
+                        const int nk = kBN / p.rows_k, nv = 64 / p.rows_v;
+                        int id_next = raw_id(0);
+                        for (int j = 0; j < x.n_max && ok; ++j) {
+                            int id = id_next;
+                            if (j + 1 < x.n_max) id_next = raw_id(j + 1);  // in flight during tile j
+                            if (lane < per && first_key(j) < x.lk && (id < 0 || id >= p.num_blocks)) {
+                                atomicCAS(p.status, 0, kStatusIndex);  // a visible key without a block
+                                id = p.num_blocks;
+                            }
+                            uint32_t dst, fb;
+                            // K_j from the [nope | rope] key cache: columns 0-63, 64-127, 128-191
+                            for (int c = 0; c < kKChunks && ok; ++c) {
+                                if (!(ok = next_chunk(dst, fb))) break;
+                                boxes(id, j, dst, &tm_k, fb, 64 * c, j * kBN, p.rows_k, nk);
+                            }
+                            // V_j: keys 0-63, keys 64-127; each chunk holds V cols 0-63 then 64-127
+                            for (int hh = 0; hh < kVChunks && ok; ++hh) {
+                                if (!(ok = next_chunk(dst, fb))) break;
+                                boxes(id, j, dst, &tm_v, fb, 0, j * kBN + hh * 64, p.rows_v, nv);
+                                boxes(id, j, dst + kVHalfBytes, &tm_v, fb, 64, j * kBN + hh * 64, p.rows_v, nv);
+                            }
+                        }
+                    } else {
+                        for (int j = 0; j < x.n_max && ok; ++j) {
+                            const int tok = x.k_tok0 + j * kBN;
+                            uint32_t dst, fb;
+                            // K_j: nope cols 0-63, nope cols 64-127, rope
+                            if (!(ok = next_chunk(dst, fb))) break;
+                            ptx::tma_load_3d(dst, &tm_k, fb, 0, x.kh, tok, pol_kv);
+                            if (!(ok = next_chunk(dst, fb))) break;
+                            ptx::tma_load_3d(dst, &tm_k, fb, 64, x.kh, tok, pol_kv);
+                            if (!(ok = next_chunk(dst, fb))) break;
+                            ptx::tma_load_3d(dst, &tm_kr, fb, 0, x.kh, tok, pol_kv);
+                            // V_j: keys 0-63, keys 64-127; each chunk holds V cols 0-63 then 64-127
+                            for (int hh = 0; hh < kVChunks && ok; ++hh) {
+                                if (!(ok = next_chunk(dst, fb))) break;
+                                ptx::tma_load_3d(dst, &tm_v, fb, 0, x.kh, tok + hh * 64, pol_kv);
+                                ptx::tma_load_3d(dst + kVHalfBytes, &tm_v, fb, 64, x.kh, tok + hh * 64, pol_kv);
+                            }
+                        }
                     }
                 }
-            }
-            // Let every copy this thread started land before the block can exit.
-            if (ql0) wait_bar(bar(bars->q_full[0]), (ql0 - 1) & 1, bars, p.status);
-            if (ql1) wait_bar(bar(bars->q_full[1]), (ql1 - 1) & 1, bars, p.status);
-            for (uint32_t s = 0; s < kRing; ++s) {
-                const uint32_t n = rc / kRing + (s < rc % kRing ? 1 : 0);
-                if (n) wait_bar(bar(bars->ch_full[s]), (n - 1) & 1, bars, p.status);
+                // Let every copy this warp started land before the block can exit.
+                if (ql0) wait(bar(bars->q_full[0]), (ql0 - 1) & 1);
+                if (ql1) wait(bar(bars->q_full[1]), (ql1 - 1) & 1);
+                for (uint32_t s = 0; s < kRing; ++s) {
+                    const uint32_t n = rc / kRing + (s < rc % kRing ? 1 : 0);
+                    if (n) wait(bar(bars->ch_full[s]), (n - 1) & 1);
+                }
+            };
+            if constexpr (kKvAny) {
+                if (p.paged) producer(std::true_type{});
+                else if (lane == 0) producer(std::false_type{});
+            } else {
+                if (lane == 0) producer(std::false_type{});
             }
         } else if (warp == 1) {
             // -------------------------------------------------------- MMA issuer
@@ -638,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl2 = p.scale_log2;
         uint32_t sf = 0, of = 0;
         bool ok = true;
-        uint32_t ss = 0;
+        uint32_t ss = 0, ring_seq = 0;
         while (ok) {
             const uint32_t slot = ss % kSched;
             ok = wait_bar_warp(bar(bars->sched_full[slot]), (ss / kSched) & 1, bars, p.status);
@@ -649,6 +737,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++ss;
             if (it < 0) break;
             const WorkItem x = decode_item(p, it, num_units, kCausal);
+            // ring index of this unit's first K chunk: key tile j holds V in chunks vbase + 5j + {0, 1}
+            const uint32_t vbase = ring_seq + kKChunks;
+            ring_seq += (kKChunks + kVChunks) * x.n_max;
             const int n_t = t ? x.n[1] : x.n[0];
             const bool row_valid = row < (t ? x.rows[1] : x.rows[0]);
             const int i = x.u0 + t * kBM + row;  // query row within the sequence
@@ -666,6 +757,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int tile_q0 = x.u0 + t * kBM;
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < n_t; ++j) {
+                // Keys past Lk have p = 0, but 0 * (NaN or Inf) is NaN: where those V rows may hold
+                // anything, this thread zeroes key row `row` of V_j once it has landed (both
+                // warpgroups write the same zeros; P V_j is issued only after this warpgroup's
+                // P-ready arrival for this tile, and the chunk is refilled only after that MMA).
+                if (kKvAny && (j + 1) * kBN > x.lk) {
+                    const uint32_t vch = vbase + 5 * j + (row >> 6);
+                    ok = wait_bar_warp(bar(bars->ch_full[vch % kRing]), (vch / kRing) & 1, bars, p.status);
+                    if (!ok) break;
+                    if (j * kBN + row >= x.lk) {
+                        uint4 *vr = reinterpret_cast<uint4 *>(smem + kSmemRing + (vch % kRing) * kChunkBytes +
+                                                              (row & 63) * 128);
+                        const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            vr[e] = z;
+                            vr[kVHalfBytes / 16 + e] = z;
+                        }
+                        ptx::fence_proxy_async_smem();
+                    }
+                }
                 ok = wait_bar_warp(bar(bars->s_full[t]), sf & 1, bars, p.status);
                 ++sf;
                 if (!ok) break;

@@ -19,7 +19,6 @@ namespace mla {
 
 constexpr int kGatherThreads = 256;
 constexpr int kPagedPlanThreads = 1024;
-constexpr int kStatusIndex = 10;  // mirrors MLA_ERR_INDEX
 
 // Lengths (plain or running sums) -> packed offsets, clamped to the output's
 // token count (kStatusSeqlen on any inconsistency).  offs[batch] = total rows.

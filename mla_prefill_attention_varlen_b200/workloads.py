@@ -125,3 +125,41 @@ def sample_rows(seq_len: int, n: int, seed: int) -> np.ndarray:
     k = max(0, min(n - len(fixed), rest.size))
     drawn = np.random.default_rng(seed).choice(rest, size=k, replace=False) if k else np.array([], dtype=np.int64)
     return np.sort(np.concatenate([np.asarray(fixed, dtype=np.int64), drawn.astype(np.int64)]))
+
+
+def paged_cache(k, k_rope, v, kv_seqlens, block_size, seed=7, spare_blocks=0, slot_fill=0.0, table_fill=-1):
+    """Scatters packed keys / values into a block-paged cache (the ND keyCache / valueCache
+    layout of the PagedCacheLoadOperation page), blocks handed out in a seeded random order.
+
+    Returns (key_cache [blocks, block_size, G, 192] holding K_nope | K_rope per slot,
+    value_cache [blocks, block_size, G, 128], block_tables [batch, W] int32).  Slots no key
+    occupies (the tail of each sequence's last block, the spare blocks) hold `slot_fill`; table
+    entries past a sequence's last block hold `table_fill`.  Pure data movement.
+    """
+    device = k.device
+    G = k.shape[1]
+    kcat = torch.cat([k, k_rope], dim=2)
+    need = [(L + block_size - 1) // block_size for L in kv_seqlens]
+    nb = sum(need) + spare_blocks
+    perm = torch.randperm(max(nb, 1), generator=torch.Generator().manual_seed(seed))[:nb]
+    kc = torch.full((max(nb, 1), block_size, G, kcat.shape[2]), slot_fill, dtype=k.dtype, device=device)
+    vc = torch.full((max(nb, 1), block_size, G, v.shape[2]), slot_fill, dtype=v.dtype, device=device)
+    table = torch.full((len(need), max(need + [1])), table_fill, dtype=torch.int32)
+    used = start = 0
+    for b, L in enumerate(kv_seqlens):
+        n = need[b]
+        if n:
+            idx = perm[used:used + n]
+            table[b, :n] = idx.to(torch.int32)
+            full = L // block_size
+            dev_idx = idx.to(device)
+            if full:
+                kc[dev_idx[:full]] = kcat[start:start + full * block_size].view(full, block_size, G, -1)
+                vc[dev_idx[:full]] = v[start:start + full * block_size].view(full, block_size, G, -1)
+            rem = L - full * block_size
+            if rem:
+                kc[int(idx[full]), :rem] = kcat[start + full * block_size:start + L]
+                vc[int(idx[full]), :rem] = v[start + full * block_size:start + L]
+        used += n
+        start += L
+    return kc, vc, table.to(device)

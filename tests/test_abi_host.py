@@ -230,3 +230,74 @@ def test_paged_rejects_bad_arguments(lib):
     assert paged_call(lib, a, starts=torch.zeros(3, dtype=torch.int32)) == 3
     b = dict(a, value=a["key"])
     assert paged_call(lib, b) == 6  # outputs overlap
+
+
+# ---------------------------------------------------------------------------
+# mla_prefill_paged host-side validation (descriptors are never dereferenced)
+# ---------------------------------------------------------------------------
+
+def prefill_paged_args(T=64, H=4, G=2, nb=8, bs=16, W=4, batch=2, dtype=torch.bfloat16):
+    return dict(q=torch.zeros(T, H, 128, dtype=dtype), q_rope=torch.zeros(T, H, 64, dtype=dtype),
+                kc=torch.zeros(nb, bs, G, 192, dtype=dtype), vc=torch.zeros(nb, bs, G, 128, dtype=dtype),
+                table=torch.zeros(batch, W, dtype=torch.int32), q_seqlen=torch.zeros(batch, dtype=torch.int32),
+                kv_seqlen=torch.zeros(batch, dtype=torch.int32), out=torch.zeros(T, H, 128, dtype=dtype)), H, G
+
+
+def prefill_paged_call(lib, a, H, G, mask=1, scale=0.5):
+    d = {k: mla.as_mla_tensor(v) for k, v in a.items()}
+    r = lambda k: ctypes.byref(d[k])
+    return lib.mla_prefill_paged(r("q"), r("q_rope"), r("kc"), r("vc"), r("table"), r("q_seqlen"), r("kv_seqlen"),
+                                 mask, H, G, scale, r("out"), None)
+
+
+@pytest.mark.parametrize("bs,ok", [(8, True), (16, True), (64, True), (128, True), (256, True), (384, True),
+                                   (4, False), (12, False), (48, False), (96, False), (136, False), (200, False)])
+def test_prefill_paged_block_sizes(lib, bs, ok):
+    a, H, G = prefill_paged_args(bs=bs)
+    rc = prefill_paged_call(lib, a, H, G)
+    if ok:
+        if not torch.cuda.is_available():
+            assert rc == 7  # well formed: reaches CUDA
+    else:
+        assert rc == 6
+
+
+def test_prefill_paged_rejects_bad_arguments(lib):
+    a, H, G = prefill_paged_args()
+    d = {k: mla.as_mla_tensor(v) for k, v in a.items()}
+    assert lib.mla_prefill_paged(ctypes.byref(d["q"]), ctypes.byref(d["q_rope"]), None, ctypes.byref(d["vc"]),
+                                 ctypes.byref(d["table"]), ctypes.byref(d["q_seqlen"]), ctypes.byref(d["kv_seqlen"]),
+                                 1, H, G, 0.5, ctypes.byref(d["out"]), None) == 1
+    b = dict(a, kc=torch.zeros(8, 16, G, 128, dtype=torch.bfloat16))
+    assert prefill_paged_call(lib, b, H, G) == 3  # key cache must be 192 wide (nope | rope)
+    b = dict(a, vc=torch.zeros(9, 16, G, 128, dtype=torch.bfloat16))
+    assert prefill_paged_call(lib, b, H, G) == 3  # block counts differ
+    b = dict(a, vc=torch.zeros(8, 32, G, 128, dtype=torch.bfloat16))
+    assert prefill_paged_call(lib, b, H, G) == 3  # block sizes differ
+    b = dict(a, kc=torch.zeros(8, 16, 1, 192, dtype=torch.bfloat16))
+    assert prefill_paged_call(lib, b, H, G) == 3  # kv heads differ from kv_head_num
+    b = dict(a, vc=torch.zeros(8, 16, G, 128, dtype=torch.float16))
+    assert prefill_paged_call(lib, b, H, G) == 2  # cache dtype differs from q
+    b = dict(a, table=torch.zeros(2, 4, dtype=torch.int64))
+    assert prefill_paged_call(lib, b, H, G) == 2
+    b = dict(a, table=torch.zeros(3, 4, dtype=torch.int32))
+    assert prefill_paged_call(lib, b, H, G) == 3  # table rows != batch
+    b = dict(a, table=torch.zeros(4, 2, dtype=torch.int32).t())
+    assert prefill_paged_call(lib, b, H, G) == 4  # table rows not contiguous
+    wide = torch.zeros(8, 16, G, 200, dtype=torch.bfloat16)
+    b = dict(a, kc=wide[..., 4:196])
+    assert prefill_paged_call(lib, b, H, G) == 4  # 8-byte base offset
+    wide = torch.zeros(8, 16, G, 196, dtype=torch.bfloat16)
+    b = dict(a, kc=wide[..., :192])
+    assert prefill_paged_call(lib, b, H, G) == 4  # head stride not a multiple of 8 elements
+    assert prefill_paged_call(lib, a, 4, 3) == 5
+    assert prefill_paged_call(lib, a, H, G, mask=5) == 6
+    buf = torch.zeros(8 * 16 * G * 192 + 64 * H * 128, dtype=torch.bfloat16)
+    b = dict(a, kc=buf[:8 * 16 * G * 192].view(8, 16, G, 192), out=buf[8 * 16 * G * 192 - 128:][:64 * H * 128]
+             .view(64, H, 128))
+    assert prefill_paged_call(lib, b, H, G) == 6  # out overlaps the key cache
+
+
+def test_prefill_paged_empty_batch_is_a_no_op(lib):
+    a, H, G = prefill_paged_args(batch=0)
+    assert prefill_paged_call(lib, a, H, G) == 0

@@ -286,11 +286,11 @@ def test_inconsistent_seqlens_are_clamped_and_reported(bad):
 # the page's padded K/V layout [batch, max_seq, kv_head * dim]
 # ---------------------------------------------------------------------------
 
-def _to_padded(x, lens_k, max_seq, G):
-    """Packed K/K_rope/V -> dense padded [batch, max_seq, G*W] tensors (rows past Lk_b filled with 9)."""
+def _to_padded(x, lens_k, max_seq, G, fill=9.0):
+    """Packed K/K_rope/V -> dense padded [batch, max_seq, G*W] tensors (rows past Lk_b filled with `fill`)."""
     out = {}
     for key, w in (("k", 128), ("k_rope", 64), ("v", 128)):
-        buf = torch.full((len(lens_k), max_seq, G * w), 9.0, dtype=x[key].dtype, device=DEV)
+        buf = torch.full((len(lens_k), max_seq, G * w), fill, dtype=x[key].dtype, device=DEV)
         start = 0
         for b, L in enumerate(lens_k):
             buf[b, :L] = x[key][start:start + L].reshape(L, G * w)
@@ -312,6 +312,19 @@ def test_padded_kv_layout_matches_packed(case):
     torch.cuda.synchronize()
     assert torch.equal(packed, padded)  # same keys, same tiles: bit-identical
     check_against_oracle(x, padded, H, G, 0.07)
+    assert status() == 0
+
+
+@pytest.mark.parametrize("fill", [float("nan"), float("inf"), -float("inf")])
+def test_padded_kv_padding_never_reaches_the_result(fill):
+    # padding rows past Lk_b share key tiles with real keys; P = 0 there, and 0 * NaN would be NaN
+    lq, lk, H, G = [40, 130, 3], [100, 130, 77], 4, 2
+    _, x = problem(lq, lk, H, G, seed=503)
+    packed = run(x, H, G, 0.07).clone()
+    y = dict(x, **_to_padded(x, lk, 200, G, fill=fill))
+    padded = run(y, H, G, 0.07)
+    torch.cuda.synchronize()
+    assert torch.equal(packed, padded)
     assert status() == 0
 
 
