@@ -568,7 +568,8 @@ def main():
         "tokens_per_s": tokens_per_s,
         "north_star_literal_tflops": 2 * value,
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": kern_tflops / peak, "traffic": None if paged else measured_traffic(wl.name),
+                     "frac": kern_tflops / peak,
+                     "traffic": measured_traffic("%s_paged%d" % (wl.name, args.block_size) if paged else wl.name),
                      "peak_source": peak_src,
                      "peak_kind": "burst", "frac_of_sustained": kern_tflops / peak_sus,
                      "kernel": "mla_prefill_sm100_kernel", "kernel_ms": kms,
