@@ -163,3 +163,54 @@ def paged_cache(k, k_rope, v, kv_seqlens, block_size, seed=7, spare_blocks=0, sl
         used += n
         start += L
     return kc, vc, table.to(device)
+
+
+@dataclass
+class PrologShape:
+    """Sizes of the MlaProlog step (the page's supported configuration by default:
+    h 4096, q_lora_rank 1024, 64 heads of head_dim 512, rope_dim 64)."""
+    name: str
+    tokens: int
+    hidden: int = 4096
+    q_lora_rank: int = 1024
+    num_heads: int = 64
+    head_dim: int = 512
+    rope_dim: int = 64
+    seed: int = 6
+
+
+def prolog_shapes() -> dict:
+    return {s.name: s for s in [
+        PrologShape("prolog_small", tokens=77, hidden=512, q_lora_rank=256, num_heads=4, head_dim=256,
+                    rope_dim=64, seed=61),
+        PrologShape("prolog", tokens=4096),
+    ]}
+
+
+def make_prolog_inputs(s: PrologShape, device="cpu", positions=None):
+    """Synthetic bf16 inputs of the MlaProlog step on ``device``.
+
+    token_x ~ N(0, 1); projection weights ~ N(0, 1 / fan_in) (random init, no trained weights);
+    RmsNorm weights 1 + 0.25 N(0, 1); rope_cos / rope_sin for token positions (default
+    0 .. tokens-1) at angles pos * 10000^(-2i / rope_dim), each value repeated for the two
+    channels of its interleaved pair.  Drawn in fp32 with a seeded CPU generator, rounded to bf16.
+    """
+    gen = torch.Generator().manual_seed(s.seed)
+
+    def draw(*shape, scale=1.0, shift=0.0):
+        return (torch.randn(*shape, generator=gen) * scale + shift).to(torch.bfloat16).to(device)
+
+    t, h, r, d = s.tokens, s.hidden, s.q_lora_rank, s.head_dim
+    pos = torch.arange(t, dtype=torch.float64) if positions is None else torch.as_tensor(positions, dtype=torch.float64)
+    inv = 10000.0 ** (-torch.arange(0, s.rope_dim, 2, dtype=torch.float64) / s.rope_dim)
+    ang = pos[:, None] * inv[None, :]
+    return {
+        "token_x": draw(t, h),
+        "wq_a": draw(h, r, scale=h ** -0.5),
+        "wq_b": draw(r, s.num_heads * d, scale=r ** -0.5),
+        "wkv": draw(h, d, scale=h ** -0.5),
+        "rope_cos": torch.cos(ang).repeat_interleave(2, dim=1).to(torch.bfloat16).to(device),
+        "rope_sin": torch.sin(ang).repeat_interleave(2, dim=1).to(torch.bfloat16).to(device),
+        "gamma_cq": draw(r, scale=0.25, shift=1.0),
+        "gamma_ckv": draw(d, scale=0.25, shift=1.0),
+    }
