@@ -395,6 +395,128 @@ def bench_paged(args):
     return 0
 
 
+def bench_prolog(args):
+    """mla_prolog on the page's configuration: projection TFLOP/s for the whole step, plus the
+    HBM roofline of the per-head RmsNorm / RoPE kernel (the largest kernel of this library in it)."""
+    import torch
+
+    import mla_prefill_attention_varlen_b200 as mla
+    from mla_prefill_attention_varlen_b200 import workloads as W
+
+    rank, world, local = dist_setup(args.gpus)
+    s = W.prolog_shapes()["prolog"]
+    if args.tokens:
+        s.tokens = args.tokens
+    dev = torch.device("cuda", torch.cuda.current_device())
+    mla.load_library()
+    x = W.make_prolog_inputs(s, device=dev)
+    order = ("token_x", "wq_a", "wq_b", "wkv", "rope_cos", "rope_sin", "gamma_cq", "gamma_ckv")
+    t, h, r, H, d, R = s.tokens, s.hidden, s.q_lora_rank, s.num_heads, s.head_dim, s.rope_dim
+    q = torch.empty(t, H, d, dtype=torch.bfloat16, device=dev)
+    kv = torch.empty(t, d, dtype=torch.bfloat16, device=dev)
+    cq = torch.empty(t, r, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call(inp, qo, kvo, cqo):
+        mla.mla_prolog(*[inp[k] for k in order], H, qo, kvo, cqo, stream=stream)
+
+    flops = 2.0 * t * (h * r + r * H * d + h * d)
+    norm_bytes = t * H * d * (4 + 2) + 2 * t * R * 2  # fp32 rows in, bf16 rows out, cos / sin
+    for _ in range(args.warmup):
+        call(x, q, kv, cq)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    smi = ClockSampler(torch.cuda.current_device())
+    barrier(world)
+    with smi:
+        time.sleep(0.1)
+        smi.mark_start()
+        for i in range(args.steps):
+            mla.set_profile_events(k_starts[i], k_stops[i])
+            starts[i].record(stream)
+            call(x, q, kv, cq)
+            stops[i].record(stream)
+        mla.set_profile_events(None, None)
+        torch.cuda.synchronize()
+        smi.mark_stop()
+    barrier(world)
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in zip(starts, stops)])), world)
+    kms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in zip(k_starts, k_stops)])), world)
+    value = job_throughput(world, flops, ms) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    in_bytes = sum(v.numel() * v.element_size() for v in x.values())
+
+    e2e = None
+    if not args.no_e2e:
+        hx = {k: v.cpu().pin_memory() for k, v in x.items()}
+        dx = {k: torch.empty_like(v) for k, v in x.items()}
+        hq = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        hkv = torch.empty(kv.shape, dtype=kv.dtype).pin_memory()
+
+        def e2e_step():
+            for k in dx:
+                dx[k].copy_(hx[k], non_blocking=True)
+            call(dx, q, kv, None)
+            hq.copy_(q, non_blocking=True)
+            hkv.copy_(kv, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(in_bytes),
+               "d2h_bytes_per_step": int(hq.numel() * 2 + hkv.numel() * 2)}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle.prolog as prolog
+
+        cpu = {k: v.cpu() for k, v in x.items()}
+        n = 8
+        t0 = time.time()
+        reps = 0
+        while True:
+            sub = dict(cpu, token_x=cpu["token_x"][:n], rope_cos=cpu["rope_cos"][:n], rope_sin=cpu["rope_sin"][:n])
+            prolog.mla_prolog(*[sub[k] for k in order], H)
+            reps += 1
+            if time.time() - t0 > min(args.cpu_seconds, 10.0):
+                break
+        dt = time.time() - t0
+        cpu_baseline = {"value": reps * n * flops / t / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                        "kind": "oracle", "sample": "%d x %d tokens of the prolog workload (fp64 numpy)" % (reps, n)}
+
+    line = {
+        "metric": "MLA prolog TFLOP/s (projection FLOPs 2 t (h r + r H d + h d))", "value": value,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "prolog", "tokens": t, "hidden": h, "q_lora_rank": r, "num_heads": H, "head_dim": d,
+                   "rope_dim": R, "weights": "random init", "l2": "inputs and outputs %.2f GB > 126 MB L2" % (
+                       (in_bytes + q.numel() * 2) / 1e9)},
+        "roofline": {"bound": "hbm", "achieved": norm_bytes / (kms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": norm_bytes / (kms * 1e-3) / 1e9 / hbm, "traffic": None, "peak_source": peak_src,
+                     "kernel": "rms_norm_rope_kernel (q rows)", "kernel_ms": kms,
+                     "algorithmic_bytes_per_launch": norm_bytes,
+                     "step_tensor_frac": value / world / peak},
+        "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": smi.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,10 +527,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--op", default="prefill", choices=["prefill", "prefill_paged", "paged_cache_load"],
+    ap.add_argument("--op", default="prefill", choices=["prefill", "prefill_paged", "paged_cache_load", "prolog"],
                     help="prefill: mla_prefill on packed K/V; prefill_paged: mla_prefill_paged reading a "
                          "paged cache in place; paged_cache_load: the gather alone")
     ap.add_argument("--block-size", type=int, default=64, help="paged ops: tokens per cache block")
+    ap.add_argument("--tokens", type=int, default=0, help="prolog: tokens (default: the prolog workload's)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: scale head_num and kv_head_num down to this many query heads")
     args = ap.parse_args()
@@ -426,6 +549,8 @@ def main():
         return reference_arm(args, wl)
     if args.op == "paged_cache_load":
         return bench_paged(args)
+    if args.op == "prolog":
+        return bench_prolog(args)
 
     import torch
 

@@ -251,6 +251,48 @@ int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, const mla_t
                       const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num, float qk_scale,
                       mla_tensor *out, mla_stream_t stream);
 
+/*
+ * mla_prolog -- the MLA Prolog step, non-quantised (the "MlaProlog" page of
+ * cann-recipes-infer: 功能说明 / 计算公式 / 参数说明 sections), asynchronous on
+ * `stream`.  For each token row x of token_x:
+ *
+ *   c^Q = RmsNorm(x wq_a) * gamma_cq                       (stored as bf16)
+ *   q   = RmsNorm(c^Q wq_b) per head, weight 1;  q[h, d-R:] = ROPE(q[h, d-R:])
+ *   kv  = RmsNorm(x wkv) * gamma_ckv;            kv[d-R:]   = ROPE(kv[d-R:])
+ *
+ * RmsNorm(v) = v / sqrt(mean(v^2) + eps) over the row (over each head's d
+ * channels for q).  ROPE is the interleaved rotation of adjacent channel pairs
+ * with the token's cos / sin rows: y[2i] = v[2i] cos[2i] - v[2i+1] sin[2i],
+ * y[2i+1] = v[2i+1] cos[2i+1] + v[2i] sin[2i+1].
+ *
+ *   token_x   [t, h]          MLA_BF16 (page: token_x)
+ *   wq_a      [h, r]          MLA_BF16 (page: wq_a; r = q_lora_rank)
+ *   wq_b      [r, H*d]        MLA_BF16 (page: wq_b, here unquantised; H = num_heads, d = head_dim)
+ *   wkv       [h, d]          MLA_BF16 (page: wkv)
+ *   rope_cos, rope_sin [t, R] MLA_BF16 (page: rope_cos / rope_sin; R = rope_dim)
+ *   gamma_cq  [r], gamma_ckv [d]  MLA_BF16 (page: gamma_cq / gamma_ckv)
+ *   num_heads H >= 1; eps >= 0 (not printed on the page; 1e-6 is the usual value)
+ * Outputs (bf16): q_out [t, H, d] or [t, H*d] (page: q_out), kv_out [t, d]
+ * (page: kv_out), and cq_out [t, r] (c^Q, the non-quantised counterpart of the
+ * page's qr_out) or NULL.
+ * The page's supported sizes are h 4096, r 1024, H 64, d 512, R 64, t up to
+ * 64k; any sizes work with r, d, R multiples of 4 and R <= d.  Matrices have a
+ * contiguous last dimension, a row stride that is a multiple of 8 elements and
+ * 16-byte aligned bases; vectors are contiguous.  Outputs must not overlap each
+ * other or any input.
+ *
+ * The projections run as bf16 GEMMs with fp32 results (cuBLAS); nothing is
+ * rounded before the norms except c^Q, which is rounded to bf16 once before
+ * the q projection.  Scratch (fp32 projections of up to 4096 tokens at a time)
+ * lives in the per-GPU workspace shared with mla_prefill: order calls on one
+ * stream.  Argument errors return before any launch.  Returns MLA_OK or an
+ * mla_status error code.
+ */
+int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, const mla_tensor *wq_b, const mla_tensor *wkv,
+               const mla_tensor *rope_cos, const mla_tensor *rope_sin, const mla_tensor *gamma_cq,
+               const mla_tensor *gamma_ckv, int num_heads, float eps, mla_tensor *q_out, mla_tensor *kv_out,
+               mla_tensor *cq_out, mla_stream_t stream);
+
 /* A static, human-readable name for a status code (never NULL). */
 const char *mla_status_string(int status);
 

@@ -13,7 +13,7 @@ from . import workloads  # noqa: F401  (seeded synthetic inputs)
 
 __all__ = [
     "MLA_MASK_NONE", "MLA_MASK_CAUSAL", "MlaError", "load_library", "mla_prefill", "mla_prefill_noalloc",
-    "mla_paged_cache_load", "mla_prefill_paged", "mla_prefill_device_status", "mla_status_string", "prefill",
+    "mla_paged_cache_load", "mla_prefill_paged", "mla_prolog", "mla_prefill_device_status", "mla_status_string", "prefill",
     "workloads",
 ]
 
@@ -68,6 +68,8 @@ def load_library(path=None):
     lib.mla_prefill_paged.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
                                       T, ctypes.c_void_p]
     lib.mla_prefill_paged.restype = ctypes.c_int
+    lib.mla_prolog.argtypes = [T, T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_float, T, T, T, ctypes.c_void_p]
+    lib.mla_prolog.restype = ctypes.c_int
     lib.mla_prefill_set_profile_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.mla_prefill_set_profile_events.restype = ctypes.c_int
     lib.mla_prefill_version.argtypes = []
@@ -185,6 +187,21 @@ def mla_prefill_paged(q, q_rope, key_cache, value_cache, block_tables, q_seqlen,
     if rc != 0:
         raise MlaError(rc, "mla_prefill_paged")
     return out
+
+
+def mla_prolog(token_x, wq_a, wq_b, wkv, rope_cos, rope_sin, gamma_cq, gamma_ckv, num_heads, q_out, kv_out,
+               cq_out=None, eps=1e-6, stream=None):
+    """Call the C ABI ``mla_prolog`` (MLA Prolog, non-quantised): writes q_out [t, H, d],
+    kv_out [t, d] and, if given, cq_out [t, q_lora_rank] (bf16) in place."""
+    lib = load_library()
+    d = [as_mla_tensor(t) for t in (token_x, wq_a, wq_b, wkv, rope_cos, rope_sin, gamma_cq, gamma_ckv, q_out,
+                                    kv_out)]
+    cq = ctypes.byref(as_mla_tensor(cq_out)) if cq_out is not None else None
+    rc = lib.mla_prolog(*(ctypes.byref(x) for x in d[:8]), int(num_heads), float(eps), ctypes.byref(d[8]),
+                        ctypes.byref(d[9]), cq, _stream_handle(stream, token_x.device))
+    if rc != 0:
+        raise MlaError(rc, "mla_prolog")
+    return q_out, kv_out
 
 
 def set_profile_events(start=None, stop=None):

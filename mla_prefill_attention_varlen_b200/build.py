@@ -22,6 +22,8 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC,-O2,-Wall",
     "-shared",
 ]
+# the MLA Prolog projections are library GEMMs
+LINK_FLAGS = ["-lcublas", "-Xlinker", "-rpath," + os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64")]
 
 
 def _nvcc():
@@ -45,7 +47,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [_nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", tmp] + sources()
+    cmd = [_nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", tmp] + sources() + LINK_FLAGS
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

@@ -2,6 +2,7 @@
 // TMA tensor-map encoding and the two launches (plan kernel, attention kernel)
 // behind the C ABI declared in include/mla_prefill.h.
 #include <cuda.h>
+#include <cublas_v2.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -13,6 +14,7 @@
 #include "../../include/mla_prefill.h"
 #include "mla_prefill_sm100.cuh"
 #include "paged_cache_load.cuh"
+#include "prolog_norm_rope.cuh"
 
 namespace {
 
@@ -784,4 +786,180 @@ extern "C" int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, 
     std::lock_guard<std::mutex> lock(g_mu);
     if ((rc = device_state(dev, stream, lay.total, &ds)) != MLA_OK) return rc;
     return enqueue(pr, lay, static_cast<uint8_t *>(ds->ws), ds->status, ds->sm_count, ds, stream);
+}
+
+// ---------------------------------------------------------------------------
+// MLA Prolog: the three projections as library GEMMs (bf16 operands, fp32
+// results), then the RmsNorm / RoPE rows of prolog_norm_rope.cuh
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kPrologSlab = 4096;  // tokens per pass: bounds the fp32 scratch
+cublasHandle_t g_blas[kMaxDevices] = {};
+
+// A 2-D bf16 matrix [rows, cols] with a contiguous last dimension and a row stride that is a
+// multiple of 8 elements (16 bytes).  want_rows / want_cols < 0 accept any extent.
+struct Mat {
+    void *data;
+    int64_t rows, cols, ld;
+};
+
+int mat2(const mla_tensor *t, int64_t want_rows, int64_t want_cols, Mat *m) {
+    if (!t) return MLA_ERR_NULL;
+    if (t->dtype != MLA_BF16) return MLA_ERR_DTYPE;
+    if (t->ndim != 2) return MLA_ERR_SHAPE;
+    if ((want_rows >= 0 && t->shape[0] != want_rows) || (want_cols >= 0 && t->shape[1] != want_cols))
+        return MLA_ERR_SHAPE;
+    if (t->shape[0] < 0 || t->shape[1] < 1 || t->shape[0] > INT32_MAX || t->shape[1] > INT32_MAX)
+        return MLA_ERR_SHAPE;
+    if (t->shape[0] > 0 && !t->data) return MLA_ERR_NULL;
+    if (t->shape[1] > 1 && t->stride[1] != 1) return MLA_ERR_ALIGN;
+    const int64_t ld = t->shape[0] > 1 ? t->stride[0] : t->shape[1];
+    if (ld < t->shape[1] || ld % 8 || ld > INT32_MAX || !aligned16(t->data)) return MLA_ERR_ALIGN;
+    *m = Mat{t->data, t->shape[0], t->shape[1], ld};
+    return MLA_OK;
+}
+
+int vec1(const mla_tensor *t, int64_t n, const void **p) {
+    if (!t || !t->data) return MLA_ERR_NULL;
+    if (t->dtype != MLA_BF16) return MLA_ERR_DTYPE;
+    if (t->ndim != 1 || t->shape[0] != n) return MLA_ERR_SHAPE;
+    if (n > 1 && t->stride[0] != 1) return MLA_ERR_ALIGN;
+    if (!aligned16(t->data)) return MLA_ERR_ALIGN;
+    *p = t->data;
+    return MLA_OK;
+}
+
+struct Range {
+    uintptr_t lo, hi;
+};
+Range mat_range(const Mat &m) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(m.data);
+    return Range{lo, m.rows > 0 ? lo + static_cast<uintptr_t>(((m.rows - 1) * m.ld + m.cols) * 2) : lo};
+}
+Range view_range(const View3 &v) {
+    Range r;
+    byte_range(v, &r.lo, &r.hi);
+    return r;
+}
+bool ranges_overlap(const Range &a, const Range &b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// C[M, N] (fp32, row stride ldc) = A[M, K] B[K, N] (bf16, row-major): the column-major library
+// call computes C^T = B^T A^T.
+int gemm_rowmajor(cublasHandle_t h, int64_t M, int64_t N, int64_t K, const void *A, int64_t lda, const void *B,
+                  int64_t ldb, float *C, int64_t ldc) {
+    const float one = 1.f, zero = 0.f;
+    const cublasStatus_t s =
+        cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(N), static_cast<int>(M), static_cast<int>(K), &one,
+                     B, CUDA_R_16BF, static_cast<int>(ldb), A, CUDA_R_16BF, static_cast<int>(lda), &zero, C,
+                     CUDA_R_32F, static_cast<int>(ldc), CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+    return s == CUBLAS_STATUS_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int launch_norm(const mla::NormParams &np, int sm_count, cudaStream_t stream) {
+    const long long rows = np.job[0].rows + (np.njobs > 1 ? np.job[1].rows : 0);
+    if (rows == 0) return MLA_OK;
+    const long long want = (rows + mla::kNormThreads / 32 - 1) / (mla::kNormThreads / 32);
+    const long long cap = static_cast<long long>(sm_count) * 8;
+    mla::rms_norm_rope_kernel<<<static_cast<int>(want < cap ? want : cap), mla::kNormThreads, 0, stream>>>(np);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, const mla_tensor *wq_b,
+                          const mla_tensor *wkv, const mla_tensor *rope_cos, const mla_tensor *rope_sin,
+                          const mla_tensor *gamma_cq, const mla_tensor *gamma_ckv, int num_heads, float eps,
+                          mla_tensor *q_out, mla_tensor *kv_out, mla_tensor *cq_out, mla_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!q_out || !kv_out) return MLA_ERR_NULL;
+    if (num_heads < 1) return MLA_ERR_HEADS;
+    if (!std::isfinite(eps) || eps < 0.f) return MLA_ERR_UNSUPPORTED;
+    int rc;
+    Mat x, wa, wb, wk, cs, sn, kvo, cqo{};
+    if ((rc = mat2(token_x, -1, -1, &x)) != MLA_OK) return rc;
+    const int64_t t = x.rows, h = x.cols;
+    if ((rc = mat2(wq_a, h, -1, &wa)) != MLA_OK) return rc;
+    if ((rc = mat2(wkv, h, -1, &wk)) != MLA_OK) return rc;
+    const int64_t r = wa.cols, d = wk.cols, H = num_heads;
+    if (H * d > INT32_MAX) return MLA_ERR_SHAPE;
+    if ((rc = mat2(wq_b, r, H * d, &wb)) != MLA_OK) return rc;
+    if ((rc = mat2(rope_cos, t, -1, &cs)) != MLA_OK) return rc;
+    const int64_t R = cs.cols;
+    if ((rc = mat2(rope_sin, t, R, &sn)) != MLA_OK) return rc;
+    if (r % 4 || d % 4 || R % 4 || R > d) return MLA_ERR_UNSUPPORTED;  // rows move in groups of 4 channels
+    const void *g_cq, *g_ckv;
+    if ((rc = vec1(gamma_cq, r, &g_cq)) != MLA_OK) return rc;
+    if ((rc = vec1(gamma_ckv, d, &g_ckv)) != MLA_OK) return rc;
+    View3 qo;
+    if ((rc = view3(q_out, MLA_BF16, H, d, &qo)) != MLA_OK) return rc;
+    if (qo.tokens != t) return MLA_ERR_SHAPE;
+    if ((rc = mat2(kv_out, t, d, &kvo)) != MLA_OK) return rc;
+    if (cq_out && (rc = mat2(cq_out, t, r, &cqo)) != MLA_OK) return rc;
+    // outputs overlap neither each other nor any input
+    const Range outs[3] = {view_range(qo), mat_range(kvo), cq_out ? mat_range(cqo) : Range{0, 0}};
+    const Range ins[6] = {mat_range(x), mat_range(wa), mat_range(wb), mat_range(wk), mat_range(cs), mat_range(sn)};
+    for (int i = 0; i < 3; ++i) {
+        for (int k = i + 1; k < 3; ++k)
+            if (ranges_overlap(outs[i], outs[k])) return MLA_ERR_UNSUPPORTED;
+        for (const Range &in : ins)
+            if (ranges_overlap(outs[i], in)) return MLA_ERR_UNSUPPORTED;
+    }
+    if (t == 0) return MLA_OK;
+
+    // scratch per slab: [S, r + d] fp32 (x wq_a | x wkv), [S, H d] fp32 (c^Q wq_b), [S, r] bf16 c^Q
+    const int64_t slab = t < kPrologSlab ? t : kPrologSlab;
+    const size_t pre_bytes = align_up(static_cast<size_t>(slab * (r + d)) * 4, 256);
+    const size_t q_bytes = align_up(static_cast<size_t>(slab * H * d) * 4, 256);
+    const size_t cq_bytes = cq_out ? 0 : align_up(static_cast<size_t>(slab * r) * 2, 256);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState *ds = nullptr;
+    if ((rc = device_state(dev, stream, pre_bytes + q_bytes + cq_bytes, &ds)) != MLA_OK) return rc;
+    if (!g_blas[dev] && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS) {
+        g_blas[dev] = nullptr;
+        return MLA_ERR_CUDA;
+    }
+    cublasHandle_t bl = g_blas[dev];
+    if (cublasSetStream(bl, stream) != CUBLAS_STATUS_SUCCESS) return MLA_ERR_CUDA;
+    uint8_t *ws = static_cast<uint8_t *>(ds->ws);
+    float *pre = reinterpret_cast<float *>(ws);
+    float *qpre = reinterpret_cast<float *>(ws + pre_bytes);
+    __nv_bfloat16 *cq_scratch = reinterpret_cast<__nv_bfloat16 *>(ws + pre_bytes + q_bytes);
+    const auto bf = [](const void *p, int64_t elems) {
+        return reinterpret_cast<__nv_bfloat16 *>(const_cast<uint8_t *>(static_cast<const uint8_t *>(p)) + elems * 2);
+    };
+
+    for (int64_t s0 = 0; s0 < t; s0 += slab) {
+        const int64_t S = t - s0 < slab ? t - s0 : slab;
+        const void *xs = bf(x.data, s0 * x.ld);
+        // x wq_a -> pre[:, 0:r],  x wkv -> pre[:, r:r+d]
+        if ((rc = gemm_rowmajor(bl, S, r, h, xs, x.ld, wa.data, wa.ld, pre, r + d)) != MLA_OK) return rc;
+        if ((rc = gemm_rowmajor(bl, S, d, h, xs, x.ld, wk.data, wk.ld, pre + r, r + d)) != MLA_OK) return rc;
+        __nv_bfloat16 *cq = cq_out ? bf(cqo.data, s0 * cqo.ld) : cq_scratch;
+        const int64_t cq_ld = cq_out ? cqo.ld : r;
+        mla::NormParams np{};
+        np.eps = eps;
+        np.njobs = 2;
+        np.job[0] = mla::NormJob{pre, r + d, cq, cq_ld, 0, static_cast<const __nv_bfloat16 *>(g_cq), nullptr,
+                                 nullptr, 0, 0, static_cast<int>(r), 0, 1, S};
+        np.job[1] = mla::NormJob{pre + r, r + d, bf(kvo.data, s0 * kvo.ld), kvo.ld, 0,
+                                 static_cast<const __nv_bfloat16 *>(g_ckv), bf(cs.data, s0 * cs.ld),
+                                 bf(sn.data, s0 * sn.ld), cs.ld, sn.ld, static_cast<int>(d), static_cast<int>(R), 1,
+                                 S};
+        if ((rc = launch_norm(np, ds->sm_count, stream)) != MLA_OK) return rc;
+        // c^Q wq_b -> qpre [S, H d]; per-head RmsNorm (weight 1) and rope into q_out
+        if ((rc = gemm_rowmajor(bl, S, H * d, r, cq, cq_ld, wb.data, wb.ld, qpre, H * d)) != MLA_OK) return rc;
+        mla::NormParams nq{};
+        nq.eps = eps;
+        nq.njobs = 1;
+        nq.job[0] = mla::NormJob{qpre, H * d, bf(qo.data, s0 * qo.st_tok), qo.st_tok, qo.st_head, nullptr,
+                                 bf(cs.data, s0 * cs.ld), bf(sn.data, s0 * sn.ld), cs.ld, sn.ld,
+                                 static_cast<int>(d), static_cast<int>(R), static_cast<int>(H), S * H};
+        if (t_prof_start && cudaEventRecord(t_prof_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
+        if ((rc = launch_norm(nq, ds->sm_count, stream)) != MLA_OK) return rc;
+        if (t_prof_stop && cudaEventRecord(t_prof_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
 }

@@ -68,6 +68,20 @@ def rope_interleaved(v, cos, sin):
     return out
 
 
+def mla_prolog_q(c_q, wq_b, rope_cos, rope_sin, num_heads, eps=1e-6):
+    """The query half after c^Q: q = RmsNorm(c^Q . wq_b) per head (weight 1), then the interleaved
+    rope on each head's last rope_dim channels.  Returns q [t, num_heads, head_dim] in fp64."""
+    c_q, wq_b = f64(c_q), f64(wq_b)
+    cos, sin = f64(rope_cos), f64(rope_sin)
+    t = c_q.shape[0]
+    head_dim = wq_b.shape[1] // num_heads
+    rope_dim = cos.shape[1]
+    q = (c_q @ wq_b).reshape(t, num_heads, head_dim)
+    q = rms_norm(q, 1.0, eps)
+    q[..., head_dim - rope_dim:] = rope_interleaved(q[..., head_dim - rope_dim:], cos[:, None, :], sin[:, None, :])
+    return q
+
+
 def mla_prolog(token_x, wq_a, wq_b, wkv, rope_cos, rope_sin, gamma_cq, gamma_ckv, num_heads, eps=1e-6,
                round_cq=True):
     """Returns (q [t, num_heads, head_dim], kv [t, head_dim], c^Q [t, q_lora_rank]) in fp64.
@@ -89,10 +103,7 @@ def mla_prolog(token_x, wq_a, wq_b, wkv, rope_cos, rope_sin, gamma_cq, gamma_ckv
     c_q = rms_norm(x @ wq_a, gamma_cq, eps)
     if round_cq:
         c_q = round_bf16(c_q)
-    # up-projection, per-head RmsNorm with weight 1, interleaved rope on each head's last rope_dim channels
-    q = (c_q @ wq_b).reshape(t, num_heads, head_dim)
-    q = rms_norm(q, 1.0, eps)
-    q[..., head_dim - rope_dim:] = rope_interleaved(q[..., head_dim - rope_dim:], cos[:, None, :], sin[:, None, :])
+    q = mla_prolog_q(c_q, wq_b, cos, sin, num_heads, eps)
     # key-value latent: down-projection, RmsNorm, interleaved rope on the last rope_dim channels
     kv = rms_norm(x @ wkv, gamma_ckv, eps)
     kv[..., head_dim - rope_dim:] = rope_interleaved(kv[..., head_dim - rope_dim:], cos, sin)

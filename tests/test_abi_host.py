@@ -301,3 +301,58 @@ def test_prefill_paged_rejects_bad_arguments(lib):
 def test_prefill_paged_empty_batch_is_a_no_op(lib):
     a, H, G = prefill_paged_args(batch=0)
     assert prefill_paged_call(lib, a, H, G) == 0
+
+
+# ---------------------------------------------------------------------------
+# mla_prolog host-side validation (descriptors are never dereferenced)
+# ---------------------------------------------------------------------------
+
+def prolog_args(t=8, h=64, r=32, H=2, d=32, R=16, dtype=torch.bfloat16):
+    z = lambda *s: torch.zeros(*s, dtype=dtype)
+    return dict(x=z(t, h), wq_a=z(h, r), wq_b=z(r, H * d), wkv=z(h, d), cos=z(t, R), sin=z(t, R), g_cq=z(r),
+                g_ckv=z(d), q=z(t, H, d), kv=z(t, d), cq=z(t, r)), H
+
+
+def prolog_call(lib, a, H, eps=1e-6, with_cq=True):
+    d = {k: mla.as_mla_tensor(v) for k, v in a.items()}
+    r = lambda k: ctypes.byref(d[k])
+    return lib.mla_prolog(r("x"), r("wq_a"), r("wq_b"), r("wkv"), r("cos"), r("sin"), r("g_cq"), r("g_ckv"), H, eps,
+                          r("q"), r("kv"), r("cq") if with_cq else None, None)
+
+
+def test_prolog_accepts_well_formed_arguments(lib):
+    if torch.cuda.is_available():
+        pytest.skip("host-only check")
+    a, H = prolog_args()
+    assert prolog_call(lib, a, H) == 7  # reaches CUDA
+    assert prolog_call(lib, a, H, with_cq=False) == 7
+    a["q"] = a["q"].reshape(8, H * 32)  # [t, H*d] form
+    assert prolog_call(lib, a, H) == 7
+    a, H = prolog_args(t=0)
+    assert prolog_call(lib, a, H) == 0  # no tokens: nothing to do
+
+
+def test_prolog_rejects_bad_arguments(lib):
+    a, H = prolog_args()
+    assert prolog_call(lib, a, 0) == 5
+    assert prolog_call(lib, a, H, eps=-1.0) == 6
+    assert prolog_call(lib, a, H, eps=float("nan")) == 6
+    assert prolog_call(lib, dict(a, wkv=a["wkv"].half()), H) == 2
+    assert prolog_call(lib, dict(a, g_cq=torch.zeros(32, dtype=torch.float32)), H) == 2
+    assert prolog_call(lib, dict(a, wq_a=torch.zeros(48, 32, dtype=torch.bfloat16)), H) == 3  # h mismatch
+    assert prolog_call(lib, dict(a, wq_b=torch.zeros(32, 48, dtype=torch.bfloat16)), H) == 3  # not H*d wide
+    assert prolog_call(lib, dict(a, sin=torch.zeros(8, 8, dtype=torch.bfloat16)), H) == 3  # cos / sin widths
+    assert prolog_call(lib, dict(a, cos=torch.zeros(7, 16, dtype=torch.bfloat16)), H) == 3  # one row per token
+    assert prolog_call(lib, dict(a, kv=torch.zeros(8, 16, dtype=torch.bfloat16)), H) == 3
+    assert prolog_call(lib, dict(a, q=torch.zeros(8, 3, 32, dtype=torch.bfloat16)), H) == 3
+    assert prolog_call(lib, dict(a, g_ckv=torch.zeros(16, dtype=torch.bfloat16)), H) == 3
+    a2, _ = prolog_args(R=6, d=32)
+    assert prolog_call(lib, a2, H) == 4  # a 6-wide cos row stride is not a multiple of 8 elements
+    a3, _ = prolog_args(R=40, d=32)
+    assert prolog_call(lib, a3, H) == 6  # rope wider than the head
+    wide = torch.zeros(8, 72, dtype=torch.bfloat16)
+    assert prolog_call(lib, dict(a, x=wide[:, 4:68]), H) == 4  # 8-byte offset base
+    assert prolog_call(lib, dict(a, x=torch.zeros(8, 68, dtype=torch.bfloat16)[:, :64]), H) == 4  # row stride 68
+    buf = torch.zeros(8 * 64 + 8 * 32, dtype=torch.bfloat16)
+    assert prolog_call(lib, dict(a, kv=buf[:256].view(8, 32), cq=buf[128:384].view(8, 32)), H) == 6  # outputs overlap
+    assert prolog_call(lib, dict(a, kv=a["x"][:, :32]), H) == 6  # output over an input
