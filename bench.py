@@ -532,6 +532,8 @@ def main():
                          "paged cache in place; paged_cache_load: the gather alone")
     ap.add_argument("--block-size", type=int, default=64, help="paged ops: tokens per cache block")
     ap.add_argument("--tokens", type=int, default=0, help="prolog: tokens (default: the prolog workload's)")
+    ap.add_argument("--split", type=int, default=-1,
+                    help="split-KV chunk in 128-key tiles for the prefill ops: -1 automatic (default), 0 off")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: scale head_num and kv_head_num down to this many query heads")
     args = ap.parse_args()
@@ -559,6 +561,7 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     mla.load_library()
+    mla.set_split_tiles(args.split)
     x = W.make_inputs(wl, device=dev)
     out = torch.empty(wl.t_q, wl.head_num, wl.d_nope, dtype=wl.dtype, device=dev)
     H, G, scale = wl.head_num, wl.kv_head_num, wl.qk_scale
@@ -686,7 +689,7 @@ def main():
                    "parallelism": "replicas" if world > 1 else "single", "l2": (
                        "flushed between steps (512 MB write)" if flush is not None else
                        "inputs %.2f GB > 126 MB L2" % (in_bytes / 1e9)),
-                   "visible_triples": triples,
+                   "visible_triples": triples, "split_kv": "automatic" if args.split < 0 else args.split,
                    **({"kv_layout": "paged", "block_size": args.block_size, "blocks": int(x["key_cache"].shape[0])}
                       if paged else {"kv_layout": "packed"})},
         "pct_of_peak": 100.0 * value / world / peak,

@@ -307,6 +307,26 @@ const char *mla_status_string(int status);
 struct CUevent_st;
 int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *stop);
 
+/*
+ * mla_prefill_set_split_tiles -- split-KV control for later mla_prefill and
+ * mla_prefill_paged calls on this host thread (no counterpart on the pages).
+ * A 256-row query unit normally walks all its key tiles in one work item; with
+ * split-KV its key tiles go in chunks of `tiles` 128-key tiles, each chunk a
+ * separate item that writes O / l and the row's log-sum-exp in fp32 to the
+ * library workspace, and a combine kernel merges the chunks into attenOut
+ * (the same softmax over the union of the chunks' keys).  This fills the GPU
+ * when few long units exist (a long sequence at low head counts).
+ *   tiles = -1  automatic (the default): split only when (units x heads) is
+ *               below twice the SM count and the work is at least 16 key
+ *               tiles per SM, in chunks giving ~3 items per SM;
+ *   tiles =  0  never split;
+ *   tiles >  0  split every unit longer than `tiles` key tiles (the chunk is
+ *               doubled if the fp32 partial rows would exceed 2 GiB).
+ * mla_prefill_noalloc never splits.  Returns MLA_OK, or MLA_ERR_UNSUPPORTED
+ * for tiles < -1.
+ */
+int mla_prefill_set_split_tiles(int tiles);
+
 /* Library version as 10000*major + 100*minor + patch. */
 int mla_prefill_version(void);
 

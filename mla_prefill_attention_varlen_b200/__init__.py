@@ -13,7 +13,7 @@ from . import workloads  # noqa: F401  (seeded synthetic inputs)
 
 __all__ = [
     "MLA_MASK_NONE", "MLA_MASK_CAUSAL", "MlaError", "load_library", "mla_prefill", "mla_prefill_noalloc",
-    "mla_paged_cache_load", "mla_prefill_paged", "mla_prolog", "mla_prefill_device_status", "mla_status_string", "prefill",
+    "mla_paged_cache_load", "mla_prefill_paged", "mla_prolog", "set_split_tiles", "mla_prefill_device_status", "mla_status_string", "prefill",
     "workloads",
 ]
 
@@ -72,6 +72,8 @@ def load_library(path=None):
     lib.mla_prolog.restype = ctypes.c_int
     lib.mla_prefill_set_profile_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.mla_prefill_set_profile_events.restype = ctypes.c_int
+    lib.mla_prefill_set_split_tiles.argtypes = [ctypes.c_int]
+    lib.mla_prefill_set_split_tiles.restype = ctypes.c_int
     lib.mla_prefill_version.argtypes = []
     lib.mla_prefill_version.restype = ctypes.c_int
     if path is None:
@@ -202,6 +204,13 @@ def mla_prolog(token_x, wq_a, wq_b, wkv, rope_cos, rope_sin, gamma_cq, gamma_ckv
     if rc != 0:
         raise MlaError(rc, "mla_prolog")
     return q_out, kv_out
+
+
+def set_split_tiles(tiles):
+    """Split-KV chunk (in 128-key tiles) for later prefill calls on this thread: -1 automatic, 0 off."""
+    rc = load_library().mla_prefill_set_split_tiles(int(tiles))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_set_split_tiles")
 
 
 def set_profile_events(start=None, stop=None):

@@ -32,6 +32,7 @@ struct DeviceState {
 
 std::mutex g_mu;
 thread_local cudaEvent_t t_prof_start = nullptr, t_prof_stop = nullptr;
+thread_local int t_split_tiles = -1;  // split-KV chunk in key tiles: -1 automatic, 0 off
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -169,13 +170,28 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
     size_t seq_info, unit_off, hist, units, num_units, total;
+    size_t split_off, entry_tab, part_lse, part_o;  // split-KV sections (empty without split)
     int hist_len;
+    int split_tiles;
 };
 
-WsLayout ws_layout(int64_t batch, int64_t t_q, int64_t t_k) {
+int64_t max_units_for(int64_t batch, int64_t t_q) { return (t_q + mla::kUnitRows - 1) / mla::kUnitRows + batch; }
+
+// Upper bound of work-list entries when each unit's key tiles go in chunks of `split` (at most
+// ceil(key_extent / 128) tiles per unit).
+int64_t max_entries_for(int64_t max_units, int64_t key_extent, int split) {
+    const int64_t tiles = (key_extent + mla::kBN - 1) / mla::kBN;
+    return split > 0 ? max_units * ((tiles + split - 1) / split > 1 ? (tiles + split - 1) / split : 1) : max_units;
+}
+
+// t_k: key tokens of the K/V tensors; key_extent: the most keys one sequence can have;
+// split: key tiles per split-KV chunk (0: none); heads: query heads.
+WsLayout ws_layout(int64_t batch, int64_t t_q, int64_t t_k, int64_t key_extent = 0, int split = 0,
+                   int64_t heads = 0) {
     WsLayout l;
-    const int64_t max_units = (t_q + mla::kUnitRows - 1) / mla::kUnitRows + batch;
+    const int64_t max_units = max_units_for(batch, t_q);
     l.hist_len = static_cast<int>((t_k + mla::kBN - 1) / mla::kBN + 2);
+    l.split_tiles = split;
     size_t off = 0;
     l.num_units = off;
     off = align_up(off + 16, 256);
@@ -187,6 +203,18 @@ WsLayout ws_layout(int64_t batch, int64_t t_q, int64_t t_k) {
     off = align_up(off + sizeof(int) * l.hist_len, 256);
     l.units = off;
     off = align_up(off + sizeof(int2) * max_units, 256);
+    l.split_off = l.entry_tab = l.part_lse = l.part_o = off;
+    if (split > 0) {
+        const int64_t entries = max_entries_for(max_units, key_extent, split);
+        l.split_off = off;
+        off = align_up(off + sizeof(int) * (max_units + 1), 256);
+        l.entry_tab = off;
+        off = align_up(off + sizeof(int2) * entries, 256);
+        l.part_lse = off;
+        off = align_up(off + sizeof(float) * entries * heads * mla::kUnitRows, 256);
+        l.part_o = off;
+        off = align_up(off + sizeof(float) * entries * heads * mla::kUnitRows * mla::kDn, 256);
+    }
     l.total = off;
     return l;
 }
@@ -220,10 +248,10 @@ int device_state(int dev, cudaStream_t stream, size_t ws_need, DeviceState **out
     return MLA_OK;
 }
 
-template <typename T, bool kCausal, bool kPos, bool kKvAny>
+template <typename T, bool kCausal, bool kPos, bool kGeneral>
 int launch_attention(DeviceState *ds, int slot, int grid, cudaStream_t stream, const CUtensorMap (&maps)[5],
                      const mla::Params &p) {
-    auto kern = mla::mla_prefill_sm100_kernel<T, kCausal, kPos, kKvAny>;
+    auto kern = mla::mla_prefill_sm100_kernel<T, kCausal, kPos, kGeneral>;
     if (!ds->attr_set[slot]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kSmemAlloc) != cudaSuccess)
             return MLA_ERR_CUDA;
@@ -351,6 +379,9 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
 
     int *num_units = reinterpret_cast<int *>(ws + lay.num_units);
     int *work_counter = num_units + 1;  // second word of the 16-byte header
+    int *num_entries = num_units + 2;   // third word
+    int *split_off = reinterpret_cast<int *>(ws + lay.split_off);
+    int2 *entry_tab = reinterpret_cast<int2 *>(ws + lay.entry_tab);
     int4 *seq_info = reinterpret_cast<int4 *>(ws + lay.seq_info);
     int *unit_off = reinterpret_cast<int *>(ws + lay.unit_off);
     int *hist = reinterpret_cast<int *>(ws + lay.hist);
@@ -359,7 +390,7 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
         pr.q_seqlen, pr.kv_seqlen, static_cast<int>(pr.batch), pr.q.tokens, pr.k.tokens, pr.kv_pad,
         pr.paged ? 1 : 0, pr.causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
-        status);
+        lay.split_tiles, split_off, entry_tab, num_entries, status);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
     mla::Params p;
@@ -382,23 +413,72 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     p.rows_k = rows_k > 0 ? rows_k : 1;
     p.rows_v = rows_v > 0 ? rows_v : 1;
     p.paged = pr.paged ? 1 : 0;
-    const bool kv_any = pr.paged || pr.kv_pad > 0;  // padded or paged K/V
+    p.split_tiles = lay.split_tiles;
+    p.entry_tab = entry_tab;
+    p.num_entries = num_entries;
+    p.part_lse = reinterpret_cast<float *>(ws + lay.part_lse);
+    p.part_o = reinterpret_cast<float *>(ws + lay.part_o);
+    const bool general = pr.paged || pr.kv_pad > 0 || lay.split_tiles > 0;  // padded / paged K/V or split-KV
 
-    const int64_t max_items = ((pr.q.tokens + mla::kUnitRows - 1) / mla::kUnitRows + pr.batch) * pr.head_num;
+    const int64_t max_units = max_units_for(pr.batch, pr.q.tokens);
+    const int64_t max_items =
+        max_entries_for(max_units, pr.kv_pad > 0 ? pr.kv_pad : pr.k.tokens, lay.split_tiles) * pr.head_num;
     const int grid = static_cast<int>(max_items < sm_count ? max_items : sm_count);
     const bool pos = pr.qk_scale > 0.f;
     DeviceState *ls = launch_flags;
-    const int slot = (pr.bf16 ? 0 : 4) + (pr.causal ? 0 : 2) + (pos ? 0 : 1) + (kv_any ? 8 : 0);
+    const int slot = (pr.bf16 ? 0 : 4) + (pr.causal ? 0 : 2) + (pos ? 0 : 1) + (general ? 8 : 0);
 #define MLA_LAUNCH(T, C, P, G) launch_attention<T, C, P, G>(ls, slot, grid, stream, maps, p)
-#define MLA_PICK(T, C, P) (kv_any ? MLA_LAUNCH(T, C, P, true) : MLA_LAUNCH(T, C, P, false))
+#define MLA_PICK(T, C, P) (general ? MLA_LAUNCH(T, C, P, true) : MLA_LAUNCH(T, C, P, false))
     if (pr.bf16) {
-        if (pr.causal) return pos ? MLA_PICK(__nv_bfloat16, true, true) : MLA_PICK(__nv_bfloat16, true, false);
-        return pos ? MLA_PICK(__nv_bfloat16, false, true) : MLA_PICK(__nv_bfloat16, false, false);
+        if (pr.causal) rc = pos ? MLA_PICK(__nv_bfloat16, true, true) : MLA_PICK(__nv_bfloat16, true, false);
+        else rc = pos ? MLA_PICK(__nv_bfloat16, false, true) : MLA_PICK(__nv_bfloat16, false, false);
+    } else {
+        if (pr.causal) rc = pos ? MLA_PICK(__half, true, true) : MLA_PICK(__half, true, false);
+        else rc = pos ? MLA_PICK(__half, false, true) : MLA_PICK(__half, false, false);
     }
-    if (pr.causal) return pos ? MLA_PICK(__half, true, true) : MLA_PICK(__half, true, false);
-    return pos ? MLA_PICK(__half, false, true) : MLA_PICK(__half, false, false);
 #undef MLA_PICK
 #undef MLA_LAUNCH
+    if (rc != MLA_OK || lay.split_tiles <= 0) return rc;
+    // split-KV: merge the chunks of every unit that has several
+    mla::CombineParams c;
+    c.seq_info = seq_info;
+    c.units = units;
+    c.num_units = num_units;
+    c.split_off = split_off;
+    c.part_o = p.part_o;
+    c.part_lse = p.part_lse;
+    c.out = pr.o.data;
+    c.out_st = pr.o.st_tok;
+    c.out_sh = pr.o.st_head;
+    c.head_num = pr.head_num;
+    const dim3 cgrid(static_cast<unsigned>(max_units), static_cast<unsigned>(pr.head_num), mla::kCombineRowGroups);
+    if (pr.bf16) mla::mla_split_combine_kernel<__nv_bfloat16><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
+    else mla::mla_split_combine_kernel<__half><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Split-KV chunk (key tiles) for a problem: the thread's override, else automatic -- only when the
+// (unit, head) items cannot fill the GPU twice over and there are at least 16 key tiles of work per
+// SM, in chunks that make about three items per SM.
+// The fp32 partial rows are kept under 2 GiB.
+int choose_split(const Problem &pr, int sm_count) {
+    const int64_t units = max_units_for(pr.batch, pr.q.tokens);
+    const int64_t ext = pr.kv_pad > 0 ? pr.kv_pad : pr.k.tokens;
+    const int64_t tiles = (ext + mla::kBN - 1) / mla::kBN;
+    int64_t split = t_split_tiles;
+    if (split < 0) {
+        if (units * pr.head_num >= 2LL * sm_count) return 0;
+        const int64_t work = pr.head_num * units * tiles / (pr.causal ? 2 : 1);  // key tiles, at most
+        if (work < 16LL * sm_count) return 0;  // too little work to be worth a second kernel
+        split = (work + 3LL * sm_count - 1) / (3LL * sm_count);
+        if (split < 4) split = 4;
+    }
+    if (split <= 0) return 0;
+    const auto bytes = [&](int64_t c) {
+        return max_entries_for(units, ext, static_cast<int>(c)) * pr.head_num * mla::kUnitRows * (mla::kDn + 1) * 4;
+    };
+    while (split < tiles && bytes(split) > (int64_t(2) << 30)) split *= 2;
+    return split >= tiles ? 0 : static_cast<int>(split);
 }
 
 }  // namespace
@@ -417,9 +497,12 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-    const WsLayout lay = ws_layout(pr.batch, pr.q.tokens, pr.k.tokens);
     DeviceState *ds = nullptr;
     std::lock_guard<std::mutex> lock(g_mu);
+    if ((rc = device_state(dev, stream, 0, &ds)) != MLA_OK) return rc;  // SM count
+    const int split = choose_split(pr, ds->sm_count);
+    const WsLayout lay = ws_layout(pr.batch, pr.q.tokens, pr.k.tokens, pr.kv_pad > 0 ? pr.kv_pad : pr.k.tokens,
+                                   split, pr.head_num);
     if ((rc = device_state(dev, stream, lay.total, &ds)) != MLA_OK) return rc;
     return enqueue(pr, lay, static_cast<uint8_t *>(ds->ws), ds->status, ds->sm_count, ds, stream);
 }
@@ -458,6 +541,12 @@ const char *mla_status_string(int status) {
         case MLA_ERR_INDEX: return "MLA_ERR_INDEX: a paged-cache block index was out of range (row zeroed)";
         default: return "unknown mla_status";
     }
+}
+
+int mla_prefill_set_split_tiles(int tiles) {
+    if (tiles < -1) return MLA_ERR_UNSUPPORTED;
+    t_split_tiles = tiles;
+    return MLA_OK;
 }
 
 int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *stop) {
@@ -781,9 +870,12 @@ extern "C" int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, 
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-    const WsLayout lay = ws_layout(pr.batch, pr.q.tokens, pr.k.tokens);
     DeviceState *ds = nullptr;
     std::lock_guard<std::mutex> lock(g_mu);
+    if ((rc = device_state(dev, stream, 0, &ds)) != MLA_OK) return rc;  // SM count
+    const int split = choose_split(pr, ds->sm_count);
+    const WsLayout lay = ws_layout(pr.batch, pr.q.tokens, pr.k.tokens, pr.kv_pad > 0 ? pr.kv_pad : pr.k.tokens,
+                                   split, pr.head_num);
     if ((rc = device_state(dev, stream, lay.total, &ds)) != MLA_OK) return rc;
     return enqueue(pr, lay, static_cast<uint8_t *>(ds->ws), ds->status, ds->sm_count, ds, stream);
 }

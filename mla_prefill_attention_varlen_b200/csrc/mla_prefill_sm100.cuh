@@ -95,7 +95,15 @@ struct Params {
     long long table_stride;
     int table_width, num_blocks, block_size;
     int rows_k, rows_v;  // tokens per TMA box: min(128, block_size), min(64, block_size)
-    int paged;  // K/V read from paged caches through the block table (kKvAny kernels only)
+    int paged;  // K/V read from paged caches through the block table (kGeneral kernels only)
+    // split-KV (kGeneral kernels only): a unit's key tiles go in chunks of split_tiles (0: none); entry e of the work
+    // list is chunk entry_tab[e].y of unit entry_tab[e].x.  Chunks of a unit with more than one
+    // write O / l (fp32) and the base-2 log-sum-exp of each row to part_o / part_lse at
+    // ((e * head_num + h) * 256 + row); mla_split_combine_kernel merges them.
+    int split_tiles;
+    const int2 *entry_tab;
+    const int *num_entries;
+    float *part_o, *part_lse;
 };
 
 struct Barriers {
@@ -135,21 +143,30 @@ struct WorkItem {
     int q_tok0, k_tok0;  // first packed token of the unit / of the sequence's keys
     int lq, lk, off;     // off = Lk - Lq
     int rows[2];         // valid rows of tile 0 / 1
-    int n[2];            // key tiles of tile 0 / 1
+    int j0;              // first key tile of this item (split-KV chunk start; 0 without split)
+    int n[2];            // key tiles of tile 0 / 1 from j0 on
     int n_max;
+    int e, nsplit;       // work-list entry; chunks of its unit (1: the item writes attenOut itself)
 };
 
 // Work items are ordered kv-head-major: for each kv head, its units in the
 // sorted (longest-first) order, and for each unit the query heads of the group.
 // Concurrently running CTAs then read the same kv head's K/V (L2 reuse), and the
 // last items of the grid are the cheapest units.
-__device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num_units, bool causal) {
-    const int per_kh = num_units * p.group;
+template <bool kSplit>  // kSplit: the kernel may run split-KV work lists
+__device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num_entries, bool causal) {
+    const int per_kh = num_entries * p.group;
     WorkItem x;
     x.kh = it / per_kh;
     const int rem = it - x.kh * per_kh;
-    const int u = rem / p.group;
-    x.h = x.kh * p.group + (rem - u * p.group);
+    x.e = rem / p.group;
+    x.h = x.kh * p.group + (rem - x.e * p.group);
+    int u = x.e, chunk = 0;
+    if (kSplit && p.split_tiles > 0) {
+        const int2 uc = p.entry_tab[x.e];
+        u = uc.x;
+        chunk = uc.y;
+    }
     const int2 bm = p.units[u];
     x.b = bm.x;
     const int4 s = p.seq_info[bm.x];
@@ -159,12 +176,33 @@ __device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num
     x.lq = s.z;
     x.lk = s.w;
     x.off = s.w - s.z;
+    x.j0 = 0;
+    x.nsplit = 1;
+    if constexpr (!kSplit) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            x.rows[t] = tile_rows(x.u0 + t * kBM, s.z);
+            x.n[t] = kv_tiles_for(x.u0 + t * kBM, x.rows[t], s.z, s.w, causal);
+        }
+        x.n_max = max(x.n[0], x.n[1]);
+        return x;
+    }
+    int full[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         x.rows[t] = tile_rows(x.u0 + t * kBM, s.z);
-        x.n[t] = kv_tiles_for(x.u0 + t * kBM, x.rows[t], s.z, s.w, causal);
+        full[t] = kv_tiles_for(x.u0 + t * kBM, x.rows[t], s.z, s.w, causal);
     }
-    x.n_max = max(x.n[0], x.n[1]);
+    const int nf = max(full[0], full[1]);
+    int j1 = nf;
+    if (p.split_tiles > 0 && nf > p.split_tiles) {
+        x.nsplit = (nf + p.split_tiles - 1) / p.split_tiles;
+        x.j0 = chunk * p.split_tiles;
+        j1 = min(nf, x.j0 + p.split_tiles);
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) x.n[t] = max(0, min(full[t], j1) - x.j0);
+    x.n_max = j1 - x.j0;
     return x;
 }
 
@@ -261,7 +299,8 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
                                                                 int paged, int causal,
                                                                 int4 *seq_info, int *unit_off, int *hist,
                                                                 int hist_len, int2 *units, int *num_units,
-                                                                int *work_counter, int *status) {
+                                                                int *work_counter, int split_tiles, int *split_off,
+                                                                int2 *entry_tab, int *num_entries, int *status) {
     __shared__ long long warp_sums[32];
     __shared__ int bad;
     if (threadIdx.x == 0) bad = 0;
@@ -337,8 +376,35 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
         const int pos = atomicAdd(&hist[min(cost, hist_len - 1)], 1);
         units[pos] = make_int2(b, m);
     }
+    __syncthreads();
+
+    // 5. split-KV: unit u (sorted order) becomes ceil(cost / split_tiles) entries, in unit order
+    long long entries = total;
+    if (split_tiles > 0) {
+        long long carry_e = 0;
+        for (int base = 0; base < total; base += blockDim.x) {
+            const int u = base + threadIdx.x;
+            long long ns = 0;
+            if (u < total) {
+                const int2 bm = units[u];
+                const int4 s = seq_info[bm.x];
+                const int cost = unit_cost(bm.y * kUnitRows, s.z, s.w, causal != 0);
+                ns = cost > split_tiles ? (cost + split_tiles - 1) / split_tiles : 1;
+            }
+            long long tot;
+            const long long pe = carry_e + block_exclusive_scan(ns, tot, warp_sums);
+            if (u < total) {
+                split_off[u] = static_cast<int>(pe);
+                for (int c = 0; c < ns; ++c) entry_tab[pe + c] = make_int2(u, c);
+            }
+            carry_e += tot;
+        }
+        entries = carry_e;
+        if (threadIdx.x == 0) split_off[total] = static_cast<int>(carry_e);
+    }
     if (threadIdx.x == 0) {
         *num_units = total;
+        *num_entries = static_cast<int>(entries);
         *work_counter = 0;
         if (bad) atomicCAS(status, 0, kStatusSeqlen);
     }
@@ -364,10 +430,11 @@ __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
 // ---------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------
-// kKvAny: padded or paged K/V, where rows of the last key tile past Lk may hold anything
-// (padding, unwritten cache slots).  Packed K/V (kKvAny = false) has only real keys or
-// TMA's zero fill there.
-template <typename T, bool kCausal, bool kPositiveScale, bool kKvAny>
+// kGeneral: padded or paged K/V, where rows of the last key tile past Lk may hold anything
+// (padding, unwritten cache slots), or a split-KV work list.  The packed, unsplit kernels
+// (kGeneral = false) carry none of that code: their last key tile holds only real keys or
+// TMA's zero fill.
+template <typename T, bool kCausal, bool kPositiveScale, bool kGeneral>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
                              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kr,
@@ -413,8 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    const int num_units = *p.num_units;
-    const int n_items = num_units * p.head_num;
+    const int num_entries = *p.num_entries;
+    const int n_items = num_entries * p.head_num;
 
     if (warp < 4) {
         ptx::regs_dec<kRegsLow>();
@@ -472,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (next >= n_items) next = -1;
                     }
                     if (kW) next = __shfl_sync(0xffffffffu, next, 0);
-                    const WorkItem x = decode_item(p, it, num_units, kCausal);
+                    const WorkItem x = decode_item<kGeneral>(p, it, num_entries, kCausal);
                     if (x.n_max == 0) continue;
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
@@ -517,10 +584,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 ptx::tma_load_4d(dst + r * rows * 128, map, fb, c0, x.kh, pos - lb * bs, blk, pol_kv);
                         };
                         const int nk = kBN / p.rows_k, nv = 64 / p.rows_v;
-                        int id_next = raw_id(0);
-                        for (int j = 0; j < x.n_max && ok; ++j) {
+                        int id_next = raw_id(x.j0);
+                        for (int jl = 0; jl < x.n_max && ok; ++jl) {
+                            const int j = x.j0 + jl;  // absolute key tile
                             int id = id_next;
-                            if (j + 1 < x.n_max) id_next = raw_id(j + 1);  // in flight during tile j
+                            if (jl + 1 < x.n_max) id_next = raw_id(j + 1);  // in flight during tile j
                             if (lane < per && first_key(j) < x.lk && (id < 0 || id >= p.num_blocks)) {
                                 atomicCAS(p.status, 0, kStatusIndex);  // a visible key without a block
                                 id = p.num_blocks;
@@ -539,8 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     } else {
-                        for (int j = 0; j < x.n_max && ok; ++j) {
-                            const int tok = x.k_tok0 + j * kBN;
+                        for (int jl = 0; jl < x.n_max && ok; ++jl) {
+                            const int tok = x.k_tok0 + (x.j0 + jl) * kBN;
                             uint32_t dst, fb;
                             // K_j: nope cols 0-63, nope cols 64-127, rope
                             if (!(ok = next_chunk(dst, fb))) break;
@@ -566,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (n) wait(bar(bars->ch_full[s]), (n - 1) & 1);
                 }
             };
-            if constexpr (kKvAny) {
+            if constexpr (kGeneral) {
                 if (p.paged) producer(std::true_type{});
                 else if (lane == 0) producer(std::false_type{});
             } else {
@@ -651,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 ++ss;
                 if (it < 0) break;
-                const WorkItem x = decode_item(p, it, num_units, kCausal);
+                const WorkItem x = decode_item<kGeneral>(p, it, num_entries, kCausal);
                 if (x.n_max == 0) continue;
                 if (x.n[0]) ok = wait_bar_warp(bar(bars->q_full[0]), qf0++ & 1, bars, p.status);
                 if (ok && x.n[1]) ok = wait_bar_warp(bar(bars->q_full[1]), qf1++ & 1, bars, p.status);
@@ -736,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) ptx::mbar_arrive(bar(bars->sched_empty[slot]));
             ++ss;
             if (it < 0) break;
-            const WorkItem x = decode_item(p, it, num_units, kCausal);
+            const WorkItem x = decode_item<kGeneral>(p, it, num_entries, kCausal);
             // ring index of this unit's first K chunk: key tile j holds V in chunks vbase + 5j + {0, 1}
             const uint32_t vbase = ring_seq + kKChunks;
             ring_seq += (kKChunks + kVChunks) * x.n_max;
@@ -745,11 +813,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = x.u0 + t * kBM + row;  // query row within the sequence
             T *orow = reinterpret_cast<T *>(p.out) + (long long)(x.q_tok0 + t * kBM + row) * p.out_st +
                       (long long)x.h * p.out_sh;
+            // split-KV chunk of a unit with several: partial row at part_o / part_lse
+            const long long prow = ((long long)x.e * p.head_num + x.h) * kUnitRows + t * kBM + row;
             if (n_t == 0) {
                 if (row_valid) {
-                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    if (kGeneral && x.nsplit > 1) {
+                        p.part_lse[prow] = -INFINITY;  // no key of this chunk is visible to the row
+                    } else {
+                        const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                    for (int c = 0; c < kDn * 2 / 16; ++c) reinterpret_cast<uint4 *>(orow)[c] = z;
+                        for (int c = 0; c < kDn * 2 / 16; ++c) reinterpret_cast<uint4 *>(orow)[c] = z;
+                    }
                 }
                 continue;
             }
@@ -761,11 +835,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // anything, this thread zeroes key row `row` of V_j once it has landed (both
                 // warpgroups write the same zeros; P V_j is issued only after this warpgroup's
                 // P-ready arrival for this tile, and the chunk is refilled only after that MMA).
-                if (kKvAny && (j + 1) * kBN > x.lk) {
+                if (kGeneral && (x.j0 + j + 1) * kBN > x.lk) {
                     const uint32_t vch = vbase + 5 * j + (row >> 6);
                     ok = wait_bar_warp(bar(bars->ch_full[vch % kRing]), (vch / kRing) & 1, bars, p.status);
                     if (!ok) break;
-                    if (j * kBN + row >= x.lk) {
+                    if ((x.j0 + j) * kBN + row >= x.lk) {
                         uint4 *vr = reinterpret_cast<uint4 *>(smem + kSmemRing + (vch % kRing) * kChunkBytes +
                                                               (row & 63) * 128);
                         const uint4 z = make_uint4(0, 0, 0, 0);
@@ -794,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         s[64 + e] = __uint_as_float(r1[e]);
                     }
                 }
-                const int kv0 = j * kBN;
+                const int kv0 = (x.j0 + j) * kBN;
                 const bool tile_masked = (kv0 + kBN > x.lk) || (kCausal && kv0 + kBN - 1 > tile_q0 + x.off);
                 float m_tile;
                 if (kPositiveScale) {
@@ -866,6 +940,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             ptx::tc_fence_after();
             const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            if (kGeneral && x.nsplit > 1) {
+                // O / l in fp32 and log2(sum 2^s') = m + log2(l) over this chunk's keys
+                float *po = p.part_o + prow * kDn;
+#pragma unroll
+                for (int c = 0; c < kDn / 32; ++c) {
+                    uint32_t r[32];
+                    ptx::tmem_ld32(tO + c * 32, r);
+                    ptx::tmem_wait_ld_dep(r);
+                    if (row_valid) {
+                        float4 *dst = reinterpret_cast<float4 *>(po + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv_l, __uint_as_float(r[4 * e + 1]) * inv_l,
+                                                 __uint_as_float(r[4 * e + 2]) * inv_l,
+                                                 __uint_as_float(r[4 * e + 3]) * inv_l);
+                    }
+                }
+                if (row_valid) p.part_lse[prow] = l_run > 0.f ? m_run + log2f(l_run) : -INFINITY;
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(bar(bars->o_empty[t]));
+                continue;
+            }
 #pragma unroll
             for (int c = 0; c < kDn / 32; ++c) {
                 uint32_t r[32];
@@ -891,6 +987,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV combine: for each unit with several chunks and each head, merges the
+// chunks' partial rows (O_c / l_c in fp32 and lse_c = log2 sum_j 2^s'_j) as
+//   O = sum_c 2^(lse_c - M) (O_c / l_c) / sum_c 2^(lse_c - M),  M = max_c lse_c,
+// the same softmax over the union of the chunks' keys.  One warp per row, four
+// channels per lane; a row no chunk saw any key of is written as zeros.
+// ---------------------------------------------------------------------------
+constexpr int kCombineThreads = 256;
+constexpr int kCombineRowGroups = 8;  // blockIdx.z: rows [z * 32, z * 32 + 32) of the unit
+
+struct CombineParams {
+    const int4 *seq_info;
+    const int2 *units;
+    const int *num_units;
+    const int *split_off;  // [units + 1] first entry of each unit
+    const float *part_o, *part_lse;
+    void *out;
+    long long out_st, out_sh;
+    int head_num;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kCombineThreads) mla_split_combine_kernel(const CombineParams c) {
+    const int u = blockIdx.x, h = blockIdx.y;
+    if (u >= *c.num_units) return;
+    const int e0 = c.split_off[u], ns = c.split_off[u + 1] - e0;
+    if (ns <= 1) return;  // the attention kernel wrote this unit's rows itself
+    const int2 bm = c.units[u];
+    const int4 s = c.seq_info[bm.x];
+    const int u0 = bm.y * kUnitRows;
+    const int rows = min(kUnitRows, s.z - u0);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r_end = min(rows, (int)(blockIdx.z + 1) * (kUnitRows / kCombineRowGroups));
+    for (int r = blockIdx.z * (kUnitRows / kCombineRowGroups) + warp; r < r_end; r += kCombineThreads / 32) {
+        const long long base = (long long)e0 * c.head_num * kUnitRows + (long long)h * kUnitRows + r;
+        const long long step = (long long)c.head_num * kUnitRows;  // between chunks of the same row
+        // every chunk's log-sum-exp at once (lane k holds chunk k0 + k), then the warp maximum
+        float m = -INFINITY;
+        for (int k0 = 0; k0 < ns; k0 += 32)
+            if (k0 + lane < ns) m = fmaxf(m, c.part_lse[base + (k0 + lane) * step]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+        if (m != -INFINITY) {
+            for (int k0 = 0; k0 < ns; k0 += 32) {
+                const float l = k0 + lane < ns ? c.part_lse[base + (k0 + lane) * step] : -INFINITY;
+                const float wl = l == -INFINITY ? 0.f : exp2f(l - m);  // 0: that chunk saw no key of the row
+                const int kn = min(32, ns - k0);
+#pragma unroll 4
+                for (int k = 0; k < kn; ++k) {
+                    const float w = __shfl_sync(0xffffffffu, wl, k);
+                    if (w == 0.f) continue;
+                    const float4 o = reinterpret_cast<const float4 *>(c.part_o + (base + (k0 + k) * step) * kDn)[lane];
+                    acc.x = fmaf(w, o.x, acc.x);
+                    acc.y = fmaf(w, o.y, acc.y);
+                    acc.z = fmaf(w, o.z, acc.z);
+                    acc.w = fmaf(w, o.w, acc.w);
+                    wsum += w;
+                }
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        T *orow = reinterpret_cast<T *>(c.out) + (long long)(s.x + u0 + r) * c.out_st + (long long)h * c.out_sh;
+        const uint32_t lo = DType<T>::pack(acc.x * inv, acc.y * inv), hi = DType<T>::pack(acc.z * inv, acc.w * inv);
+        reinterpret_cast<uint2 *>(orow)[lane] = make_uint2(lo, hi);
     }
 }
 

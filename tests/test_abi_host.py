@@ -356,3 +356,11 @@ def test_prolog_rejects_bad_arguments(lib):
     buf = torch.zeros(8 * 64 + 8 * 32, dtype=torch.bfloat16)
     assert prolog_call(lib, dict(a, kv=buf[:256].view(8, 32), cq=buf[128:384].view(8, 32)), H) == 6  # outputs overlap
     assert prolog_call(lib, dict(a, kv=a["x"][:, :32]), H) == 6  # output over an input
+
+
+def test_split_tiles_control(lib):
+    assert lib.mla_prefill_set_split_tiles(-1) == 0
+    assert lib.mla_prefill_set_split_tiles(0) == 0
+    assert lib.mla_prefill_set_split_tiles(7) == 0
+    assert lib.mla_prefill_set_split_tiles(-2) == 6
+    assert lib.mla_prefill_set_split_tiles(-1) == 0
