@@ -148,3 +148,12 @@ def test_repeatable():
     a = [t.clone() for t in run(x, s)]
     b = run(x, s)
     assert all(torch.equal(u, v) for u, v in zip(a, b))
+
+
+def test_head_dim_outside_the_fused_kernel():
+    # head_dim 96 is not a tensor-memory accumulator size: the library GEMM + row kernel path
+    s = W.PrologShape("prolog_d96", tokens=50, hidden=256, q_lora_rank=96, num_heads=3, head_dim=96, rope_dim=32,
+                      seed=64)
+    x = W.make_prolog_inputs(s, device=DEV)
+    q, kv, cq = run(x, s)
+    check_all(x, s, np.arange(s.tokens), q, kv, cq)
