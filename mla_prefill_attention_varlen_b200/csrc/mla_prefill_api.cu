@@ -258,8 +258,20 @@ int launch_attention(DeviceState *ds, int slot, int grid, cudaStream_t stream, c
         ds->attr_set[slot] = true;
     }
     if (t_prof_start && cudaEventRecord(t_prof_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
-    kern<<<grid, mla::kThreads, mla::kSmemAlloc, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    // programmatic dependent launch: the CTAs start (barriers, tensor memory) while the plan
+    // kernel runs, and wait for it in the kernel before reading the work list
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(mla::kThreads);
+    cfg.dynamicSmemBytes = mla::kSmemAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], p) != cudaSuccess)
+        return MLA_ERR_CUDA;
     if (t_prof_stop && cudaEventRecord(t_prof_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;
 }

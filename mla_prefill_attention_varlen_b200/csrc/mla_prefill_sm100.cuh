@@ -303,6 +303,8 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
                                                                 int2 *entry_tab, int *num_entries, int *status) {
     __shared__ long long warp_sums[32];
     __shared__ int bad;
+    // the attention grid may be scheduled now: it sets itself up and then waits for this grid
+    ptx::griddep_launch_dependents();
     if (threadIdx.x == 0) bad = 0;
     __syncthreads();
 
@@ -480,6 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
+    // everything above overlaps the plan kernel; the work list is read only after it has finished
+    ptx::griddep_wait();
     const int num_entries = *p.num_entries;
     const int n_items = num_entries * p.head_num;
 
