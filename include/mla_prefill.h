@@ -327,6 +327,18 @@ int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *
  */
 int mla_prefill_set_split_tiles(int tiles);
 
+/*
+ * mla_selftest_wait_timeout -- diagnostic for the device timeout path (no
+ * counterpart on the pages).  Launches, on `stream`, one warp that runs the
+ * attention kernel's bounded pipeline wait on an mbarrier nothing arrives at,
+ * with a limit of wait_ms milliseconds (1..10000) instead of the kernel's 2 s.
+ * The wait gives up, records MLA_ERR_DEVICE_TIMEOUT in the device status word
+ * (read it with mla_prefill_device_status) and the kernel returns: no fault,
+ * no trap, and the context stays usable.  Returns MLA_OK, MLA_ERR_UNSUPPORTED
+ * for wait_ms out of range, or MLA_ERR_CUDA.
+ */
+int mla_selftest_wait_timeout(int wait_ms, mla_stream_t stream);
+
 /* Library version as 10000*major + 100*minor + patch. */
 int mla_prefill_version(void);
 

@@ -555,6 +555,19 @@ const char *mla_status_string(int status) {
     }
 }
 
+int mla_selftest_wait_timeout(int wait_ms, mla_stream_t stream_) {
+    if (wait_ms < 1 || wait_ms > 10000) return MLA_ERR_UNSUPPORTED;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    DeviceState *ds = nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int rc;
+    if ((rc = device_state(dev, stream, 0, &ds)) != MLA_OK) return rc;
+    mla::mla_selftest_wait_kernel<<<1, 32, 0, stream>>>(ds->status, static_cast<unsigned long long>(wait_ms) * 1000000ull);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int mla_prefill_set_split_tiles(int tiles) {
     if (tiles < -1) return MLA_ERR_UNSUPPORTED;
     t_split_tiles = tiles;

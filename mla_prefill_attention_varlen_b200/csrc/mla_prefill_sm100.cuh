@@ -208,14 +208,15 @@ __device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num
 
 // Bounded mbarrier wait.  Gives up (and makes every role give up) when another
 // role has aborted or after kWaitLimitNs, recording kStatusTimeout.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Barriers *bars, int *status) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Barriers *bars, int *status,
+                                         uint64_t limit_ns = kWaitLimitNs) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (ptx::mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0) {
             if (*reinterpret_cast<volatile int *>(&bars->abort)) return false;
-            if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (ptx::globaltimer_ns() - t0 > limit_ns) {
                 *reinterpret_cast<volatile int *>(&bars->abort) = 1;
                 atomicCAS(status, 0, kStatusTimeout);
                 return false;
@@ -226,8 +227,9 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, Barriers
 
 // The same wait for a whole warp: every lane polls, and the result is made
 // warp-uniform so that all lanes take the same path afterwards.
-__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, Barriers *bars, int *status) {
-    const bool ok = wait_bar(bar, parity, bars, status);
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, Barriers *bars, int *status,
+                                              uint64_t limit_ns = kWaitLimitNs) {
+    const bool ok = wait_bar(bar, parity, bars, status, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -1061,6 +1063,24 @@ __global__ void __launch_bounds__(kCombineThreads) mla_split_combine_kernel(cons
         const uint32_t lo = DType<T>::pack(acc.x * inv, acc.y * inv), hi = DType<T>::pack(acc.z * inv, acc.w * inv);
         reinterpret_cast<uint2 *>(orow)[lane] = make_uint2(lo, hi);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Diagnostic: the pipeline's bounded wait on an mbarrier that nothing arrives at.
+// It gives up after limit_ns, records kStatusTimeout in the status word and
+// returns -- the path every role of the attention kernel takes when a wait runs
+// out -- so that a test can check the timeout reporting without a real fault.
+// ---------------------------------------------------------------------------
+__global__ void mla_selftest_wait_kernel(int *status, unsigned long long limit_ns) {
+    __shared__ Barriers b;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(ptx::smem_addr(&b.drain), 1);
+        b.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    // phase 0 of a fresh barrier completes only when someone arrives: nobody does
+    wait_bar_warp(ptx::smem_addr(&b.drain), 0, &b, status, limit_ns);
 }
 
 }  // namespace mla
