@@ -229,7 +229,7 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
-    """The maximum of a per-rank float over all ranks (device time is judged by the slowest rank)."""
+    """The maximum of a per-rank float over all ranks (device time is that of the slowest rank)."""
     if world == 1:
         return x
     import torch
@@ -694,7 +694,7 @@ def main():
                       if paged else {"kv_layout": "packed"})},
         "pct_of_peak": 100.0 * value / world / peak,
         "tokens_per_s": tokens_per_s,
-        "north_star_literal_tflops": 2 * value,
+        "tflops_counting_1280_flops_per_pair": 2 * value,
         "roofline": {"bound": "tensor", "achieved": kern_tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": kern_tflops / peak,
                      "traffic": measured_traffic("%s_paged%d" % (wl.name, args.block_size) if paged else wl.name),
