@@ -623,6 +623,7 @@ def main():
     kern_ms = [a.elapsed_time(b) for a, b in zip(k_starts, k_stops)]
     ms = max_over_ranks(float(np.mean(step_ms)), world)
     kms = max_over_ranks(float(np.mean(kern_ms)), world)
+    launches_per_step = mla.load_library().mla_prefill_last_launches()  # plan + attention (+ combine)
     st = mla.mla_prefill_device_status()
     if st != 0:
         raise RuntimeError("device status after timing: %s" % mla.mla_status_string(st))
@@ -704,7 +705,7 @@ def main():
                      "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": algorithmic_bytes(wl)},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if rank == 0:

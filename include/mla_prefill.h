@@ -339,6 +339,10 @@ int mla_prefill_set_split_tiles(int tiles);
  */
 int mla_selftest_wait_timeout(int wait_ms, mla_stream_t stream);
 
+/* Kernels the last mla_prefill / mla_prefill_paged / mla_prefill_noalloc call of this host thread
+ * enqueued: 2 (plan + attention), 3 with split-KV (+ combine), 0 if it launched nothing. */
+int mla_prefill_last_launches(void);
+
 /* Library version as 10000*major + 100*minor + patch. */
 int mla_prefill_version(void);
 

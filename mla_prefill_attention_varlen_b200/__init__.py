@@ -74,6 +74,8 @@ def load_library(path=None):
     lib.mla_prefill_set_profile_events.restype = ctypes.c_int
     lib.mla_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_void_p]
     lib.mla_selftest_wait_timeout.restype = ctypes.c_int
+    lib.mla_prefill_last_launches.argtypes = []
+    lib.mla_prefill_last_launches.restype = ctypes.c_int
     lib.mla_prefill_set_split_tiles.argtypes = [ctypes.c_int]
     lib.mla_prefill_set_split_tiles.restype = ctypes.c_int
     lib.mla_prefill_version.argtypes = []

@@ -33,6 +33,7 @@ struct DeviceState {
 std::mutex g_mu;
 thread_local cudaEvent_t t_prof_start = nullptr, t_prof_stop = nullptr;
 thread_local int t_split_tiles = -1;  // split-KV chunk in key tiles: -1 automatic, 0 off
+thread_local int t_last_launches = 0;  // kernels the last prefill call of this thread enqueued
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -450,7 +451,9 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     }
 #undef MLA_PICK
 #undef MLA_LAUNCH
+    t_last_launches = 2;  // plan + attention
     if (rc != MLA_OK || lay.split_tiles <= 0) return rc;
+    t_last_launches = 3;  // + combine
     // split-KV: merge the chunks of every unit that has several
     mla::CombineParams c;
     c.seq_info = seq_info;
@@ -500,6 +503,7 @@ extern "C" {
 int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
                 const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
                 int head_num, int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
+    t_last_launches = 0;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     Problem pr;
     int rc = validate(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
@@ -567,6 +571,8 @@ int mla_selftest_wait_timeout(int wait_ms, mla_stream_t stream_) {
     mla::mla_selftest_wait_kernel<<<1, 32, 0, stream>>>(ds->status, static_cast<unsigned long long>(wait_ms) * 1000000ull);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
+
+int mla_prefill_last_launches(void) { return t_last_launches; }
 
 int mla_prefill_set_split_tiles(int tiles) {
     if (tiles < -1) return MLA_ERR_UNSUPPORTED;
@@ -636,6 +642,7 @@ extern "C" int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope
                                    const mla_tensor *k_rope, const mla_tensor *v, const mla_tensor *q_seqlen,
                                    const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num,
                                    float qk_scale, mla_tensor *out, mla_stream_t stream_) {
+    t_last_launches = 0;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     Problem pr;
     int rc = validate(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
@@ -848,6 +855,7 @@ extern "C" int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, 
                                  const mla_tensor *value_cache, const mla_tensor *block_tables,
                                  const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type, int head_num,
                                  int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
+    t_last_launches = 0;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (!key_cache || !value_cache || !block_tables) return MLA_ERR_NULL;
     Problem pr;

@@ -364,3 +364,9 @@ def test_split_tiles_control(lib):
     assert lib.mla_prefill_set_split_tiles(7) == 0
     assert lib.mla_prefill_set_split_tiles(-2) == 6
     assert lib.mla_prefill_set_split_tiles(-1) == 0
+
+
+def test_last_launches_is_zero_without_work(lib):
+    t, H, G = make_args(batch=0)
+    assert call(lib, t, H, G) == 0
+    assert lib.mla_prefill_last_launches() == 0

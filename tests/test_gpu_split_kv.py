@@ -62,7 +62,9 @@ def test_split_against_oracle_and_unsplit(case):
     wl = W.Workload("split_case", lq, lk, H, G, dtype=dtype, seed=800 + case)
     x = W.make_inputs(wl, device=DEV)
     whole = run(x, H, G, wl.qk_scale, mask, 0)
+    assert mla.load_library().mla_prefill_last_launches() == 2  # plan + attention
     parts = run(x, H, G, wl.qk_scale, mask, split)
+    assert mla.load_library().mla_prefill_last_launches() == 3  # + combine
     assert mla.mla_prefill_device_status() == 0
     check(x, parts, H, G, wl.qk_scale, mask)
     n = sum(lq)
