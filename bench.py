@@ -287,6 +287,16 @@ def to_numpy_f64(x):
     return {k: (v.double().numpy() if v.is_floating_point() else v.numpy()) for k, v in x.items()}
 
 
+METRIC = "causal MLA prefill TFLOP/s (visible pairs x 640 FLOPs), % of B200 dense bf16 peak, tokens/s"
+
+
+def workload_config(wl):
+    """The workload fields both arms report in `config`."""
+    return {"workload": wl.name, "description": wl.description, "batch": wl.batch, "t_q": wl.t_q, "t_k": wl.t_k,
+            "head_num": wl.head_num, "kv_head_num": wl.kv_head_num, "qk_scale": wl.qk_scale, "mask": "causal",
+            "visible_triples": visible_triples(wl)}
+
+
 def reference_arm(args, wl):
     """The fp64 CPU oracle timed as the reference implementation (rank 0 only)."""
     import torch
@@ -309,11 +319,11 @@ def reference_arm(args, wl):
         trips.append(tr)
     tflops = sum(trips) * FLOPS_PER_TRIPLE / sum(times) / 1e12
     line = {
-        "impl": "reference", "metric": "causal MLA prefill TFLOP/s (visible pairs x 640 FLOPs)",
+        "impl": "reference", "metric": METRIC,
         "value": tflops, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "description": wl.description, "sampled": True},
+        "config": dict(workload_config(wl), sampled="oracle on seeded query rows of every sequence and head"),
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": oracle.core_count(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -704,13 +714,11 @@ def main():
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     clocks = smi.summary()
     line = {
-        "metric": "causal MLA prefill TFLOP/s (visible pairs x 640 FLOPs), % of B200 dense bf16 peak, tokens/s"
-                  + (" (K/V read in place from a paged cache)" if paged else ""),
+        "metric": METRIC + (" (K/V read in place from a paged cache)" if paged else ""),
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f16", "data": "synthetic",
-        "config": {"workload": wl.name, "description": wl.description, "batch": wl.batch, "t_q": wl.t_q,
-                   "t_k": wl.t_k, "head_num": H, "kv_head_num": G, "qk_scale": scale, "mask": "causal",
+        "config": {**workload_config(wl),
                    "parallelism": "replicas" if world > 1 else "single", "l2": (
                        "flushed between steps (512 MB write)" if flush is not None else
                        "inputs %.2f GB > 126 MB L2" % (in_bytes / 1e9)),
