@@ -301,8 +301,11 @@ const char *mla_status_string(int status);
  * non-NULL, every later mla_prefill call on this host thread records `start`
  * on its stream immediately before the attention kernel launch and `stop`
  * immediately after it, so the caller can time that kernel alone with
- * cudaEventElapsedTime.  The events are CUDA events (cudaEvent_t) owned by
- * the caller.  Passing NULL, NULL turns the hook off.  Returns MLA_OK.
+ * cudaEventElapsedTime (while the hook is on, the kernel is launched without
+ * programmatic dependent launch, so none of it starts before `start`).  The
+ * mla_prolog call records them around its query-row RmsNorm / RoPE launch.
+ * The events are CUDA events (cudaEvent_t) owned by the caller.  Passing
+ * NULL, NULL turns the hook off.  Returns MLA_OK.
  */
 struct CUevent_st;
 int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *stop);
