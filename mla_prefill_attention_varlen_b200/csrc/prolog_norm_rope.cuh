@@ -10,9 +10,10 @@
 //   y[2i+1] = v[2i+1] cos[2i+1] + v[2i]   sin[2i+1]
 // where cos / sin are the token's rows of rope_cos / rope_sin [t, R].
 //
-// HBM-bound: one warp per row, 16-byte loads of the fp32 row (coalesced across
-// the warp) kept in registers for rows up to 1024 channels, a warp-shuffle sum
-// of squares, then scale, rotate and store 8-byte groups of four bf16 values.
+// HBM-bound: one warp per row, 16-byte loads of the fp32 row kept in registers
+// for rows up to 1024 channels (eight adjacent channels per lane and group), a
+// warp-shuffle sum of squares, then scale, rotate and store 16-byte groups of
+// eight bf16 values.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -55,10 +56,8 @@ __device__ __forceinline__ float4 load_bf16x4(const __nv_bfloat16 *p) {
     return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
-// Scales, weights, rotates and stores the four channels c .. c+3 of a row.
-__device__ __forceinline__ void finish4(const NormJob &j, long long token, __nv_bfloat16 *out, int i, float4 v,
-                                       float inv) {
-    const int c = i << 2;
+// Scales, weights and rotates the four channels c .. c+3 of a row; returns them as bf16.
+__device__ __forceinline__ uint2 norm4(const NormJob &j, long long token, int c, float4 v, float inv) {
     v.x *= inv;
     v.y *= inv;
     v.z *= inv;
@@ -78,10 +77,20 @@ __device__ __forceinline__ void finish4(const NormJob &j, long long token, __nv_
         const float y2 = v.z * cs.z - v.w * sn.z, y3 = v.w * cs.w + v.z * sn.w;
         v = make_float4(y0, y1, y2, y3);
     }
-    reinterpret_cast<uint2 *>(out)[i] = pack_bf16x4(v.x, v.y, v.z, v.w);
+    return pack_bf16x4(v.x, v.y, v.z, v.w);
 }
 
-constexpr int kNormRegVecs = 8;  // rows up to 32 x 8 x 4 = 1024 channels stay in registers
+__device__ __forceinline__ float sumsq4(float4 v, float ss) {
+    return fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+}
+
+__device__ __forceinline__ float warp_sum(float ss) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    return ss;
+}
+
+constexpr int kNormRegGroups = 4;  // rows of up to 32 lanes x 4 groups x 8 = 1024 channels stay in registers
 
 __global__ void __launch_bounds__(kNormThreads) rms_norm_rope_kernel(const NormParams p) {
     const int lane = threadIdx.x & 31;
@@ -95,38 +104,39 @@ __global__ void __launch_bounds__(kNormThreads) rms_norm_rope_kernel(const NormP
         const int head = static_cast<int>(r - token * j.heads);
         const float4 *in = reinterpret_cast<const float4 *>(j.in + token * j.in_tok + (long long)head * j.width);
         __nv_bfloat16 *out = j.out + token * j.out_tok + (long long)head * j.out_head;
-        const int n4 = j.width >> 2;
         const float rw = 1.f / static_cast<float>(j.width);
-        if (n4 <= 32 * kNormRegVecs) {
-            // the whole row in registers: every load of the row in flight at once, one pass over HBM
-            float4 v[kNormRegVecs];
+        if ((j.width & 7) == 0 && j.width <= 256 * kNormRegGroups) {
+            // the whole row in registers, eight adjacent channels per lane and group: every load of
+            // the row in flight at once, one pass over HBM, 16-byte stores of eight bf16 values
+            const int n8 = j.width >> 3;
+            float4 lo[kNormRegGroups], hi[kNormRegGroups];
             float ss = 0.f;
 #pragma unroll
-            for (int k = 0; k < kNormRegVecs; ++k) {
+            for (int k = 0; k < kNormRegGroups; ++k) {
                 const int i = lane + 32 * k;
-                v[k] = i < n4 ? __ldg(in + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                lo[k] = i < n8 ? __ldg(in + 2 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                hi[k] = i < n8 ? __ldg(in + 2 * i + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int k = 0; k < kNormRegVecs; ++k)
-                ss = fmaf(v[k].x, v[k].x, fmaf(v[k].y, v[k].y, fmaf(v[k].z, v[k].z, fmaf(v[k].w, v[k].w, ss))));
+            for (int k = 0; k < kNormRegGroups; ++k) ss = sumsq4(hi[k], sumsq4(lo[k], ss));
+            const float inv = rsqrtf(warp_sum(ss) * rw + p.eps);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float inv = rsqrtf(ss * rw + p.eps);
-#pragma unroll
-            for (int k = 0; k < kNormRegVecs; ++k)
-                if (lane + 32 * k < n4) finish4(j, token, out, lane + 32 * k, v[k], inv);
+            for (int k = 0; k < kNormRegGroups; ++k) {
+                const int i = lane + 32 * k;
+                if (i < n8) {
+                    const uint2 a = norm4(j, token, 8 * i, lo[k], inv), b = norm4(j, token, 8 * i + 4, hi[k], inv);
+                    reinterpret_cast<uint4 *>(out)[i] = make_uint4(a.x, a.y, b.x, b.y);
+                }
+            }
         } else {
-            // longer rows: sum of squares, then a second pass over the row (an L1 / L2 hit)
+            // other rows: sum of squares, then a second pass over the row (an L1 / L2 hit)
+            const int n4 = j.width >> 2;
             float ss = 0.f;
 #pragma unroll 4
-            for (int i = lane; i < n4; i += 32) {
-                const float4 v = __ldg(in + i);
-                ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float inv = rsqrtf(ss * rw + p.eps);
-            for (int i = lane; i < n4; i += 32) finish4(j, token, out, i, __ldg(in + i), inv);
+            for (int i = lane; i < n4; i += 32) ss = sumsq4(__ldg(in + i), ss);
+            const float inv = rsqrtf(warp_sum(ss) * rw + p.eps);
+            for (int i = lane; i < n4; i += 32)
+                reinterpret_cast<uint2 *>(out)[i] = norm4(j, token, 4 * i, __ldg(in + i), inv);
         }
     }
 }
