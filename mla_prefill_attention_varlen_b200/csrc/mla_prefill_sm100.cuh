@@ -54,6 +54,7 @@ constexpr int kKChunks = 3;                   // Kn lo | Kn hi | Kr            (
 constexpr int kVChunks = 2;                   // keys 0-63 | keys 64-127      (V cols 0-63 then 64-127 inside)
 constexpr int kVHalfBytes = 8192;             // 64 keys x 64 V columns
 constexpr int kSched = 4;                     // depth of the work-item hand-off ring
+constexpr int kTileBars = 4;                  // key-tile barrier sets (tiles in flight are at most 3)
 
 constexpr int kSmemQ = 0;
 constexpr int kSmemRing = kSmemQ + 2 * kQTileBytes;
@@ -108,7 +109,11 @@ struct Params {
 
 struct Barriers {
     uint64_t q_full[2], q_empty[2];
-    uint64_t ch_full[kRing], ch_empty[kRing];
+    // key tile g (counted per CTA across its units) occupies ring chunks 5g .. 5g + 4 (slot = chunk % kRing):
+    // K_g in 5g .. 5g + 2, V_g in 5g + 3, 5g + 4.  Set g % kTileBars of these barriers tracks it:
+    // k_full / v_full complete when its K / V bytes have landed; k_empty / v_empty when the last MMA
+    // reading its K / V has completed.
+    uint64_t k_full[kTileBars], v_full[kTileBars], k_empty[kTileBars], v_empty[kTileBars];
     uint64_t s_full[2], p_full[2];
     uint64_t o_full[2], o_empty[2];
     uint64_t sched_full[kSched], sched_empty[kSched];
@@ -463,9 +468,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(bars->o_full[t]), 1);
             ptx::mbar_init(bar(bars->o_empty[t]), kBM);
         }
-        for (int c = 0; c < kRing; ++c) {
-            ptx::mbar_init(bar(bars->ch_full[c]), 1);
-            ptx::mbar_init(bar(bars->ch_empty[c]), 1);
+        for (int c = 0; c < kTileBars; ++c) {
+            ptx::mbar_init(bar(bars->k_full[c]), 1);
+            ptx::mbar_init(bar(bars->v_full[c]), 1);
+            ptx::mbar_init(bar(bars->k_empty[c]), 1);
+            ptx::mbar_init(bar(bars->v_empty[c]), 1);
         }
         for (int i = 0; i < kSched; ++i) {
             ptx::mbar_init(bar(bars->sched_full[i]), 1);
@@ -512,16 +519,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint64_t pol_q = ptx::policy_evict_first();
                 const uint64_t pol_kv = ptx::policy_evict_last();
-                uint32_t rc = 0;            // ring chunks filled
+                uint32_t tk = 0, tv = 0;    // key tiles whose K / V loads have been issued
                 uint32_t ql0 = 0, ql1 = 0;  // Q tiles loaded per tile slot
                 bool ok = true;
-                auto next_chunk = [&](uint32_t &dst, uint32_t &fb) -> bool {
-                    const uint32_t slot = rc % kRing;
-                    if (!wait(bar(bars->ch_empty[slot]), ((rc / kRing) & 1) ^ 1)) return false;
-                    dst = sRing + slot * kChunkBytes;
-                    fb = bar(bars->ch_full[slot]);
-                    if (lead) ptx::mbar_arrive_expect_tx(fb, kChunkBytes);
-                    ++rc;
+                auto chunk = [&](uint32_t c) { return sRing + (c % kRing) * kChunkBytes; };
+                // K_g's chunks last held K_{g-2}[2] and V_{g-2}: free once the last MMA reading V_{g-2} has
+                // completed (it was issued after every MMA reading K_{g-2}).  V_g's chunks last held
+                // K_{g-1}[0, 1].  Each returns the tile's full barrier, armed with its byte count.
+                auto begin_k = [&](uint32_t g, uint32_t &fb) -> bool {
+                    if (g >= 2 && !wait(bar(bars->v_empty[(g - 2) % kTileBars]), ((g - 2) / kTileBars) & 1))
+                        return false;
+                    fb = bar(bars->k_full[g % kTileBars]);
+                    if (lead) ptx::mbar_arrive_expect_tx(fb, kKChunks * kChunkBytes);
+                    ++tk;
+                    return true;
+                };
+                auto begin_v = [&](uint32_t g, uint32_t &fb) -> bool {
+                    if (g >= 1 && !wait(bar(bars->k_empty[(g - 1) % kTileBars]), ((g - 1) / kTileBars) & 1))
+                        return false;
+                    fb = bar(bars->v_full[g % kTileBars]);
+                    if (lead) ptx::mbar_arrive_expect_tx(fb, kVChunks * kChunkBytes);
+                    ++tv;
                     return true;
                 };
                 // Dynamic scheduling: the first item is blockIdx.x, later ones come from a global
@@ -599,15 +617,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 atomicCAS(p.status, 0, kStatusIndex);  // a visible key without a block
                                 id = p.num_blocks;
                             }
-                            uint32_t dst, fb;
+                            const uint32_t g = tk, c0 = 5 * g;
+                            uint32_t fb;
                             // K_j from the [nope | rope] key cache: columns 0-63, 64-127, 128-191
-                            for (int c = 0; c < kKChunks && ok; ++c) {
-                                if (!(ok = next_chunk(dst, fb))) break;
-                                boxes(id, j, dst, &tm_k, fb, 64 * c, j * kBN, p.rows_k, nk);
-                            }
+                            if (!(ok = begin_k(g, fb))) break;
+                            for (int c = 0; c < kKChunks; ++c)
+                                boxes(id, j, chunk(c0 + c), &tm_k, fb, 64 * c, j * kBN, p.rows_k, nk);
                             // V_j: keys 0-63, keys 64-127; each chunk holds V cols 0-63 then 64-127
-                            for (int hh = 0; hh < kVChunks && ok; ++hh) {
-                                if (!(ok = next_chunk(dst, fb))) break;
+                            if (!(ok = begin_v(g, fb))) break;
+                            for (int hh = 0; hh < kVChunks; ++hh) {
+                                const uint32_t dst = chunk(c0 + kKChunks + hh);
                                 boxes(id, j, dst, &tm_v, fb, 0, j * kBN + hh * 64, p.rows_v, nv);
                                 boxes(id, j, dst + kVHalfBytes, &tm_v, fb, 64, j * kBN + hh * 64, p.rows_v, nv);
                             }
@@ -615,17 +634,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         for (int jl = 0; jl < x.n_max && ok; ++jl) {
                             const int tok = x.k_tok0 + (x.j0 + jl) * kBN;
-                            uint32_t dst, fb;
+                            const uint32_t g = tk, c0 = 5 * g;
+                            uint32_t fb;
                             // K_j: nope cols 0-63, nope cols 64-127, rope
-                            if (!(ok = next_chunk(dst, fb))) break;
-                            ptx::tma_load_3d(dst, &tm_k, fb, 0, x.kh, tok, pol_kv);
-                            if (!(ok = next_chunk(dst, fb))) break;
-                            ptx::tma_load_3d(dst, &tm_k, fb, 64, x.kh, tok, pol_kv);
-                            if (!(ok = next_chunk(dst, fb))) break;
-                            ptx::tma_load_3d(dst, &tm_kr, fb, 0, x.kh, tok, pol_kv);
+                            if (!(ok = begin_k(g, fb))) break;
+                            ptx::tma_load_3d(chunk(c0), &tm_k, fb, 0, x.kh, tok, pol_kv);
+                            ptx::tma_load_3d(chunk(c0 + 1), &tm_k, fb, 64, x.kh, tok, pol_kv);
+                            ptx::tma_load_3d(chunk(c0 + 2), &tm_kr, fb, 0, x.kh, tok, pol_kv);
                             // V_j: keys 0-63, keys 64-127; each chunk holds V cols 0-63 then 64-127
-                            for (int hh = 0; hh < kVChunks && ok; ++hh) {
-                                if (!(ok = next_chunk(dst, fb))) break;
+                            if (!(ok = begin_v(g, fb))) break;
+                            for (int hh = 0; hh < kVChunks; ++hh) {
+                                const uint32_t dst = chunk(c0 + kKChunks + hh);
                                 ptx::tma_load_3d(dst, &tm_v, fb, 0, x.kh, tok + hh * 64, pol_kv);
                                 ptx::tma_load_3d(dst + kVHalfBytes, &tm_v, fb, 64, x.kh, tok + hh * 64, pol_kv);
                             }
@@ -635,10 +654,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Let every copy this warp started land before the block can exit.
                 if (ql0) wait(bar(bars->q_full[0]), (ql0 - 1) & 1);
                 if (ql1) wait(bar(bars->q_full[1]), (ql1 - 1) & 1);
-                for (uint32_t s = 0; s < kRing; ++s) {
-                    const uint32_t n = rc / kRing + (s < rc % kRing ? 1 : 0);
-                    if (n) wait(bar(bars->ch_full[s]), (n - 1) & 1);
-                }
+                // (older tiles have been consumed by the MMA warp, so their bytes have landed)
+                for (uint32_t g = tk > kTileBars ? tk - kTileBars : 0; g < tk; ++g)
+                    wait(bar(bars->k_full[g % kTileBars]), (g / kTileBars) & 1);
+                for (uint32_t g = tv > kTileBars ? tv - kTileBars : 0; g < tv; ++g)
+                    wait(bar(bars->v_full[g % kTileBars]), (g / kTileBars) & 1);
             };
             if constexpr (kGeneral) {
                 if (p.paged) producer(std::true_type{});
@@ -659,11 +679,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_lo = ptx::desc_lo(sQ, 16);
             const uint32_t ring_k_lo = ptx::desc_lo(sRing, 16);
             const uint32_t ring_v_lo = ptx::desc_lo(sRing, kVHalfBytes);
-            uint32_t rc = 0;
+            uint32_t tg = 0;  // key tiles of earlier units: the unit's key tile j is tile tg + j
             uint32_t qf0 = 0, qf1 = 0, pf0 = 0, pf1 = 0, oe0 = 0, oe1 = 0;
             bool ok = true;
-            auto wait_chunk = [&](uint32_t c) -> bool {
-                return wait_bar_warp(bar(bars->ch_full[c % kRing]), (c / kRing) & 1, bars, p.status);
+            auto wait_tile = [&](uint64_t (&full)[kTileBars], uint32_t g) -> bool {
+                return wait_bar_warp(bar(full[g % kTileBars]), (g / kTileBars) & 1, bars, p.status);
             };
             auto commit = [&](uint64_t &b) {
                 if (ptx::elect_one()) ptx::mma_commit(bar(b));
@@ -730,21 +750,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (x.n[0]) ok = wait_bar_warp(bar(bars->q_full[0]), qf0++ & 1, bars, p.status);
                 if (ok && x.n[1]) ok = wait_bar_warp(bar(bars->q_full[1]), qf1++ & 1, bars, p.status);
                 if (!ok) break;
-                // key tile j uses ring chunks K: rc + 5j + {0,1,2}, V: rc + 5j + {3,4}
-                ok = wait_chunk(rc) && wait_chunk(rc + 1) && wait_chunk(rc + 2);
+                // key tile g = tg + j: K_g in ring chunks 5g + {0,1,2}, V_g in 5g + {3,4}.  The last MMA
+                // reading a key tile is tile 1's when tile 1 reads it (issued after tile 0's), else tile 0's.
+                ok = wait_tile(bars->k_full, tg);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 if (x.n[0] > 0) {
-                    issue_s(0, rc);
+                    issue_s(0, 5 * tg);
                     if (x.n[0] == 1) commit(bars->q_empty[0]);
                 }
                 if (x.n[1] > 0) {
-                    issue_s(1, rc);
+                    issue_s(1, 5 * tg);
                     if (x.n[1] == 1) commit(bars->q_empty[1]);
                 }
-                for (int c = 0; c < kKChunks; ++c) commit(bars->ch_empty[(rc + c) % kRing]);
+                commit(bars->k_empty[tg % kTileBars]);
                 for (int j = 0; j < x.n_max && ok; ++j) {
-                    const uint32_t kc = rc + 5 * j, vc = kc + 3, kn = kc + 5;
+                    const uint32_t g = tg + j, kc = 5 * g, vc = kc + 3, kn = kc + 5;
                     bool v_ready = false, k_next_ready = false;
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
@@ -753,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             uint32_t &oe = t ? oe1 : oe0;
                             ok = wait_bar_warp(bar(bars->p_full[t]), pf++ & 1, bars, p.status);
                             if (ok && !v_ready) {
-                                ok = wait_chunk(vc) && wait_chunk(vc + 1);
+                                ok = wait_tile(bars->v_full, g);
                                 v_ready = true;
                             }
                             if (ok && j == 0) ok = wait_bar_warp(bar(bars->o_empty[t]), (oe++ & 1) ^ 1, bars, p.status);
@@ -761,28 +782,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 ptx::tc_fence_after();
                                 issue_pv(t, vc, j > 0);
                                 if (j == x.n[t] - 1) commit(bars->o_full[t]);
+                                if (t == 1 || j >= x.n[1]) commit(bars->v_empty[g % kTileBars]);  // last P V_g
                             }
                         }
                         if (ok && j + 1 < x.n[t]) {
                             if (!k_next_ready) {
-                                ok = wait_chunk(kn) && wait_chunk(kn + 1) && wait_chunk(kn + 2);
+                                ok = wait_tile(bars->k_full, g + 1);
                                 k_next_ready = true;
                                 if (ok) ptx::tc_fence_after();
                             }
                             if (ok) {
                                 issue_s(t, kn);
                                 if (j + 2 == x.n[t]) commit(bars->q_empty[t]);  // last S_t of the unit
+                                if (t == 1 || j + 1 >= x.n[1]) commit(bars->k_empty[(g + 1) % kTileBars]);  // last S of K_{g+1}
                             }
                         }
                     }
-                    if (!ok) break;
-                    commit(bars->ch_empty[vc % kRing]);
-                    commit(bars->ch_empty[(vc + 1) % kRing]);
-                    if (j + 1 < x.n_max)
-                        for (int c = 0; c < kKChunks; ++c) commit(bars->ch_empty[(kn + c) % kRing]);
                 }
                 if (!ok) break;
-                rc += 5 * x.n_max;
+                tg += x.n_max;
             }
             // Drain: wait until every MMA this warp issued has completed.
             commit(bars->drain);
@@ -800,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl2 = p.scale_log2;
         uint32_t sf = 0, of = 0;
         bool ok = true;
-        uint32_t ss = 0, ring_seq = 0;
+        uint32_t ss = 0, tiles_seen = 0;
         while (ok) {
             const uint32_t slot = ss % kSched;
             ok = wait_bar_warp(bar(bars->sched_full[slot]), (ss / kSched) & 1, bars, p.status);
@@ -811,9 +829,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++ss;
             if (it < 0) break;
             const WorkItem x = decode_item<kGeneral>(p, it, num_entries, kCausal);
-            // ring index of this unit's first K chunk: key tile j holds V in chunks vbase + 5j + {0, 1}
-            const uint32_t vbase = ring_seq + kKChunks;
-            ring_seq += (kKChunks + kVChunks) * x.n_max;
+            // the unit's key tile j is this CTA's key tile g = g0 + j, its V in ring chunks 5g + {3, 4}
+            const uint32_t g0 = tiles_seen;
+            tiles_seen += x.n_max;
             const int n_t = t ? x.n[1] : x.n[0];
             const bool row_valid = row < (t ? x.rows[1] : x.rows[0]);
             const int i = x.u0 + t * kBM + row;  // query row within the sequence
@@ -842,8 +860,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // warpgroups write the same zeros; P V_j is issued only after this warpgroup's
                 // P-ready arrival for this tile, and the chunk is refilled only after that MMA).
                 if (kGeneral && (x.j0 + j + 1) * kBN > x.lk) {
-                    const uint32_t vch = vbase + 5 * j + (row >> 6);
-                    ok = wait_bar_warp(bar(bars->ch_full[vch % kRing]), (vch / kRing) & 1, bars, p.status);
+                    const uint32_t g = g0 + j, vch = 5 * g + kKChunks + (row >> 6);
+                    ok = wait_bar_warp(bar(bars->v_full[g % kTileBars]), (g / kTileBars) & 1, bars, p.status);
                     if (!ok) break;
                     if ((x.j0 + j) * kBN + row >= x.lk) {
                         uint4 *vr = reinterpret_cast<uint4 *>(smem + kSmemRing + (vch % kRing) * kChunkBytes +
