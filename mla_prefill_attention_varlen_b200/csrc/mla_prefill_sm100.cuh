@@ -190,24 +190,24 @@ __device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num
             x.n[t] = kv_tiles_for(x.u0 + t * kBM, x.rows[t], s.z, s.w, causal);
         }
         x.n_max = max(x.n[0], x.n[1]);
-        return x;
-    }
-    int full[2];
+    } else {
+        int full[2];
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        x.rows[t] = tile_rows(x.u0 + t * kBM, s.z);
-        full[t] = kv_tiles_for(x.u0 + t * kBM, x.rows[t], s.z, s.w, causal);
-    }
-    const int nf = max(full[0], full[1]);
-    int j1 = nf;
-    if (p.split_tiles > 0 && nf > p.split_tiles) {
-        x.nsplit = (nf + p.split_tiles - 1) / p.split_tiles;
-        x.j0 = chunk * p.split_tiles;
-        j1 = min(nf, x.j0 + p.split_tiles);
-    }
+        for (int t = 0; t < 2; ++t) {
+            x.rows[t] = tile_rows(x.u0 + t * kBM, s.z);
+            full[t] = kv_tiles_for(x.u0 + t * kBM, x.rows[t], s.z, s.w, causal);
+        }
+        const int nf = max(full[0], full[1]);
+        int j1 = nf;
+        if (p.split_tiles > 0 && nf > p.split_tiles) {
+            x.nsplit = (nf + p.split_tiles - 1) / p.split_tiles;
+            x.j0 = chunk * p.split_tiles;
+            j1 = min(nf, x.j0 + p.split_tiles);
+        }
 #pragma unroll
-    for (int t = 0; t < 2; ++t) x.n[t] = max(0, min(full[t], j1) - x.j0);
-    x.n_max = j1 - x.j0;
+        for (int t = 0; t < 2; ++t) x.n[t] = max(0, min(full[t], j1) - x.j0);
+        x.n_max = j1 - x.j0;
+    }
     return x;
 }
 
