@@ -9,7 +9,10 @@ whole workload, inputs resident in HBM.  Prints ONE JSON line (rank 0).
   FLOPs (2*192 for Q.K^T plus 2*128 for P.V) / device time per step, summed over
   ranks (each rank runs an independent replica: "scaling": "weak").
 * roofline: the attention kernel alone (timed with CUDA events recorded by the
-  library around its launch) against the measured dense bf16 peak.
+  library around its launch) against the measured dense bf16 peak; the same
+  launch's algorithmic bytes against the measured HBM bandwidth beside it.
+* warm_l2: workloads smaller than twice the L2 are timed with the L2 flushed
+  before every step; the same steps without the flush are reported here.
 * e2e: the same metric through the public call with pinned HOST inputs: every
   step copies the inputs host->device, runs the call and copies attenOut back.
 * cpu_baseline: the fp64 CPU oracle on a bounded sample of the same workload.
@@ -638,6 +641,25 @@ def main():
     if st != 0:
         raise RuntimeError("device status after timing: %s" % mla.mla_status_string(st))
 
+    # Small workloads are timed with a cold L2 (flushed before every step); the same steps with the
+    # inputs left in L2 are reported beside them, outside the timed region above.
+    warm_ms = warm_kms = None
+    if flush is not None:
+        w_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        w_stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        wk_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        wk_stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        step()
+        for i in range(args.steps):
+            mla.set_profile_events(wk_starts[i], wk_stops[i])
+            w_starts[i].record(stream)
+            step()
+            w_stops[i].record(stream)
+        mla.set_profile_events(None, None)
+        torch.cuda.synchronize()
+        warm_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in zip(w_starts, w_stops)])), world)
+        warm_kms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in zip(wk_starts, wk_stops)])), world)
+
     triples = visible_triples(wl)
     flops = triples * FLOPS_PER_TRIPLE
     value = job_throughput(world, flops, ms) / 1e12
@@ -712,6 +734,8 @@ def main():
 
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    algo_bytes = algorithmic_bytes(wl)
     clocks = smi.summary()
     line = {
         "metric": METRIC + (" (K/V read in place from a paged cache)" if paged else ""),
@@ -734,7 +758,13 @@ def main():
                      "peak_source": peak_src,
                      "peak_kind": "burst", "frac_of_sustained": kern_tflops / peak_sus,
                      "kernel": "mla_prefill_sm100_kernel", "kernel_ms": kms,
-                     "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": algorithmic_bytes(wl)},
+                     "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": algo_bytes,
+                     # the same launch against the HBM roofline (the bound near the ridge, e.g. `uniform`)
+                     "hbm_achieved_gbs": algo_bytes / (kms * 1e-3) / 1e9, "hbm_peak_gbs": hbm_peak,
+                     "hbm_frac": algo_bytes / (kms * 1e-3) / 1e9 / hbm_peak},
+        "warm_l2": None if warm_ms is None else {
+            "ms_per_step": warm_ms, "value": job_throughput(world, flops, warm_ms) / 1e12, "unit": "TFLOP/s",
+            "kernel_ms": warm_kms, "kernel_frac": flops / (warm_kms * 1e-3) / 1e12 / peak},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
