@@ -116,6 +116,25 @@ CASES = [
 ]
 
 
+def many_short_lengths(seed, n_short, long_lens):
+    """n_short lengths in [1, 300] (one or two key tiles) with a few long ones, shuffled."""
+    rng = np.random.default_rng(seed)
+    lens = [int(v) for v in rng.integers(1, 301, n_short)] + list(long_lens)
+    return [lens[i] for i in rng.permutation(len(lens))]
+
+
+def test_many_short_units_per_cta():
+    # About twenty units per CTA, most of one or two key tiles, mixed with long sequences: the
+    # kernel's key-tile barriers (four sets, reused in turn across units) and its Q / O hand-offs
+    # cycle through many phases per CTA.  Every row against the oracle.
+    lens = many_short_lengths(77, 600, [2000, 1999, 2048])
+    _, x = problem(lens, lens, 4, 2, seed=4242, extra_tokens=3)
+    out = run(x, 4, 2, 0.07)
+    check_against_oracle(x, out, 4, 2, 0.07)
+    assert torch.all(out[sum(lens):] == 7.0)
+    assert status() == 0
+
+
 @pytest.mark.parametrize("case", range(len(CASES)))
 def test_ragged_cases(case):
     lq, lk, H, G, dtype, scale, mask = CASES[case]

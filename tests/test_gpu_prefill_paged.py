@@ -179,3 +179,18 @@ def test_chunked_workload_sampled_rows():
     torch.cuda.synchronize()
     assert status() == 0
     assert torch.equal(out, ref)
+
+
+def test_many_short_sequences_paged_equals_packed():
+    # many one- and two-tile units per CTA through the warp-wide paged producer
+    rng = np.random.default_rng(78)
+    lens = [int(v) for v in rng.integers(1, 301, 400)] + [1500, 2048]
+    lens = [lens[i] for i in rng.permutation(len(lens))]
+    wl, x = problem(lens, lens, 4, 2, torch.bfloat16, seed=7800)
+    ref = packed(x, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL)
+    kc, vc, table = W.paged_cache(x["k"], x["k_rope"], x["v"], lens, 32, seed=78, spare_blocks=5, slot_fill=NAN,
+                                  table_fill=1 << 30)
+    out = paged(x, kc, vc, table, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL)
+    torch.cuda.synchronize()
+    assert status() == 0
+    assert torch.equal(out, ref)

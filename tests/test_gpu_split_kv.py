@@ -119,3 +119,19 @@ def test_automatic_split_long_sequence_one_head():
 def test_split_control_rejects_bad_values():
     with pytest.raises(mla.MlaError):
         mla.set_split_tiles(-2)
+
+
+def test_one_tile_chunks_over_many_short_sequences():
+    # every work item a single key tile: the pipeline turns over once per item; units of one key
+    # tile are written directly, the others (up to nine chunks) merged by the combine kernel
+    rng = np.random.default_rng(79)
+    lens = [int(v) for v in rng.integers(1, 301, 300)] + [1100, 1024]
+    lens = [lens[i] for i in rng.permutation(len(lens))]
+    wl = W.Workload("split_many", lens, lens, 4, 2, seed=812)
+    x = W.make_inputs(wl, device=DEV)
+    whole = run(x, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL, 0)
+    parts = run(x, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL, 1)
+    assert mla.mla_prefill_device_status() == 0
+    check(x, parts, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL)
+    d = (parts.float() - whole.float()).abs()
+    assert d.max().item() <= 4 * 2.0 ** -8 * max(1.0, whole.float().abs().max().item())
