@@ -1,0 +1,216 @@
+"""Host model of the attention kernel's shared-memory ring protocol (no GPU).
+
+The attention kernel (mla_prefill_sm100.cuh) streams key tiles through a ring of eight
+16 KB chunks: key tile g, counted per CTA across its work units, occupies chunks
+5g .. 5g + 4 (K_g in the first three, V_g in the last two; slot = chunk mod 8).  Four
+barrier sets, indexed g mod 4, track the tiles:
+
+  producer  K_g: waits v_empty(g - 2), arms k_full(g), issues the loads
+            V_g: waits k_empty(g - 1), arms v_full(g), issues the loads
+  MMA       per unit: wait k_full(first); S_0, S_1; release K(first)
+            per key tile j: for t = 0, 1: wait P_t(j) (and v_full once), P V_t(j),
+            release V when it is the last reader; wait k_full(j + 1) once, S_t(j + 1),
+            release K(j + 1) when it is the last reader.  One thread issues every MMA;
+            they complete in issue order, and a release (tcgen05.commit) completes once
+            every MMA issued before it has.
+  softmax   tile t: wait S_t(j) -> publish P_t(j)
+
+This file re-states that protocol as Python coroutines and runs it under random
+interleavings of the roles, the TMA completions and the in-order MMA completions, on
+random unit sequences (including units where tile 1 has no rows or one key tile
+fewer than tile 0).  It checks that nothing deadlocks, that no wait ever sees its
+barrier more than one phase away from the intended one (mbarrier parity waits cannot
+tell phases two apart), that no chunk is refilled while an MMA still reads it, and
+that no MMA reads a chunk before its load has landed.  Planted protocol mistakes must
+be caught, which shows the checks have teeth.  The model mirrors the kernel's logic
+by hand: a change to the kernel's barrier protocol must be made here too.
+"""
+import random
+
+import pytest
+
+RING, TILE_SETS = 8, 4
+
+
+class Barrier:
+    """mbarrier with an arrival count; `done` counts completed phases."""
+
+    def __init__(self, name, count=1):
+        self.name, self.count, self.pending, self.done = name, count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending == 0:
+            self.done += 1
+            self.pending = self.count
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+def ready(bar, phase):
+    """A parity wait for completed phase `phase`; the barrier must be within one phase of it."""
+    if bar.done not in (phase, phase + 1):
+        raise ProtocolError("phase aliasing on %s: %d completed, waiting for %d" % (bar.name, bar.done, phase))
+    return bar.done >= phase + 1
+
+
+def simulate(units, seed, bug=None):
+    """units: [(n0, n1)] key tiles of query tile 0 / 1 per unit (n_max = max(n0, n1) > 0)."""
+    rnd = random.Random(seed)
+    bars = {}
+    for kind in ("k_full", "v_full", "k_empty", "v_empty"):
+        for i in range(TILE_SETS):
+            bars[kind, i] = Barrier("%s[%d]" % (kind, i))
+    for t in range(2):
+        bars["s_full", t] = Barrier("s_full[%d]" % t)
+        bars["p_full", t] = Barrier("p_full[%d]" % t)
+    slot_owner = {}   # ring slot -> (tile, "K" | "V") last loaded into it
+    readers = {}      # (tile, kind) -> MMAs issued and not yet completed
+    landed = set()
+    tma = []          # loads in flight: (barrier, (tile, kind))
+    mma_queue = []    # in issue order: ("mma", (tile, kind)) or ("commit", barrier)
+
+    def b(kind, g):
+        return bars[kind, g % TILE_SETS]
+
+    def fill(g, kind, chunks):
+        for c in chunks:
+            slot = (5 * g + c) % RING
+            prev = slot_owner.get(slot)
+            if prev is not None and readers.get(prev, 0):
+                raise ProtocolError("slot %d refilled with %s %d while an MMA reads %s" % (slot, kind, g, prev))
+            slot_owner[slot] = (g, kind)
+
+    def producer():
+        g = 0
+        for n0, n1 in units:
+            for _ in range(max(n0, n1)):
+                lag = 3 if bug == "k_waits_tile_g_minus_3" else 2
+                if g >= lag:
+                    while not ready(b("v_empty", g - lag), (g - lag) // TILE_SETS):
+                        yield
+                fill(g, "K", (0, 1, 2))
+                tma.append((b("k_full", g), (g, "K")))
+                if g >= 1 and bug != "no_v_slot_wait":
+                    while not ready(b("k_empty", g - 1), (g - 1) // TILE_SETS):
+                        yield
+                fill(g, "V", (3, 4))
+                tma.append((b("v_full", g), (g, "V")))
+                g += 1
+                yield
+
+    def issue(operand):
+        if operand not in landed:
+            raise ProtocolError("MMA reads %s before it landed" % (operand,))
+        readers[operand] = readers.get(operand, 0) + 1
+        mma_queue.append(("mma", operand))
+
+    def commit(bar):
+        mma_queue.append(("commit", bar))
+
+    def last_reader(t, j, n):
+        if bug == "release_by_tile_0":
+            return t == 0 or j >= n[1]
+        return t == 1 or j >= n[1]
+
+    def mma():
+        tg, pf = 0, [0, 0]
+        for n0, n1 in units:
+            n = (n0, n1)
+            while not ready(b("k_full", tg), tg // TILE_SETS):
+                yield
+            for t in range(2):
+                if n[t] > 0:
+                    issue((tg, "K"))
+                    commit(bars["s_full", t])
+            commit(b("k_empty", tg))
+            for j in range(max(n)):
+                g = tg + j
+                v_ready = k_ready = False
+                for t in range(2):
+                    if j < n[t]:
+                        while not ready(bars["p_full", t], pf[t]):
+                            yield
+                        pf[t] += 1
+                        if not v_ready and bug != "no_v_full_wait":
+                            while not ready(b("v_full", g), g // TILE_SETS):
+                                yield
+                            v_ready = True
+                        issue((g, "V"))
+                        if last_reader(t, j, n):
+                            commit(b("v_empty", g))
+                    if j + 1 < n[t]:
+                        if not k_ready:
+                            while not ready(b("k_full", g + 1), (g + 1) // TILE_SETS):
+                                yield
+                            k_ready = True
+                        issue((g + 1, "K"))
+                        commit(bars["s_full", t])
+                        if last_reader(t, j + 1, n):
+                            commit(b("k_empty", g + 1))
+                    yield
+            tg += max(n)
+
+    def softmax(t):
+        sf = 0
+        for unit in units:
+            for _ in range(unit[t]):
+                while not ready(bars["s_full", t], sf):
+                    yield
+                sf += 1
+                yield
+                bars["p_full", t].arrive()
+
+    roles = [producer(), mma(), softmax(0), softmax(1)]
+    alive = [True] * len(roles)
+    for _ in range(400000):
+        if not (any(alive) or tma or mma_queue):
+            return
+        acts = [("role", i) for i, a in enumerate(alive) if a]
+        if tma:
+            acts.append(("tma", rnd.randrange(len(tma))))
+        if mma_queue:
+            acts.append(("mma", 0))
+        act, arg = rnd.choice(acts)
+        if act == "role":
+            try:
+                next(roles[arg])
+            except StopIteration:
+                alive[arg] = False
+        elif act == "tma":
+            bar, operand = tma.pop(arg)
+            landed.add(operand)
+            bar.arrive()
+        else:
+            op, x = mma_queue.pop(0)
+            if op == "mma":
+                readers[x] -= 1
+            else:
+                x.arrive()
+    raise ProtocolError("deadlock")
+
+
+def random_units(rng):
+    units = []
+    for _ in range(rng.randint(1, 7)):
+        n1 = rng.randint(0, 8)
+        n0 = rng.choice([n1, max(0, n1 - 1), 0, rng.randint(1, 6) if n1 == 0 else n1])
+        if max(n0, n1):
+            units.append((n0, n1))
+    return units or [(1, 1)]
+
+
+def test_protocol_holds_under_random_schedules():
+    rng = random.Random(2024)
+    for trial in range(400):
+        simulate(random_units(rng), seed=trial)
+
+
+@pytest.mark.parametrize("bug", ["no_v_slot_wait", "k_waits_tile_g_minus_3", "no_v_full_wait", "release_by_tile_0"])
+def test_planted_protocol_mistakes_are_caught(bug):
+    rng = random.Random(7)
+    with pytest.raises(ProtocolError):
+        for trial in range(400):
+            simulate(random_units(rng), seed=trial, bug=bug)
