@@ -20,7 +20,6 @@ whole workload, inputs resident in HBM.  Prints ONE JSON line (rank 0).
 """
 import argparse
 import json
-import math
 import os
 import subprocess
 import sys
