@@ -27,6 +27,8 @@ import subprocess
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import oracle
 from oracle import MASK_CAUSAL, MASK_NONE
@@ -246,6 +248,27 @@ ALL_CHECKS = [check_hand_cases, check_sdpa, check_closed_forms, check_invariants
 def test_oracle_pin(check):
     fails = check(oracle)
     assert not fails, "\n".join(fails[:20])
+
+
+@settings(max_examples=80, deadline=None, derandomize=True)
+@given(st.data())
+def test_oracle_matches_library_attention_on_random_shapes(data):
+    # the library pin over drawn ragged shapes: empty sequences, Lq > Lk and Lq < Lk, GQA ratios,
+    # no rope part, both masks, negative and zero scales
+    batch = data.draw(st.integers(1, 4))
+    lens_q = data.draw(st.lists(st.integers(0, 12), min_size=batch, max_size=batch))
+    lens_k = data.draw(st.lists(st.integers(0, 12), min_size=batch, max_size=batch))
+    G = data.draw(st.sampled_from([1, 2, 3]))
+    H = G * data.draw(st.sampled_from([1, 2, 3]))
+    r = data.draw(st.sampled_from([0, 2, 3]))
+    scale = data.draw(st.floats(-2.0, 2.0, allow_nan=False))
+    mask_type = data.draw(st.sampled_from([MASK_CAUSAL, MASK_NONE]))
+    p = _problem(np.random.default_rng(data.draw(st.integers(0, 2 ** 31 - 1))), lens_q, lens_k, H, G, r=r)
+    got = _run(oracle, p, scale, mask_type)
+    ref, has_key = _sdpa_reference(p, scale, mask_type == MASK_CAUSAL)
+    if has_key.any():
+        assert np.abs(got[has_key] - ref[has_key]).max() <= TOL
+    assert np.all(got[~has_key] == 0.0)
 
 
 def test_oracle_rejects_inconsistent_seqlens():
