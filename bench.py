@@ -66,22 +66,18 @@ def kernel_sources_hash():
 
 
 def measured_traffic(workload):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    summary is missing or was taken on different kernel sources."""
-    path = os.path.join(ROOT, "profiles", "mla_prefill_sm100_kernel_%s_dram.md" % workload)
+    """DRAM bytes per launch from the committed ncu figures (profiles/traffic.json), or None when
+    there is no figure for this workload or it was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    fields = {}
-    for line in open(path):
-        line = line.strip().strip("`")
-        if line.startswith("traffic_bytes_per_launch=") or line.startswith("kernel_sources_sha256="):
-            k, v = line.split("=", 1)
-            fields[k] = v.strip()
-    if fields.get("kernel_sources_sha256") != kernel_sources_hash():
+    with open(path) as f:
+        entry = json.load(f).get("launches", {}).get(workload)
+    if not entry or entry.get("kernel_sources_sha256") != kernel_sources_hash():
         return None
     try:
-        return int(fields["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+        return int(entry["traffic_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 

@@ -126,9 +126,12 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
 
 /*
  * mla_prefill_device_status -- synchronises `stream`, then reads and clears the
- * device status word of the current GPU (MLA_OK, MLA_ERR_SEQLEN,
- * MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_INDEX; the first error recorded since the
- * last read by mla_prefill, mla_prefill_paged or mla_paged_cache_load).
+ * device status words of the current GPU (MLA_OK, MLA_ERR_SEQLEN,
+ * MLA_ERR_DEVICE_TIMEOUT or MLA_ERR_INDEX): the library's word, which
+ * mla_prefill, mla_prefill_paged and mla_paged_cache_load write, and the word
+ * in mla_prefill_noalloc's static array.  Each keeps the first error recorded
+ * since it was last read; the library's is reported when both hold one.
+ * Allocates nothing (a 4-byte copy and a 4-byte memset per word).
  * Writes it to *status and returns MLA_OK, or returns MLA_ERR_NULL /
  * MLA_ERR_CUDA.
  */
@@ -165,8 +168,8 @@ int mla_prefill_device_status(mla_stream_t stream, int *status);
  * results; order them on one stream.  Nothing in the array needs clearing
  * between calls: each call rewrites every entry it later reads.
  * Inconsistent seqlens are clamped exactly as in mla_prefill (no out-of-bounds
- * access), but the status word they set lives in the static array and is not
- * reported: mla_prefill_device_status() covers mla_prefill calls only.
+ * access) and recorded in a status word kept in the static array;
+ * mla_prefill_device_status() reads and clears it without allocating.
  * Returns MLA_OK or an mla_status error code, like mla_prefill.
  */
 int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,

@@ -496,6 +496,48 @@ int choose_split(const Problem &pr, int sm_count) {
     return split >= tiles ? 0 : static_cast<int>(split);
 }
 
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.  Same validation and the same two kernels as
+// mla_prefill, but the plan workspace and the status word live in one static
+// device array of fixed size instead of library-allocated device memory.
+// ---------------------------------------------------------------------------
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;               // 1 MiB on every GPU that loads the library
+constexpr size_t kNoAllocStatusOffset = kNoAllocScratchBytes - 256;    // last 256 bytes: status word
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocDevice {
+    bool ready = false;
+    int sm_count = 0;
+    uint8_t *scratch = nullptr;  // device address of g_noalloc_scratch on this GPU
+    DeviceState launch;          // only its dynamic-shared-memory opt-in flags are used
+};
+
+NoAllocDevice g_noalloc[kMaxDevices];
+
+// One-time set-up per GPU, with that GPU current: the array's device address
+// (the host-side symbol is only a stand-in), the SM count, the arch check.
+int noalloc_setup(int dev, NoAllocDevice **out) {
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    NoAllocDevice &d = g_noalloc[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MLA_ERR_CUDA;
+        d.scratch = static_cast<uint8_t *>(ptr);
+        d.ready = true;
+    }
+    *out = &d;
+    return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -530,15 +572,21 @@ int mla_prefill_device_status(mla_stream_t stream_, int *status) {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    DeviceState &d = g_dev[dev];
-    if (!d.ready) {
-        *status = MLA_OK;
-        return MLA_OK;
+    // the library's word (mla_prefill and the other allocating entry points) and the word in the
+    // static array of mla_prefill_noalloc: the first error of either is reported, both are cleared
+    int *words[2] = {g_dev[dev].ready ? g_dev[dev].status : nullptr,
+                     g_noalloc[dev].ready
+                         ? reinterpret_cast<int *>(g_noalloc[dev].scratch + kNoAllocStatusOffset)
+                         : nullptr};
+    int first = MLA_OK;
+    for (int *w : words) {
+        if (!w) continue;
+        int h = 0;
+        if (cudaMemcpy(&h, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+        if (h != MLA_OK && cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+        if (first == MLA_OK) first = h;
     }
-    int h = 0;
-    if (cudaMemcpy(&h, d.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
-    if (cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
-    *status = h;
+    *status = first;
     return MLA_OK;
 }
 
@@ -594,49 +642,6 @@ int mla_prefill_version(void) { return kVersion; }
 
 }  // extern "C"
 
-// ---------------------------------------------------------------------------
-// Allocation-free entry point.  Same validation and the same two kernels as
-// mla_prefill, but the plan workspace and the status word live in one static
-// device array of fixed size instead of library-allocated device memory.
-// ---------------------------------------------------------------------------
-namespace {
-
-constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;               // 1 MiB on every GPU that loads the library
-constexpr size_t kNoAllocStatusOffset = kNoAllocScratchBytes - 256;    // last 256 bytes: status word
-
-__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-
-struct NoAllocDevice {
-    bool ready = false;
-    int sm_count = 0;
-    uint8_t *scratch = nullptr;  // device address of g_noalloc_scratch on this GPU
-    DeviceState launch;          // only its dynamic-shared-memory opt-in flags are used
-};
-
-NoAllocDevice g_noalloc[kMaxDevices];
-
-// One-time set-up per GPU, with that GPU current: the array's device address
-// (the host-side symbol is only a stand-in), the SM count, the arch check.
-int noalloc_setup(int dev, NoAllocDevice **out) {
-    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
-    NoAllocDevice &d = g_noalloc[dev];
-    if (!d.ready) {
-        int major = 0, minor = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return MLA_ERR_CUDA;
-        if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MLA_ERR_CUDA;
-        d.scratch = static_cast<uint8_t *>(ptr);
-        d.ready = true;
-    }
-    *out = &d;
-    return MLA_OK;
-}
-
-}  // namespace
 
 extern "C" int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
                                    const mla_tensor *k_rope, const mla_tensor *v, const mla_tensor *q_seqlen,

@@ -1,13 +1,17 @@
 """Shared test helpers: oracle runs on seeded inputs and the parity bound.
 
-Parity bound (stated for N(0,1) inputs, applied to every workload):
-  * mean |gpu - oracle| <= 1e-3 over all checked elements;
-  * max over elements of (|gpu - oracle| - ulp(oracle)/2) <= 1e-2, where ulp is
-    the spacing of the output dtype at the oracle value.  attenOut is stored in
-    fp16 / bf16, so an exactly computed result still carries up to half an
-    ulp of storage rounding (0.0156 for bf16 values in [4, 8)); the 1e-2 bound
-    applies to the error of the computation on top of that rounding.
-The literal max |gpu - oracle| is reported alongside.
+Parity bound (stated for N(0,1) inputs at qkScale = 1/sqrt(192), applied to every
+workload and by default to every other case):
+  * max |gpu - oracle| <= 1e-2 and mean |gpu - oracle| <= 1e-3 over all checked
+    elements ("literal", the default of ``compare``).
+A case outside those input conditions may instead be held to
+  * mean <= 1e-3 and max over elements of (|gpu - oracle| - ulp(oracle)/2) <= 1e-2
+    ("half_ulp"), where ulp is the spacing of the output dtype at the oracle
+    value: attenOut is stored in fp16 / bf16, so an exactly computed result
+    still carries up to half an ulp of storage rounding (0.0156 for bf16 values
+    in [4, 8)), and the 1e-2 bound then applies to the error of the computation
+    on top of that rounding.  Each test that asks for it states why.
+Both figures are always reported.
 """
 import numpy as np
 import torch
@@ -27,8 +31,12 @@ def half_ulp(ref, dtype):
     return 0.5 * 2.0 ** (e - mant)
 
 
-def compare(got, ref, dtype, mask=None):
-    """Returns (ok, stats) for gpu output ``got`` vs oracle ``ref`` (both [T,H,D])."""
+def compare(got, ref, dtype, mask=None, bound="literal"):
+    """Returns (ok, stats) for gpu output ``got`` vs oracle ``ref`` (both [T,H,D]).
+
+    bound: "literal" (max-abs <= 1e-2) or "half_ulp" (the excess over half an
+    output ulp <= 1e-2); mean-abs <= 1e-3 in both."""
+    assert bound in ("literal", "half_ulp")
     g = got.detach().cpu().double().numpy() if hasattr(got, "detach") else np.asarray(got, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     if mask is not None:
@@ -41,7 +49,9 @@ def compare(got, ref, dtype, mask=None):
     excess = err - half_ulp(r, dtype)
     stats = {"n": int(r.size), "max_abs": float(err.max()), "mean_abs": float(err.mean()),
              "max_excess_over_half_ulp": float(excess.max())}
-    ok = stats["max_excess_over_half_ulp"] <= MAX_ABS and stats["mean_abs"] <= MEAN_ABS
+    worst = stats["max_abs"] if bound == "literal" else stats["max_excess_over_half_ulp"]
+    stats["bound"] = bound
+    ok = worst <= MAX_ABS and stats["mean_abs"] <= MEAN_ABS
     return ok, stats
 
 

@@ -42,11 +42,12 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), "missing export %s" % n
 
 
-def test_library_is_sm100a_only():
-    out = os.popen("cuobjdump --list-elf %s 2>/dev/null" % build.LIB).read()
-    if not out:
-        pytest.skip("cuobjdump unavailable")
-    assert "sm_100a" in out
+def test_library_is_built_for_sm100a_only():
+    # the nvcc command line names exactly one target, sm_100a (no PTX for other architectures)
+    flags = build.NVCC_FLAGS
+    targets = [flags[i + 1] for i, f in enumerate(flags) if f == "-gencode"]
+    assert targets == ["arch=compute_100a,code=sm_100a"]
+    assert not any(f.startswith(("-arch", "--gpu-architecture", "--generate-code")) for f in flags)
 
 
 def test_status_strings(lib):
