@@ -525,6 +525,67 @@ def bench_prolog(args):
     return 0
 
 
+def time_other_config(name, steps, warmup, peaks):
+    """One more workload timed in the same run: step and kernel time (CUDA events), TFLOP/s, the
+    kernel's fraction of the measured bf16 peak and, from the same launch, algorithmic bytes per
+    kernel time against the measured HBM bandwidth; its own clock samples.  Workloads smaller than
+    twice the L2 are timed with the L2 flushed before every step."""
+    import torch
+
+    import mla_prefill_attention_varlen_b200 as mla
+    from mla_prefill_attention_varlen_b200 import workloads as W
+
+    wl = W.get(name)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = W.make_inputs(wl, device=dev)
+    out = torch.empty(wl.t_q, wl.head_num, wl.d_nope, dtype=wl.dtype, device=dev)
+    stream = torch.cuda.current_stream()
+    in_bytes = sum(t.numel() * t.element_size() for t in x.values())
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev) if in_bytes < 2 * L2_BYTES else None
+
+    def step():
+        mla.mla_prefill(x["q"], x["q_rope"], x["k"], x["k_rope"], x["v"], x["q_seqlen"], x["kv_seqlen"],
+                        mla.MLA_MASK_CAUSAL, wl.head_num, wl.kv_head_num, wl.qk_scale, out, stream)
+
+    for _ in range(warmup):
+        if flush is not None:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(steps)] for _ in range(4)]
+    smi = ClockSampler(torch.cuda.current_device())
+    with smi:
+        time.sleep(0.05)
+        smi.mark_start()
+        for i in range(steps):
+            if flush is not None:
+                flush.zero_()
+            mla.set_profile_events(ev[2][i], ev[3][i])
+            ev[0][i].record(stream)
+            step()
+            ev[1][i].record(stream)
+        mla.set_profile_events(None, None)
+        torch.cuda.synchronize()
+        smi.mark_stop()
+    st = mla.mla_prefill_device_status()
+    if st != 0:
+        raise RuntimeError("device status after %s: %s" % (name, mla.mla_status_string(st)))
+    ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev[0], ev[1])]))
+    kms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev[2], ev[3])]))
+    flops = visible_triples(wl) * FLOPS_PER_TRIPLE
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ab = algorithmic_bytes(wl)
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "kernel_ms": kms,
+            "kernel_tflops": flops / (kms * 1e-3) / 1e12, "frac": flops / (kms * 1e-3) / 1e12 / peak,
+            "hbm_gbs": ab / (kms * 1e-3) / 1e9, "hbm_frac": ab / (kms * 1e-3) / 1e9 / hbm,
+            "tokens_per_s": wl.t_q / (ms * 1e-3), "steps": steps, "warmup": warmup,
+            "l2": "flushed between steps (512 MB write)" if flush is not None else "inputs %.2f GB > 126 MB L2" % (
+                in_bytes / 1e9),
+            "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f16", "description": wl.description,
+            "clocks": smi.summary()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -542,6 +603,9 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="prolog: tokens (default: the prolog workload's)")
     ap.add_argument("--split", type=int, default=-1,
                     help="split-KV chunk in 128-key tiles for the prefill ops: -1 automatic (default), 0 off")
+    ap.add_argument("--other-configs", default="varlen_gqa,chunked,uniform",
+                    help="prefill on the default workload: more workloads timed in the same run and reported "
+                         "under other_configs (comma-separated; empty for none)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: scale head_num and kv_head_num down to this many query heads")
     args = ap.parse_args()
@@ -731,6 +795,12 @@ def main():
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     algo_bytes = algorithmic_bytes(wl)
+    # the other workloads, each timed in this run (single GPU, packed K/V, default workload only)
+    other = None
+    if (world == 1 and not paged and not args.heads and args.split < 0 and args.workload == "long"
+            and args.other_configs):
+        other = {n: time_other_config(n, args.steps, args.warmup, peaks)
+                 for n in args.other_configs.split(",") if n and n != wl.name}
     clocks = smi.summary()
     line = {
         "metric": METRIC + (" (K/V read in place from a paged cache)" if paged else ""),
@@ -762,6 +832,7 @@ def main():
             "kernel_ms": warm_kms, "kernel_frac": flops / (warm_kms * 1e-3) / 1e12 / peak},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
+        "other_configs": other,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }

@@ -20,10 +20,11 @@
  *           new queries sees the whole cached prefix of Lk - Lq keys)
  *   out[i,h,:] = sum_j softmax_j(s_ij) * V[j,kh,:128]     (0 if no key visible)
  *
- * Differences from the page's two-phase API: the workspace query and the
- * operation object are folded into one asynchronous call on a CUDA stream;
- * calcType is fixed to prefill, cacheMode to 0, and the Mask tensor is not
- * taken (the causal mask is computed from indices).
+ * The page's two-phase API (AtbMLAPreFillGetWorkspaceSize, then AtbMLAPreFill
+ * with a caller-allocated workspace) is mla_prefill_get_workspace_size followed
+ * by mla_prefill_ws; mla_prefill folds both into one call with a workspace the
+ * library owns.  calcType is fixed to prefill, cacheMode to 0, and the Mask
+ * tensor is not taken (the causal mask is computed from indices).
  */
 #ifndef MLA_PREFILL_H
 #define MLA_PREFILL_H
@@ -70,7 +71,8 @@ typedef enum {
     MLA_ERR_CUDA = 7,          /* a CUDA runtime/driver call failed */
     MLA_ERR_SEQLEN = 8,        /* device-detected: a negative seqlen, or sum(seqlen) above the tensor extent */
     MLA_ERR_DEVICE_TIMEOUT = 9, /* device-detected: a pipeline wait gave up (never expected) */
-    MLA_ERR_INDEX = 10          /* device-detected: a paged-cache block index out of range (row zeroed) */
+    MLA_ERR_INDEX = 10,         /* device-detected: a paged-cache block index out of range (row zeroed) */
+    MLA_ERR_WORKSPACE = 11      /* caller workspace smaller than required or not 256-byte aligned */
 } mla_status;
 
 /*
@@ -109,10 +111,13 @@ typedef enum {
  * Ownership and errors: the caller owns every buffer.  Argument errors are
  * detected on the host and returned before anything is launched; `out` is then
  * untouched.  The call enqueues work on `stream` and returns without waiting.
- * The library keeps one device workspace per GPU (created on the first call on
- * that GPU, grown when a call needs more; a call that grows it allocates
- * device memory).  Calls that share a GPU must be ordered on one stream, or
- * otherwise serialised, because they share that workspace.
+ * The library keeps one device workspace per GPU, created on the first call on
+ * that GPU and grown when a call needs more (to the need rounded up to 1 MiB).
+ * Growth is stream-ordered (cudaFreeAsync / cudaMallocAsync on `stream`): the
+ * call never waits on the host, but a call that grows the workspace does
+ * allocate device memory.  Calls that share a GPU must be ordered on one
+ * stream, or otherwise serialised, because they share that workspace; callers
+ * that want concurrent streams, or no allocation at all, use mla_prefill_ws.
  * Inconsistent seqlens (negative, summing past T_q / T_k, or Lk_b > max_seq in
  * the padded form) are detected on
  * the device: the kernel clamps to the tensor extents -- it never reads or
@@ -123,6 +128,52 @@ typedef enum {
 int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
                 const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
                 int head_num, int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream);
+
+/*
+ * mla_prefill_get_workspace_size / mla_prefill_ws -- mla_prefill with a
+ * workspace the caller allocates, in the two phases of the MLA Prefill page's
+ * API (AtbMLAPreFillGetWorkspaceSize returns the workspace size for the
+ * operation's arguments; AtbMLAPreFill runs it in the caller's workspace).
+ *
+ * mla_prefill_get_workspace_size takes the arguments of mla_prefill (only
+ * their shapes, strides, dtypes and scalars are read; no device memory is
+ * touched) and writes to *workspace_bytes the bytes of device memory that
+ * mla_prefill_ws needs for them.  The size depends on batch, T_q, T_k (or the
+ * padded form's max_seq), head_num and the split-KV choice (the calling
+ * thread's mla_prefill_set_split_tiles setting and, in its automatic mode, the
+ * current GPU's SM count), so both calls must see the same arguments and
+ * settings.  It is at least 256 bytes.  Returns MLA_OK, an argument error as
+ * mla_prefill would, MLA_ERR_NULL for a NULL workspace_bytes, or MLA_ERR_CUDA.
+ *
+ * mla_prefill_ws computes exactly what mla_prefill computes (the same kernels,
+ * bit-identical results) using `workspace` (device memory, 256-byte aligned,
+ * at least the size above, caller-owned; its previous contents do not matter)
+ * for all of its scratch: it allocates nothing and never synchronises.  Calls
+ * with different workspaces may run concurrently on different streams of one
+ * GPU; calls that share a workspace must be ordered on one stream.  The first
+ * 4 bytes of the workspace hold the call's device status (an int32 mla_status:
+ * MLA_OK, MLA_ERR_SEQLEN or MLA_ERR_DEVICE_TIMEOUT), reset by each call and
+ * readable once the call has completed, e.g. with mla_prefill_ws_status.
+ * Returns MLA_OK, an argument error as mla_prefill would (nothing launched),
+ * MLA_ERR_NULL for a NULL workspace, or MLA_ERR_WORKSPACE when the workspace
+ * is too small or misaligned.
+ */
+int mla_prefill_get_workspace_size(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
+                                   const mla_tensor *k_rope, const mla_tensor *v, const mla_tensor *q_seqlen,
+                                   const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num,
+                                   float qk_scale, const mla_tensor *out, uint64_t *workspace_bytes);
+int mla_prefill_ws(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+                   const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+                   int head_num, int kv_head_num, float qk_scale, mla_tensor *out, void *workspace,
+                   uint64_t workspace_bytes, mla_stream_t stream);
+
+/*
+ * mla_prefill_ws_status -- synchronises `stream`, then reads the status word of
+ * the last mla_prefill_ws call that used `workspace` (the int32 in its first 4
+ * bytes) into *status.  Allocates nothing.  Returns MLA_OK, MLA_ERR_NULL,
+ * MLA_ERR_WORKSPACE (misaligned) or MLA_ERR_CUDA.
+ */
+int mla_prefill_ws_status(const void *workspace, mla_stream_t stream, int *status);
 
 /*
  * mla_prefill_device_status -- synchronises `stream`, then reads and clears the
@@ -312,6 +363,23 @@ const char *mla_status_string(int status);
  */
 struct CUevent_st;
 int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *stop);
+
+/*
+ * mla_prefill_set_kernel -- attention-kernel choice for later mla_prefill,
+ * mla_prefill_ws and mla_prefill_noalloc calls on this host thread (no
+ * counterpart on the pages; the result is the same operation either way).
+ *   kernel = -1  automatic (the default): the CTA-pair kernel for packed,
+ *                unsplit K/V once its 512-row work units give at least one
+ *                work item per SM pair, else the single-CTA kernel;
+ *   kernel =  1  the single-CTA kernel (256-row units, one SM each);
+ *   kernel =  2  the CTA-pair kernel wherever it applies (packed K/V without
+ *                split-KV); padded or paged K/V and split-KV always run the
+ *                single-CTA kernel.
+ * The CTA-pair kernel runs each 512-row unit on a cluster of two SMs: M = 256
+ * tensor-core MMAs across the pair (tcgen05 cta_group::2), each SM loading half
+ * of every key tile.  Returns MLA_OK, or MLA_ERR_UNSUPPORTED for other values.
+ */
+int mla_prefill_set_kernel(int kernel);
 
 /*
  * mla_prefill_set_split_tiles -- split-KV control for later mla_prefill and

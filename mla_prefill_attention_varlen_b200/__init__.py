@@ -13,7 +13,8 @@ from . import workloads  # noqa: F401  (seeded synthetic inputs)
 
 __all__ = [
     "MLA_MASK_NONE", "MLA_MASK_CAUSAL", "MlaError", "load_library", "mla_prefill", "mla_prefill_noalloc",
-    "mla_paged_cache_load", "mla_prefill_paged", "mla_prolog", "set_split_tiles", "mla_prefill_device_status", "mla_status_string", "prefill",
+    "mla_prefill_get_workspace_size", "mla_prefill_ws", "mla_prefill_ws_status",
+    "mla_paged_cache_load", "mla_prefill_paged", "mla_prolog", "set_split_tiles", "set_kernel", "mla_prefill_device_status", "mla_status_string", "prefill",
     "workloads",
 ]
 
@@ -22,7 +23,7 @@ MLA_MASK_NONE, MLA_MASK_CAUSAL = 0, 1
 STATUS_NAMES = {
     0: "MLA_OK", 1: "MLA_ERR_NULL", 2: "MLA_ERR_DTYPE", 3: "MLA_ERR_SHAPE", 4: "MLA_ERR_ALIGN",
     5: "MLA_ERR_HEADS", 6: "MLA_ERR_UNSUPPORTED", 7: "MLA_ERR_CUDA", 8: "MLA_ERR_SEQLEN",
-    9: "MLA_ERR_DEVICE_TIMEOUT", 10: "MLA_ERR_INDEX",
+    9: "MLA_ERR_DEVICE_TIMEOUT", 10: "MLA_ERR_INDEX", 11: "MLA_ERR_WORKSPACE",
 }
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -63,6 +64,14 @@ def load_library(path=None):
     lib.mla_prefill_noalloc.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_float, T, ctypes.c_void_p]
     lib.mla_prefill_noalloc.restype = ctypes.c_int
+    lib.mla_prefill_get_workspace_size.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_float, T, ctypes.POINTER(ctypes.c_uint64)]
+    lib.mla_prefill_get_workspace_size.restype = ctypes.c_int
+    lib.mla_prefill_ws.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, T,
+                                   ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p]
+    lib.mla_prefill_ws.restype = ctypes.c_int
+    lib.mla_prefill_ws_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]
+    lib.mla_prefill_ws_status.restype = ctypes.c_int
     lib.mla_paged_cache_load.argtypes = [T, T, T, T, T, ctypes.c_int, T, T, ctypes.c_void_p]
     lib.mla_paged_cache_load.restype = ctypes.c_int
     lib.mla_prefill_paged.argtypes = [T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
@@ -76,6 +85,8 @@ def load_library(path=None):
     lib.mla_selftest_wait_timeout.restype = ctypes.c_int
     lib.mla_prefill_last_launches.argtypes = []
     lib.mla_prefill_last_launches.restype = ctypes.c_int
+    lib.mla_prefill_set_kernel.argtypes = [ctypes.c_int]
+    lib.mla_prefill_set_kernel.restype = ctypes.c_int
     lib.mla_prefill_set_split_tiles.argtypes = [ctypes.c_int]
     lib.mla_prefill_set_split_tiles.restype = ctypes.c_int
     lib.mla_prefill_version.argtypes = []
@@ -155,6 +166,45 @@ def mla_prefill_noalloc(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type,
     return out
 
 
+def mla_prefill_get_workspace_size(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num,
+                                   qk_scale, out):
+    """Call the C ABI ``mla_prefill_get_workspace_size``: bytes of device workspace ``mla_prefill_ws``
+    needs for these arguments (only shapes, strides, dtypes and scalars are read)."""
+    lib = load_library()
+    descs = [as_mla_tensor(t) for t in (q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, out)]
+    n = ctypes.c_uint64(0)
+    rc = lib.mla_prefill_get_workspace_size(*(ctypes.byref(d) for d in descs[:7]), int(mask_type), int(head_num),
+                                            int(kv_head_num), float(qk_scale), ctypes.byref(descs[7]),
+                                            ctypes.byref(n))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_get_workspace_size")
+    return n.value
+
+
+def mla_prefill_ws(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
+                   workspace, stream=None):
+    """Call the C ABI ``mla_prefill_ws``: ``mla_prefill`` with a caller-owned workspace (a uint8 CUDA
+    tensor, 256-byte aligned, at least ``mla_prefill_get_workspace_size`` bytes)."""
+    lib = load_library()
+    descs = [as_mla_tensor(t) for t in (q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, out)]
+    rc = lib.mla_prefill_ws(*(ctypes.byref(d) for d in descs[:7]), int(mask_type), int(head_num), int(kv_head_num),
+                            float(qk_scale), ctypes.byref(descs[7]), workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_ws")
+    return out
+
+
+def mla_prefill_ws_status(workspace, stream=None):
+    """Synchronise the stream and return the status of the last ``mla_prefill_ws`` call on ``workspace``."""
+    lib = load_library()
+    st = ctypes.c_int(0)
+    rc = lib.mla_prefill_ws_status(workspace.data_ptr(), _stream_handle(stream, workspace.device), ctypes.byref(st))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_ws_status")
+    return st.value
+
+
 def prefill(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, head_num, kv_head_num, qk_scale,
             mask_type=MLA_MASK_CAUSAL, out=None, stream=None):
     """Allocate ``out`` [T_q, H, 128] (if not given) and run ``mla_prefill``."""
@@ -215,6 +265,13 @@ def set_split_tiles(tiles):
     rc = load_library().mla_prefill_set_split_tiles(int(tiles))
     if rc != 0:
         raise MlaError(rc, "mla_prefill_set_split_tiles")
+
+
+def set_kernel(kernel):
+    """Attention kernel for later prefill calls on this thread: -1 automatic, 1 single-CTA, 2 CTA pair."""
+    rc = load_library().mla_prefill_set_kernel(int(kernel))
+    if rc != 0:
+        raise MlaError(rc, "mla_prefill_set_kernel")
 
 
 def set_profile_events(start=None, stop=None):

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/mla_prefill.h"
+#include "mla_prefill_pair_sm100.cuh"
 #include "mla_prefill_sm100.cuh"
 #include "paged_cache_load.cuh"
 #include "prolog_norm_rope.cuh"
@@ -27,12 +28,14 @@ struct DeviceState {
     int *status = nullptr;  // sticky device status word (own 256-byte allocation)
     void *ws = nullptr;     // plan workspace
     size_t ws_bytes = 0;
-    bool attr_set[16] = {};  // dynamic shared memory opt-in done, per kernel instantiation
+    bool attr_set[32] = {};  // dynamic shared memory opt-in done, per kernel instantiation
+    int pair_clusters = 0;   // co-resident clusters of two CTAs of the pair kernel (0: not yet queried)
 };
 
 std::mutex g_mu;
 thread_local cudaEvent_t t_prof_start = nullptr, t_prof_stop = nullptr;
 thread_local int t_split_tiles = -1;  // split-KV chunk in key tiles: -1 automatic, 0 off
+thread_local int t_kernel = -1;       // attention kernel: -1 automatic, 1 single-CTA, 2 CTA pair
 thread_local int t_last_launches = 0;  // kernels the last prefill call of this thread enqueued
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -170,6 +173,7 @@ int encode_cache_map(CUtensorMap *m, const void *data, int64_t blocks, int64_t s
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
+    size_t status;  // offset of the per-call status word (caller-owned workspaces only)
     size_t seq_info, unit_off, hist, units, num_units, total;
     size_t split_off, entry_tab, part_lse, part_o;  // split-KV sections (empty without split)
     int hist_len;
@@ -186,14 +190,17 @@ int64_t max_entries_for(int64_t max_units, int64_t key_extent, int split) {
 }
 
 // t_k: key tokens of the K/V tensors; key_extent: the most keys one sequence can have;
-// split: key tiles per split-KV chunk (0: none); heads: query heads.
+// split: key tiles per split-KV chunk (0: none); heads: query heads; status_header: the first
+// kWsHeaderBytes hold the call's status word (a caller-owned workspace).
+constexpr size_t kWsHeaderBytes = 256;
 WsLayout ws_layout(int64_t batch, int64_t t_q, int64_t t_k, int64_t key_extent = 0, int split = 0,
-                   int64_t heads = 0) {
+                   int64_t heads = 0, bool status_header = false) {
     WsLayout l;
     const int64_t max_units = max_units_for(batch, t_q);
     l.hist_len = static_cast<int>((t_k + mla::kBN - 1) / mla::kBN + 2);
     l.split_tiles = split;
-    size_t off = 0;
+    l.status = 0;
+    size_t off = status_header ? kWsHeaderBytes : 0;
     l.num_units = off;
     off = align_up(off + 16, 256);
     l.seq_info = off;
@@ -235,14 +242,18 @@ int device_state(int dev, cudaStream_t stream, size_t ws_need, DeviceState **out
         d.ready = true;
     }
     if (d.ws_bytes < ws_need) {
+        // Stream-ordered: the old workspace is released behind the work already queued on this
+        // stream and the new one is ready for the work queued next; the host never waits.
         if (d.ws) {
-            if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;
-            cudaFree(d.ws);
+            if (cudaFreeAsync(d.ws, stream) != cudaSuccess) return MLA_ERR_CUDA;
             d.ws = nullptr;
             d.ws_bytes = 0;
         }
-        const size_t bytes = align_up(ws_need * 2 > (1u << 20) ? ws_need * 2 : (1u << 20), 4096);
-        if (cudaMalloc(&d.ws, bytes) != cudaSuccess) return MLA_ERR_CUDA;
+        const size_t bytes = align_up(ws_need, size_t(1) << 20);
+        if (cudaMallocAsync(&d.ws, bytes, stream) != cudaSuccess) {
+            d.ws = nullptr;
+            return MLA_ERR_CUDA;
+        }
         d.ws_bytes = bytes;
     }
     *out = &d;
@@ -271,6 +282,46 @@ int launch_attention(DeviceState *ds, int slot, int grid, cudaStream_t stream, c
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = t_prof_start ? 0 : 1;  // with the timing hook on, its events bracket this kernel alone
+    if (cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], p) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    if (t_prof_stop && cudaEventRecord(t_prof_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_OK;
+}
+
+// The CTA-pair kernel: clusters of two CTAs, one per SM, persistent over the work list.
+template <typename T, bool kCausal, bool kPos>
+int launch_pair(DeviceState *ds, int slot, int64_t max_items, cudaStream_t stream, const CUtensorMap (&maps)[5],
+                const mla::Params &p) {
+    auto kern = mla::pair::mla_prefill_pair_kernel<T, kCausal, kPos>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(mla::kThreads);
+    cfg.dynamicSmemBytes = mla::pair::kSmemAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    if (!ds->attr_set[slot]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::pair::kSmemAlloc) !=
+            cudaSuccess)
+            return MLA_ERR_CUDA;
+        ds->attr_set[slot] = true;
+    }
+    if (ds->pair_clusters <= 0) {
+        int n = 0;
+        cfg.gridDim = dim3(2);
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return MLA_ERR_CUDA;
+        ds->pair_clusters = n;
+    }
+    const int64_t clusters = max_items < ds->pair_clusters ? max_items : ds->pair_clusters;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+    cfg.numAttrs = t_prof_start ? 1 : 2;  // with the timing hook on, its events bracket this kernel alone
+    if (t_prof_start && cudaEventRecord(t_prof_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
     if (cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], p) != cudaSuccess)
         return MLA_ERR_CUDA;
     if (t_prof_stop && cudaEventRecord(t_prof_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
@@ -367,9 +418,15 @@ int validate(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
 // holds the workspace described by `lay`; `launch_flags` records the
 // per-instantiation shared-memory opt-in for the current GPU.
 int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, int sm_count, DeviceState *launch_flags,
-            cudaStream_t stream) {
+            cudaStream_t stream, bool reset_status = false) {
     int rc;
     if ((rc = ensure_encode()) != MLA_OK) return rc;
+    const bool general = pr.paged || pr.kv_pad > 0 || lay.split_tiles > 0;  // padded / paged K/V or split-KV
+    // The CTA-pair kernel serves packed, unsplit K/V; automatically once its 512-row units give at
+    // least as many work items as there are SM pairs.
+    const int64_t pair_items = ((pr.q.tokens + mla::pair::kUnitRows - 1) / mla::pair::kUnitRows + pr.batch) *
+                               pr.head_num;
+    const bool use_pair = !general && t_kernel == 2 && pair_items > 0;
     CUtensorMap maps[5];
     if ((rc = encode_map(&maps[0], pr.q, pr.bf16, ws, 128)) != MLA_OK) return rc;
     if ((rc = encode_map(&maps[1], pr.qr, pr.bf16, ws, 128)) != MLA_OK) return rc;
@@ -385,8 +442,10 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
                                    pr.vc_block, pr.vc_slot, pr.vc_head, pr.bf16, rows_v)) != MLA_OK)
             return rc;
     } else {
-        if ((rc = encode_map(&maps[2], pr.k, pr.bf16, ws, 128)) != MLA_OK) return rc;
-        if ((rc = encode_map(&maps[3], pr.kr, pr.bf16, ws, 128)) != MLA_OK) return rc;
+        // pair kernel: each CTA loads 64 keys of K per key tile
+        const int kbox = use_pair ? 64 : 128;
+        if ((rc = encode_map(&maps[2], pr.k, pr.bf16, ws, kbox)) != MLA_OK) return rc;
+        if ((rc = encode_map(&maps[3], pr.kr, pr.bf16, ws, kbox)) != MLA_OK) return rc;
         if ((rc = encode_map(&maps[4], pr.v, pr.bf16, ws, 64)) != MLA_OK) return rc;
     }
 
@@ -403,7 +462,8 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     mla::mla_plan_kernel<<<1, mla::kPlanThreads, 0, stream>>>(
         pr.q_seqlen, pr.kv_seqlen, static_cast<int>(pr.batch), pr.q.tokens, pr.k.tokens, pr.kv_pad,
         pr.paged ? 1 : 0, pr.causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
-        lay.split_tiles, split_off, entry_tab, num_entries, status);
+        lay.split_tiles, split_off, entry_tab, num_entries, status, reset_status ? 1 : 0,
+        use_pair ? mla::pair::kUnitRows : mla::kUnitRows);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
     mla::Params p;
@@ -417,6 +477,8 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     p.out_sh = pr.o.st_head;
     p.head_num = pr.head_num;
     p.group = pr.head_num / pr.kv_head_num;
+    // unit-major (longest-first) item order when all of K, K_rope and V fit in 48 MB of the L2
+    p.lpt = !pr.paged && pr.k.tokens * pr.kv_head_num * (2 * mla::kDn + mla::kDr) * 2 <= (int64_t(48) << 20);
     p.scale_log2 = pr.qk_scale * 1.4426950408889634f;
     p.tables = pr.tables;
     p.table_stride = pr.table_stride;
@@ -431,14 +493,27 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     p.num_entries = num_entries;
     p.part_lse = reinterpret_cast<float *>(ws + lay.part_lse);
     p.part_o = reinterpret_cast<float *>(ws + lay.part_o);
-    const bool general = pr.paged || pr.kv_pad > 0 || lay.split_tiles > 0;  // padded / paged K/V or split-KV
+    const bool pos = pr.qk_scale > 0.f;
+    DeviceState *ls = launch_flags;
+    if (use_pair) {
+        const int slot = 16 + (pr.bf16 ? 0 : 4) + (pr.causal ? 0 : 2) + (pos ? 0 : 1);
+#define MLA_PAIR(T, C, P) launch_pair<T, C, P>(ls, slot, pair_items, stream, maps, p)
+        if (pr.bf16) {
+            if (pr.causal) rc = pos ? MLA_PAIR(__nv_bfloat16, true, true) : MLA_PAIR(__nv_bfloat16, true, false);
+            else rc = pos ? MLA_PAIR(__nv_bfloat16, false, true) : MLA_PAIR(__nv_bfloat16, false, false);
+        } else {
+            if (pr.causal) rc = pos ? MLA_PAIR(__half, true, true) : MLA_PAIR(__half, true, false);
+            else rc = pos ? MLA_PAIR(__half, false, true) : MLA_PAIR(__half, false, false);
+        }
+#undef MLA_PAIR
+        t_last_launches = 2;  // plan + attention
+        return rc;
+    }
 
     const int64_t max_units = max_units_for(pr.batch, pr.q.tokens);
     const int64_t max_items =
         max_entries_for(max_units, pr.kv_pad > 0 ? pr.kv_pad : pr.k.tokens, lay.split_tiles) * pr.head_num;
     const int grid = static_cast<int>(max_items < sm_count ? max_items : sm_count);
-    const bool pos = pr.qk_scale > 0.f;
-    DeviceState *ls = launch_flags;
     const int slot = (pr.bf16 ? 0 : 4) + (pr.causal ? 0 : 2) + (pos ? 0 : 1) + (general ? 8 : 0);
 #define MLA_LAUNCH(T, C, P, G) launch_attention<T, C, P, G>(ls, slot, grid, stream, maps, p)
 #define MLA_PICK(T, C, P) (general ? MLA_LAUNCH(T, C, P, true) : MLA_LAUNCH(T, C, P, false))
@@ -476,7 +551,7 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
 // (unit, head) items cannot fill the GPU twice over and there are at least 16 key tiles of work per
 // SM, in chunks that make about three items per SM.
 // The fp32 partial rows are kept under 2 GiB.
-int choose_split(const Problem &pr, int sm_count) {
+int choose_split(const Problem &pr, int sm_count) {  // sm_count is read in automatic mode only
     const int64_t units = max_units_for(pr.batch, pr.q.tokens);
     const int64_t ext = pr.kv_pad > 0 ? pr.kv_pad : pr.k.tokens;
     const int64_t tiles = (ext + mla::kBN - 1) / mla::kBN;
@@ -538,6 +613,56 @@ int noalloc_setup(int dev, NoAllocDevice **out) {
     return MLA_OK;
 }
 
+// Per-GPU facts for the caller-workspace entry points, gathered without allocating anything:
+// the architecture check, the SM count, and the kernels' shared-memory opt-in flags.
+struct LaunchInfo {
+    bool ready = false;
+    int sm_count = 0;
+    DeviceState launch;  // only its dynamic-shared-memory opt-in flags are used
+};
+LaunchInfo g_launch_info[kMaxDevices];
+
+int launch_info(int dev, LaunchInfo **out) {
+    if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+    LaunchInfo &d = g_launch_info[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MLA_ERR_CUDA;
+        if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;
+        d.ready = true;
+    }
+    *out = &d;
+    return MLA_OK;
+}
+
+// Validation and workspace layout shared by mla_prefill_get_workspace_size and mla_prefill_ws.
+// The split-KV choice depends on the thread's split setting and, in automatic mode, on the SM
+// count of the current GPU, so both calls must be made with the same settings on the same GPU.
+int ws_problem(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+               const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+               int head_num, int kv_head_num, float qk_scale, const mla_tensor *out, Problem *pr, WsLayout *lay,
+               LaunchInfo **li) {
+    int rc = validate(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
+                      pr);
+    if (rc != MLA_OK) return rc;
+    *li = nullptr;
+    int sm_count = 0;
+    if (t_split_tiles < 0 && pr->batch > 0 && pr->q.tokens > 0) {  // automatic split: needs the SM count
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+        std::lock_guard<std::mutex> lock(g_mu);
+        if ((rc = launch_info(dev, li)) != MLA_OK) return rc;
+        sm_count = (*li)->sm_count;
+    }
+    const int split = (pr->batch > 0 && pr->q.tokens > 0) ? choose_split(*pr, sm_count) : 0;
+    *lay = ws_layout(pr->batch, pr->q.tokens, pr->k.tokens, pr->kv_pad > 0 ? pr->kv_pad : pr->k.tokens, split,
+                     pr->head_num, true);
+    return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -590,6 +715,58 @@ int mla_prefill_device_status(mla_stream_t stream_, int *status) {
     return MLA_OK;
 }
 
+int mla_prefill_get_workspace_size(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k,
+                                   const mla_tensor *k_rope, const mla_tensor *v, const mla_tensor *q_seqlen,
+                                   const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num,
+                                   float qk_scale, const mla_tensor *out, uint64_t *workspace_bytes) {
+    if (!workspace_bytes) return MLA_ERR_NULL;
+    Problem pr;
+    WsLayout lay;
+    LaunchInfo *li;
+    const int rc = ws_problem(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num,
+                              qk_scale, out, &pr, &lay, &li);
+    if (rc != MLA_OK) return rc;
+    *workspace_bytes = lay.total;
+    return MLA_OK;
+}
+
+int mla_prefill_ws(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor *k, const mla_tensor *k_rope,
+                   const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
+                   int head_num, int kv_head_num, float qk_scale, mla_tensor *out, void *workspace,
+                   uint64_t workspace_bytes, mla_stream_t stream_) {
+    t_last_launches = 0;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    Problem pr;
+    WsLayout lay;
+    LaunchInfo *li;
+    int rc = ws_problem(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale,
+                        out, &pr, &lay, &li);
+    if (rc != MLA_OK) return rc;
+    if (!workspace) return MLA_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kWsHeaderBytes - 1)) || workspace_bytes < lay.total)
+        return MLA_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + lay.status);
+    if (pr.batch == 0 || pr.q.tokens == 0)  // nothing to compute: the call's status is OK
+        return cudaMemsetAsync(status, 0, sizeof(int), stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!li && (rc = launch_info(dev, &li)) != MLA_OK) return rc;
+    return enqueue(pr, lay, ws, status, li->sm_count, &li->launch, stream, true);
+}
+
+int mla_prefill_ws_status(const void *workspace, mla_stream_t stream_, int *status) {
+    if (!workspace || !status) return MLA_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(workspace) & (kWsHeaderBytes - 1)) return MLA_ERR_WORKSPACE;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MLA_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+    *status = h;
+    return MLA_OK;
+}
+
 const char *mla_status_string(int status) {
     switch (status) {
         case MLA_OK: return "MLA_OK";
@@ -603,6 +780,7 @@ const char *mla_status_string(int status) {
         case MLA_ERR_SEQLEN: return "MLA_ERR_SEQLEN: seqlens inconsistent with tensor extents (clamped)";
         case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT: a device pipeline wait gave up";
         case MLA_ERR_INDEX: return "MLA_ERR_INDEX: a paged-cache block index was out of range (row zeroed)";
+        case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace smaller than required or not 256-byte aligned";
         default: return "unknown mla_status";
     }
 }
@@ -621,6 +799,12 @@ int mla_selftest_wait_timeout(int wait_ms, mla_stream_t stream_) {
 }
 
 int mla_prefill_last_launches(void) { return t_last_launches; }
+
+int mla_prefill_set_kernel(int kernel) {
+    if (kernel != -1 && kernel != 1 && kernel != 2) return MLA_ERR_UNSUPPORTED;
+    t_kernel = kernel;
+    return MLA_OK;
+}
 
 int mla_prefill_set_split_tiles(int tiles) {
     if (tiles < -1) return MLA_ERR_UNSUPPORTED;

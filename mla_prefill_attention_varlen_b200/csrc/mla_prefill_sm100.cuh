@@ -90,6 +90,7 @@ struct Params {
     long long out_st, out_sh;  // token / head strides of out, elements
     int head_num;
     int group;         // head_num / kv_head_num
+    int lpt;           // 1: items unit-major (longest first across all heads); 0: kv-head-major
     float scale_log2;  // qk_scale * log2(e)
     // paged K/V only: logical block i of sequence b is physical block tables[b * table_stride + i]
     const int *tables;
@@ -134,11 +135,15 @@ __host__ __device__ __forceinline__ int kv_tiles_for(int q0, int rows, int lq, i
 
 __host__ __device__ __forceinline__ int tile_rows(int q0, int lq) { return max(0, min(kBM, lq - q0)); }
 
-// Key tiles a 256-row unit walks (the larger of its two tiles' counts).
-__host__ __device__ __forceinline__ int unit_cost(int u0, int lq, int lk, bool causal) {
-    const int a = kv_tiles_for(u0, tile_rows(u0, lq), lq, lk, causal);
-    const int b = kv_tiles_for(u0 + kBM, tile_rows(u0 + kBM, lq), lq, lk, causal);
-    return a > b ? a : b;
+// Key tiles a unit of unit_rows query rows (256: two tiles, 512: four) walks: the largest count
+// among its 128-row tiles.
+__host__ __device__ __forceinline__ int unit_cost(int u0, int lq, int lk, bool causal, int unit_rows = kUnitRows) {
+    int c = 0;
+    for (int r = 0; r < unit_rows; r += kBM) {
+        const int n = kv_tiles_for(u0 + r, tile_rows(u0 + r, lq), lq, lk, causal);
+        c = n > c ? n : c;
+    }
+    return c;
 }
 
 struct WorkItem {
@@ -157,15 +162,28 @@ struct WorkItem {
 // Work items are ordered kv-head-major: for each kv head, its units in the
 // sorted (longest-first) order, and for each unit the query heads of the group.
 // Concurrently running CTAs then read the same kv head's K/V (L2 reuse), and the
-// last items of the grid are the cheapest units.
+// last items of each kv head are its cheapest units.  When all of K/V fits in L2
+// with room to spare (p.lpt), reuse needs no such order: the items go unit-major
+// instead (every head of the longest unit first), the longest-first order over the
+// whole grid, which shortens the tail when there are only a few items per SM.
+__device__ __forceinline__ void item_unit_head(const Params &p, int it, int num_entries, int &e, int &h) {
+    if (p.lpt) {
+        e = it / p.head_num;
+        h = it - e * p.head_num;
+    } else {
+        const int per_kh = num_entries * p.group;
+        const int kh = it / per_kh;
+        const int rem = it - kh * per_kh;
+        e = rem / p.group;
+        h = kh * p.group + (rem - e * p.group);
+    }
+}
+
 template <bool kSplit>  // kSplit: the kernel may run split-KV work lists
 __device__ __forceinline__ WorkItem decode_item(const Params &p, int it, int num_entries, bool causal) {
-    const int per_kh = num_entries * p.group;
     WorkItem x;
-    x.kh = it / per_kh;
-    const int rem = it - x.kh * per_kh;
-    x.e = rem / p.group;
-    x.h = x.kh * p.group + (rem - x.e * p.group);
+    item_unit_head(p, it, num_entries, x.e, x.h);
+    x.kh = x.h / p.group;
     int u = x.e, chunk = 0;
     if (kSplit && p.split_tiles > 0) {
         const int2 uc = p.entry_tab[x.e];
@@ -260,8 +278,9 @@ struct DType<__half> {
 // ---------------------------------------------------------------------------
 // Plan kernel: one block of 1024 threads.  Clamps the seqlens to the tensor
 // extents (recording kStatusSeqlen on any inconsistency), writes per-sequence
-// offsets, and writes the (sequence, 256-row unit) list sorted by descending
-// number of key tiles (a counting sort; ties in arbitrary order).
+// offsets, and writes the (sequence, unit of unit_rows rows) list sorted by descending
+// number of key tiles (a counting sort; ties in arbitrary order).  With
+// reset_status, the status word is zeroed first (a word that reports one call).
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 
@@ -307,12 +326,18 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
                                                                 int4 *seq_info, int *unit_off, int *hist,
                                                                 int hist_len, int2 *units, int *num_units,
                                                                 int *work_counter, int split_tiles, int *split_off,
-                                                                int2 *entry_tab, int *num_entries, int *status) {
+                                                                int2 *entry_tab, int *num_entries, int *status,
+                                                                int reset_status, int unit_rows) {
     __shared__ long long warp_sums[32];
     __shared__ int bad;
     // the attention grid may be scheduled now: it sets itself up and then waits for this grid
     ptx::griddep_launch_dependents();
-    if (threadIdx.x == 0) bad = 0;
+    if (threadIdx.x == 0) {
+        bad = 0;
+        // a per-call status word (caller-owned workspace) starts each call at 0; the attention
+        // kernel writes it only after this grid has completed
+        if (reset_status) *status = 0;
+    }
     __syncthreads();
 
     // 1. clamped prefix sums and unit counts, in chunks of blockDim.x sequences
@@ -338,7 +363,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
         const long long ck = kb < t_k ? kb : t_k, ek = kb + lk < kcap ? (kb + lk < t_k ? kb + lk : t_k) : (kcap < t_k ? kcap : t_k);
         if (b < batch && (eq - cq != lq || ek - ck != lk)) bad = 1;
         const int lqc = static_cast<int>(eq - cq), lkc = static_cast<int>(ek - ck);
-        const long long nu = (b < batch) ? (lqc + kUnitRows - 1) / kUnitRows : 0;
+        const long long nu = (b < batch) ? (lqc + unit_rows - 1) / unit_rows : 0;
         long long tot_u;
         const long long pu = carry_u + block_exclusive_scan(nu, tot_u, warp_sums);
         if (b < batch) {
@@ -358,7 +383,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
         const int b = seq_of_unit(unit_off, batch, t);
         const int4 s = seq_info[b];
-        const int cost = unit_cost((t - unit_off[b]) * kUnitRows, s.z, s.w, causal != 0);
+        const int cost = unit_cost((t - unit_off[b]) * unit_rows, s.z, s.w, causal != 0, unit_rows);
         atomicAdd(&hist[min(cost, hist_len - 1)], 1);
     }
     __syncthreads();
@@ -381,7 +406,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
         const int b = seq_of_unit(unit_off, batch, t);
         const int4 s = seq_info[b];
         const int m = t - unit_off[b];
-        const int cost = unit_cost(m * kUnitRows, s.z, s.w, causal != 0);
+        const int cost = unit_cost(m * unit_rows, s.z, s.w, causal != 0, unit_rows);
         const int pos = atomicAdd(&hist[min(cost, hist_len - 1)], 1);
         units[pos] = make_int2(b, m);
     }
@@ -397,7 +422,7 @@ __global__ void __launch_bounds__(kPlanThreads) mla_plan_kernel(const int *__res
             if (u < total) {
                 const int2 bm = units[u];
                 const int4 s = seq_info[bm.x];
-                const int cost = unit_cost(bm.y * kUnitRows, s.z, s.w, causal != 0);
+                const int cost = unit_cost(bm.y * unit_rows, s.z, s.w, causal != 0, unit_rows);
                 ns = cost > split_tiles ? (cost + split_tiles - 1) / split_tiles : 1;
             }
             long long tot;

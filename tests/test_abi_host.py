@@ -196,6 +196,87 @@ def test_empty_batch_is_a_no_op(lib):
 
 
 # ---------------------------------------------------------------------------
+# caller-owned workspace: the size query and the host-side checks of mla_prefill_ws
+# ---------------------------------------------------------------------------
+
+def _align(x, a=256):
+    return (x + a - 1) // a * a
+
+
+def expected_workspace_bytes(batch, t_q, t_k, split=0, heads=0, key_extent=None):
+    """The workspace mla_prefill_ws needs, section by section (each rounded up to 256 bytes): the
+    status header, a 16-byte counter block, per-sequence offsets {cq, ck, Lq, Lk} (16 bytes each),
+    per-sequence unit offsets (batch + 1 ints), the key-tile histogram (ceil(T_k/128) + 2 ints) and
+    the unit list (ceil(T_q/256) + batch int pairs); with split-KV chunks of `split` key tiles also
+    the per-unit entry offsets, the entry table and the fp32 partial rows (O / l and the
+    log-sum-exp) of every entry, head and row of a 256-row unit."""
+    units = -(-t_q // 256) + batch
+    n = 256 + _align(16) + _align(16 * batch) + _align(4 * (batch + 1)) + _align(4 * (-(-t_k // 128) + 2)) \
+        + _align(8 * units)
+    if split:
+        tiles = -(-(key_extent or t_k) // 128)
+        # the chunk doubles while the fp32 partial rows (129 floats per row) would pass 2 GiB
+        while split < tiles and units * max(1, -(-tiles // split)) * heads * 256 * 129 * 4 > 2 << 30:
+            split *= 2
+        if split >= tiles:
+            return n
+        entries = units * max(1, -(-tiles // split))
+        n += _align(4 * (units + 1)) + _align(8 * entries) + _align(4 * entries * heads * 256) \
+            + _align(4 * entries * heads * 256 * 128)
+    return n
+
+
+def ws_size(lib, t, H, G, mask=1, scale=0.5):
+    d = {k: mla.as_mla_tensor(v) for k, v in t.items()}
+    n = ctypes.c_uint64(0)
+    rc = lib.mla_prefill_get_workspace_size(*(ctypes.byref(d[k]) for k in ("q", "q_rope", "k", "k_rope", "v",
+                                                                            "q_seqlen", "kv_seqlen")),
+                                            mask, H, G, scale, ctypes.byref(d["out"]), ctypes.byref(n))
+    return rc, n.value
+
+
+@pytest.mark.parametrize("T,Tk,batch,H,G", [(256, 256, 2, 4, 2), (1000, 5000, 7, 8, 8), (1, 1, 1, 1, 1),
+                                            (40000, 70000, 300, 2, 1)])
+def test_workspace_size_formula(lib, T, Tk, batch, H, G):
+    # explicit split settings: the size needs no GPU (only the automatic mode reads the SM count)
+    t, _, _ = make_args(T=T, Tk=Tk, H=H, G=G, batch=batch)
+    try:
+        mla.set_split_tiles(0)
+        rc, n = ws_size(lib, t, H, G)
+        assert rc == 0 and n == expected_workspace_bytes(batch, T, Tk)
+        mla.set_split_tiles(3)
+        rc, n = ws_size(lib, t, H, G)
+        tiles = -(-Tk // 128)
+        expect = expected_workspace_bytes(batch, T, Tk, split=3 if 3 < tiles else 0, heads=H)
+        assert rc == 0 and n == expect
+    finally:
+        mla.set_split_tiles(-1)
+
+
+def test_workspace_size_and_call_reject_bad_arguments(lib):
+    t, H, G = make_args()
+    d = {k: mla.as_mla_tensor(v) for k, v in t.items()}
+    args = [ctypes.byref(d[k]) for k in ("q", "q_rope", "k", "k_rope", "v", "q_seqlen", "kv_seqlen")]
+    assert lib.mla_prefill_get_workspace_size(*args, 1, H, G, 0.5, ctypes.byref(d["out"]), None) == 1
+    assert ws_size(lib, t, 8, G)[0] == 3  # argument errors as in mla_prefill
+    try:
+        mla.set_split_tiles(0)
+        rc, need = ws_size(lib, t, H, G)
+        assert rc == 0
+        buf = torch.zeros(need + 512, dtype=torch.uint8)
+        base = (buf.data_ptr() + 255) // 256 * 256  # never dereferenced: rejected on the host
+        assert lib.mla_prefill_ws(*args, 1, H, G, 0.5, ctypes.byref(d["out"]), None, need, None) == 1
+        assert lib.mla_prefill_ws(*args, 1, H, G, 0.5, ctypes.byref(d["out"]), base, need - 1, None) == 11
+        assert lib.mla_prefill_ws(*args, 1, H, G, 0.5, ctypes.byref(d["out"]), base + 16, need, None) == 11
+        assert lib.mla_prefill_ws(*args, 1, 8, G, 0.5, ctypes.byref(d["out"]), base, need, None) == 3
+    finally:
+        mla.set_split_tiles(-1)
+    st = ctypes.c_int(0)
+    assert lib.mla_prefill_ws_status(None, None, ctypes.byref(st)) == 1
+    assert lib.mla_prefill_ws_status(buf.data_ptr() | 8, None, ctypes.byref(st)) == 11
+
+
+# ---------------------------------------------------------------------------
 # mla_paged_cache_load host-side validation (descriptors are never dereferenced)
 # ---------------------------------------------------------------------------
 

@@ -29,6 +29,18 @@ def gpu():
     torch.cuda.synchronize()
 
 
+# Every test of this module runs on both attention kernels: the single-CTA kernel (256-row units)
+# and the CTA-pair kernel (512-row units on clusters of two SMs).  Padded K/V always runs the
+# single-CTA kernel.
+@pytest.fixture(autouse=True, params=[1, 2], ids=["single", "pair"])
+def kernel(request):
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    mla.set_kernel(request.param)
+    yield request.param
+    mla.set_kernel(-1)
+
+
 def problem(lens_q, lens_k, H, G, dtype=torch.bfloat16, std=1.0, seed=0, extra_tokens=0):
     wl = W.Workload("case", list(lens_q), list(lens_k), H, G, dtype=dtype, std=std, seed=seed)
     x = W.make_inputs(wl, device=DEV)
@@ -139,7 +151,11 @@ def test_many_short_units_per_cta():
     lens = many_short_lengths(77, 600, [2000, 1999, 2048])
     _, x = problem(lens, lens, 4, 2, seed=4242, extra_tokens=3)
     out = run(x, 4, 2, 0.07)
-    check_against_oracle(x, out, 4, 2, 0.07)
+    # Half-ulp form of the bound: 49.5M checked elements, most of them in rows with a handful of
+    # keys where |out| reaches 2-4 and the bf16 storage rounding alone is up to 0.0078 (0.0156
+    # above 4); the computation's own error on top of that rounding is what the 1e-2 bounds here.
+    _, st = check_against_oracle(x, out, 4, 2, 0.07, bound="half_ulp")
+    print("many_short", st)
     assert torch.all(out[sum(lens):] == 7.0)
     assert status() == 0
 

@@ -38,11 +38,11 @@ def run(x, H, G, scale, mask, split, out=None):
     return out
 
 
-def check(x, out, H, G, scale, mask, rows=None, head_chunk=None):
+def check(x, out, H, G, scale, mask, rows=None, head_chunk=None, bound="literal"):
     ref = oracle_rows(cpu_copy(x), H, G, scale, rows=rows,
                       mask_type=1 if mask == mla.MLA_MASK_CAUSAL else 0, head_chunk=head_chunk)
     computed = ~np.isnan(ref[:, 0, 0])
-    ok, st = compare(out.cpu(), ref, x["q"].dtype, mask=computed)
+    ok, st = compare(out.cpu(), ref, x["q"].dtype, mask=computed, bound=bound)
     assert ok, st
 
 
@@ -132,6 +132,8 @@ def test_one_tile_chunks_over_many_short_sequences():
     whole = run(x, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL, 0)
     parts = run(x, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL, 1)
     assert mla.mla_prefill_device_status() == 0
-    check(x, parts, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL)
+    # Half-ulp form of the bound: 24M checked elements, most in rows with a handful of keys where
+    # |out| reaches 2-4 and the bf16 storage rounding alone is up to 0.0078 (0.0156 above 4).
+    check(x, parts, 4, 2, wl.qk_scale, mla.MLA_MASK_CAUSAL, bound="half_ulp")
     d = (parts.float() - whole.float()).abs()
     assert d.max().item() <= 4 * 2.0 ** -8 * max(1.0, whole.float().abs().max().item())

@@ -214,3 +214,226 @@ def test_planted_protocol_mistakes_are_caught(bug):
     with pytest.raises(ProtocolError):
         for trial in range(400):
             simulate(random_units(rng), seed=trial, bug=bug)
+
+
+# ---------------------------------------------------------------------------
+# The CTA-pair kernel (mla_prefill_pair_sm100.cuh)
+# ---------------------------------------------------------------------------
+# Two CTAs (leader 0, follower 1) each stream their half of every key tile through their own
+# ring of sixteen 8 KB chunks: key tile g occupies chunks 5g .. 5g + 4 (mod 16), K_g in the
+# first three, V_g in the last two.  Each CTA also holds its 128 rows of Q for groups 0 and 1.
+#
+#   producer (each CTA)  per unit: Q_t for each group with key tiles: waits its own
+#                        q_empty(t), arms its own q_full(t), loads; per key tile:
+#                        K_g waits its own k_empty(g - 3), V_g its own v_empty(g - 3)
+#   relay (follower)     in the producer's order, waits for each of the follower's full
+#                        barriers and arrives on the leader's matching one
+#   MMA (leader)         as in the single-CTA kernel, waiting on the leader's full barriers
+#                        (two arrivals: the leader's own load, the relay); every release
+#                        (q_empty, k_empty, v_empty) and S-ready arrives in both CTAs; each
+#                        pair MMA reads both CTAs' halves
+#   softmax (each CTA)   group t: waits its own S_t(j), arrives on the leader's P_t(j)
+#                        (two arrivals: one per CTA)
+PAIR_RING = 16
+
+
+def simulate_pair(units, seed, bug=None):
+    """units: [(n0, n1)] key tiles of group 0 / 1 per 512-row unit (max > 0)."""
+    rnd = random.Random(seed)
+    bars = {}
+
+    def mk(kind, cta, i, count=1):
+        bars[kind, cta, i] = Barrier("%s[%d]@%d" % (kind, i, cta), count)
+
+    for cta in range(2):
+        full_count = 2 if cta == 0 else 1
+        for i in range(TILE_SETS):
+            mk("k_full", cta, i, full_count)
+            mk("v_full", cta, i, full_count)
+            mk("k_empty", cta, i)
+            mk("v_empty", cta, i)
+        for t in range(2):
+            mk("q_full", cta, t, full_count)
+            mk("q_empty", cta, t)
+            mk("s_full", cta, t)
+    for t in range(2):
+        mk("p_full", 0, t, 2)
+    owner = {}     # (cta, ring slot | ("Q", t)) -> operand last loaded there
+    readers = {}   # operand -> MMAs issued and not yet completed
+    landed = set()
+    tma = []       # (cta, barrier, operand)
+    mma_queue = []
+
+    def b(kind, cta, g):
+        return bars[kind, cta, g % TILE_SETS]
+
+    def fill(cta, key, operand):
+        prev = owner.get((cta, key))
+        if prev is not None and readers.get(prev, 0):
+            raise ProtocolError("%s refilled with %s while an MMA reads %s" % ((cta, key), operand, prev))
+        owner[(cta, key)] = operand
+
+    def producer(cta):
+        g = 0
+        ql = [0, 0]
+        lag = 4 if bug == "pair_lag_4" else 3
+        for n in units:
+            for t in range(2):
+                if n[t] == 0:
+                    continue
+                if ql[t] >= 1 and bug != "pair_no_q_empty_wait":
+                    while not ready(bars["q_empty", cta, t], ql[t] - 1):
+                        yield
+                fill(cta, ("Q", t), (cta, "Q", t, ql[t]))
+                tma.append((cta, bars["q_full", cta, t], (cta, "Q", t, ql[t])))
+                ql[t] += 1
+            for _ in range(max(n)):
+                if g >= lag:
+                    while not ready(b("k_empty", cta, g - lag), (g - lag) // TILE_SETS):
+                        yield
+                for c in (0, 1, 2):
+                    fill(cta, (5 * g + c) % PAIR_RING, (cta, "K", g))
+                tma.append((cta, b("k_full", cta, g), (cta, "K", g)))
+                if g >= lag and bug != "pair_no_v_slot_wait":
+                    while not ready(b("v_empty", cta, g - lag), (g - lag) // TILE_SETS):
+                        yield
+                for c in (3, 4):
+                    fill(cta, (5 * g + c) % PAIR_RING, (cta, "V", g))
+                tma.append((cta, b("v_full", cta, g), (cta, "V", g)))
+                g += 1
+                yield
+
+    def relay():
+        g = 0
+        qf = [0, 0]
+        for n in units:
+            for t in range(2):
+                if n[t] == 0:
+                    continue
+                while not ready(bars["q_full", 1, t], qf[t]):
+                    yield
+                qf[t] += 1
+                if bug != "pair_no_q_relay":
+                    bars["q_full", 0, t].arrive()
+            for _ in range(max(n)):
+                for kind in ("k_full", "v_full"):
+                    while not ready(b(kind, 1, g), g // TILE_SETS):
+                        yield
+                    if not (bug == "pair_relay_skips_v" and kind == "v_full"):
+                        b(kind, 0, g).arrive()
+                g += 1
+                yield
+
+    def issue(*operands):
+        for op in operands:
+            if op not in landed:
+                raise ProtocolError("pair MMA reads %s before it landed" % (op,))
+            readers[op] = readers.get(op, 0) + 1
+        mma_queue.append(("mma", operands))
+
+    def commit_both(kind, idx):
+        mma_queue.append(("commit", [bars[kind, 0, idx], bars[kind, 1, idx]]))
+
+    def mma():
+        tg, pf, qf, qn = 0, [0, 0], [0, 0], [0, 0]
+        for n in units:
+            for t in range(2):
+                if n[t]:
+                    while not ready(bars["q_full", 0, t], qf[t]):
+                        yield
+                    qf[t] += 1
+            while not ready(b("k_full", 0, tg), tg // TILE_SETS):
+                yield
+            for t in range(2):
+                if n[t] > 0:
+                    issue((0, "Q", t, qn[t]), (1, "Q", t, qn[t]), (0, "K", tg), (1, "K", tg))
+                    commit_both("s_full", t)
+                    if n[t] == 1:
+                        commit_both("q_empty", t)
+            commit_both("k_empty", tg % TILE_SETS)
+            for j in range(max(n)):
+                g = tg + j
+                v_ready = k_ready = False
+                for t in range(2):
+                    if j < n[t]:
+                        while not ready(bars["p_full", 0, t], pf[t]):
+                            yield
+                        pf[t] += 1
+                        if not v_ready:
+                            while not ready(b("v_full", 0, g), g // TILE_SETS):
+                                yield
+                            v_ready = True
+                        issue((0, "V", g), (1, "V", g))
+                        if t == 1 or j >= n[1]:
+                            commit_both("v_empty", g % TILE_SETS)
+                    if j + 1 < n[t]:
+                        if not k_ready:
+                            while not ready(b("k_full", 0, g + 1), (g + 1) // TILE_SETS):
+                                yield
+                            k_ready = True
+                        issue((0, "Q", t, qn[t]), (1, "Q", t, qn[t]), (0, "K", g + 1), (1, "K", g + 1))
+                        commit_both("s_full", t)
+                        if j + 2 == n[t]:
+                            commit_both("q_empty", t)
+                        if t == 1 or j + 1 >= n[1]:
+                            commit_both("k_empty", (g + 1) % TILE_SETS)
+                    yield
+            for t in range(2):
+                if n[t]:
+                    qn[t] += 1
+            tg += max(n)
+
+    def softmax(cta, t):
+        sf = 0
+        for n in units:
+            for _ in range(n[t]):
+                while not ready(bars["s_full", cta, t], sf):
+                    yield
+                sf += 1
+                yield
+                bars["p_full", 0, t].arrive()
+
+    roles = [producer(0), producer(1), relay(), mma()] + [softmax(c, t) for c in range(2) for t in range(2)]
+    alive = [True] * len(roles)
+    for _ in range(800000):
+        if not (any(alive) or tma or mma_queue):
+            return
+        acts = [("role", i) for i, a in enumerate(alive) if a]
+        if tma:
+            acts.append(("tma", rnd.randrange(len(tma))))
+        if mma_queue:
+            acts.append(("mma", 0))
+        act, arg = rnd.choice(acts)
+        if act == "role":
+            try:
+                next(roles[arg])
+            except StopIteration:
+                alive[arg] = False
+        elif act == "tma":
+            cta, bar, operand = tma.pop(arg)
+            landed.add(operand)
+            bar.arrive()
+        else:
+            op, x = mma_queue.pop(0)
+            if op == "mma":
+                for operand in x:
+                    readers[operand] -= 1
+            else:
+                for bar in x:
+                    bar.arrive()
+    raise ProtocolError("deadlock")
+
+
+def test_pair_protocol_holds_under_random_schedules():
+    rng = random.Random(4048)
+    for trial in range(300):
+        simulate_pair(random_units(rng), seed=trial)
+
+
+@pytest.mark.parametrize("bug", ["pair_lag_4", "pair_no_v_slot_wait", "pair_no_q_empty_wait", "pair_no_q_relay",
+                                 "pair_relay_skips_v"])
+def test_pair_planted_protocol_mistakes_are_caught(bug):
+    rng = random.Random(11)
+    with pytest.raises(ProtocolError):
+        for trial in range(300):
+            simulate_pair(random_units(rng), seed=trial, bug=bug)
