@@ -51,6 +51,7 @@ def algorithmic_bytes(wl):
 
 
 KERNEL_SOURCES = ["mla_prefill_attention_varlen_b200/csrc/mla_prefill_sm100.cuh",
+                  "mla_prefill_attention_varlen_b200/csrc/mla_prefill_pair_sm100.cuh",
                   "mla_prefill_attention_varlen_b200/csrc/sm100_ptx.cuh"]
 
 
@@ -606,6 +607,8 @@ def main():
     ap.add_argument("--other-configs", default="varlen_gqa,chunked,uniform",
                     help="prefill on the default workload: more workloads timed in the same run and reported "
                          "under other_configs (comma-separated; empty for none)")
+    ap.add_argument("--kernel", type=int, default=-1, choices=[-1, 1, 2],
+                    help="attention kernel: -1 automatic (default), 1 single-CTA, 2 CTA pair")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling aid: scale head_num and kv_head_num down to this many query heads")
     args = ap.parse_args()
@@ -634,6 +637,7 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     mla.load_library()
     mla.set_split_tiles(args.split)
+    mla.set_kernel(args.kernel)
     x = W.make_inputs(wl, device=dev)
     out = torch.empty(wl.t_q, wl.head_num, wl.d_nope, dtype=wl.dtype, device=dev)
     H, G, scale = wl.head_num, wl.kv_head_num, wl.qk_scale
@@ -798,7 +802,7 @@ def main():
     # the other workloads, each timed in this run (single GPU, packed K/V, default workload only)
     other = None
     if (world == 1 and not paged and not args.heads and args.split < 0 and args.workload == "long"
-            and args.other_configs):
+            and args.other_configs and args.kernel < 0):
         other = {n: time_other_config(n, args.steps, args.warmup, peaks)
                  for n in args.other_configs.split(",") if n and n != wl.name}
     clocks = smi.summary()
@@ -812,6 +816,7 @@ def main():
                        "flushed between steps (512 MB write)" if flush is not None else
                        "inputs %.2f GB > 126 MB L2" % (in_bytes / 1e9)),
                    "visible_triples": triples, "split_kv": "automatic" if args.split < 0 else args.split,
+                   "kernel": {-1: "automatic", 1: "single-CTA", 2: "CTA pair"}[args.kernel],
                    **({"kv_layout": "paged", "block_size": args.block_size, "blocks": int(x["key_cache"].shape[0])}
                       if paged else {"kv_layout": "packed"})},
         "pct_of_peak": 100.0 * value / world / peak,

@@ -369,8 +369,9 @@ int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *
  * mla_prefill_ws and mla_prefill_noalloc calls on this host thread (no
  * counterpart on the pages; the result is the same operation either way).
  *   kernel = -1  automatic (the default): the CTA-pair kernel for packed,
- *                unsplit K/V once its 512-row work units give at least one
- *                work item per SM pair, else the single-CTA kernel;
+ *                unsplit K/V with long sequences (on average 3072 keys or
+ *                more per sequence) once its 512-row work units give at least
+ *                one work item per SM pair, else the single-CTA kernel;
  *   kernel =  1  the single-CTA kernel (256-row units, one SM each);
  *   kernel =  2  the CTA-pair kernel wherever it applies (packed K/V without
  *                split-KV); padded or paged K/V and split-KV always run the

@@ -422,11 +422,15 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     int rc;
     if ((rc = ensure_encode()) != MLA_OK) return rc;
     const bool general = pr.paged || pr.kv_pad > 0 || lay.split_tiles > 0;  // padded / paged K/V or split-KV
-    // The CTA-pair kernel serves packed, unsplit K/V; automatically once its 512-row units give at
-    // least as many work items as there are SM pairs.
+    // The CTA-pair kernel serves packed, unsplit K/V.  Automatically it runs long sequences (on
+    // average 3072 keys or more per sequence), where a 512-row unit walks many key tiles; short
+    // units (a few key tiles each) run faster on the single-CTA kernel, whose per-unit start and
+    // end cost less.  Either needs at least one work item per SM pair to pay off.
     const int64_t pair_items = ((pr.q.tokens + mla::pair::kUnitRows - 1) / mla::pair::kUnitRows + pr.batch) *
                                pr.head_num;
-    const bool use_pair = !general && t_kernel == 2 && pair_items > 0;
+    const bool long_keys = pr.batch > 0 && pr.k.tokens >= 3072 * pr.batch;
+    const bool use_pair = !general && pair_items > 0 &&
+                          (t_kernel == 2 || (t_kernel < 0 && long_keys && pair_items >= sm_count / 2));
     CUtensorMap maps[5];
     if ((rc = encode_map(&maps[0], pr.q, pr.bf16, ws, 128)) != MLA_OK) return rc;
     if ((rc = encode_map(&maps[1], pr.qr, pr.bf16, ws, 128)) != MLA_OK) return rc;

@@ -18,6 +18,10 @@
 //
 //   leader   warp 0: TMA loads of its halves; claims work items and hands them to both CTAs
 //            warp 1: MMA issuer for the pair
+//            warps 2, 3: helpers of groups 0, 1: for every step, once the group's S is ready,
+//                    wait until the key tile's V and the next tile's K have landed in both CTAs
+//                    and then arrive on the group's P-ready barrier, so that the MMA issuer waits
+//                    for nothing but P-ready between its MMAs
 //   follower warp 0: TMA loads of its halves (items received from the leader)
 //            warp 1: relay: once each of its loads has landed (its own barrier), arrives on the
 //                    leader's matching barrier, so the leader's MMAs see both halves
@@ -53,10 +57,11 @@ constexpr int kSmemBytes = kSmemBar + 512;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 
-// Arrivals the leader's sched_empty barrier collects per slot: its MMA warp and 8 softmax warps,
-// the follower's producer, relay and 8 softmax warps.
-constexpr int kSchedConsumers = 1 + 8 + 1 + 1 + 8;
-constexpr int kSoftmaxWarpsPerPair = 8;  // per-warp P-ready / O-free arrivals of one group, both CTAs
+// Arrivals the leader's sched_empty barrier collects per slot: its MMA warp, 2 helpers and 8
+// softmax warps, the follower's producer, relay and 8 softmax warps.
+constexpr int kSchedConsumers = 1 + 2 + 8 + 1 + 1 + 8;
+constexpr int kSoftmaxWarpsPerPair = 8;  // per-warp O-free arrivals of one group, both CTAs
+constexpr int kPReadyArrivals = kSoftmaxWarpsPerPair + 1;  // P_t(j) published by both CTAs, data seen by the helper
 
 struct Barriers {
     // full barriers: the leader's count its own producer's arrival (with the bytes it loads) and
@@ -73,14 +78,19 @@ struct Barriers {
 };
 static_assert(sizeof(Barriers) <= 512, "barrier block too large");
 
-// Bounded wait with cluster-scope acquire.  On timeout it records kStatusTimeout and raises the
-// abort flag of both CTAs; every role of both gives up at its next wait.
+// Bounded wait.  On timeout it records kStatusTimeout and raises the abort flag of both CTAs;
+// every role of both gives up at its next wait.  kCluster: acquire at cluster scope, for the one
+// phase whose guarded data is a plain shared-memory store from the peer CTA (the work item);
+// every other phase guards tensor-memory or TMA data, ordered by the tcgen05 fences and the
+// copies' completion mechanism, and is waited for at the default (CTA) scope.
+template <bool kCluster = false>
 __device__ __forceinline__ bool wait_pair(uint32_t bar, uint32_t parity, Barriers *bars, uint32_t peer_abort,
                                           int *status) {
-    if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+    auto probe = [&]() { return kCluster ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity); };
+    if (probe()) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+        if (probe()) return true;
         if ((i & 63u) == 0) {
             if (*reinterpret_cast<volatile int *>(&bars->abort)) return false;
             if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -93,9 +103,10 @@ __device__ __forceinline__ bool wait_pair(uint32_t bar, uint32_t parity, Barrier
     }
 }
 
+template <bool kCluster = false>
 __device__ __forceinline__ bool wait_pair_warp(uint32_t bar, uint32_t parity, Barriers *bars, uint32_t peer_abort,
                                                int *status) {
-    const bool ok = wait_pair(bar, parity, bars, peer_abort, status);
+    const bool ok = wait_pair<kCluster>(bar, parity, bars, peer_abort, status);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -103,7 +114,7 @@ __device__ __forceinline__ bool wait_pair_warp(uint32_t bar, uint32_t parity, Ba
 // already issued complete: used before exit so that no copy into this CTA is still in flight.
 __device__ __forceinline__ void wait_landed(uint32_t bar, uint32_t parity) {
     const uint64_t t0 = ptx::globaltimer_ns();
-    while (!ptx::mbar_try_wait_cluster(bar, parity))
+    while (!ptx::mbar_try_wait(bar, parity))
         if (ptx::globaltimer_ns() - t0 > 100000000ull) return;
 }
 
@@ -169,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(bars->q_full[t]), full_count);
             ptx::mbar_init(bar(bars->q_empty[t]), 1);
             ptx::mbar_init(bar(bars->s_full[t]), 1);
-            ptx::mbar_init(bar(bars->p_full[t]), kSoftmaxWarpsPerPair);
+            ptx::mbar_init(bar(bars->p_full[t]), kPReadyArrivals);
             ptx::mbar_init(bar(bars->o_full[t]), 1);
             ptx::mbar_init(bar(bars->o_empty[t]), kSoftmaxWarpsPerPair);
         }
@@ -205,11 +216,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Work-item hand-off, consumer side: returns the item of ring slot sc (-1: no more work).
     auto receive = [&](uint32_t sc, bool &ok) -> int {
         const uint32_t slot = sc % kSched;
-        ok = wait_pair_warp(bar(bars->sched_full[slot]), (sc / kSched) & 1, bars, peer_abort, p.status);
+        ok = wait_pair_warp<true>(bar(bars->sched_full[slot]), (sc / kSched) & 1, bars, peer_abort, p.status);
         if (!ok) return -1;
         const int it = *reinterpret_cast<volatile int *>(&bars->sched_item[slot]);
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_cluster(lead_bar(bars->sched_empty[slot]));
+        if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->sched_empty[slot]));
         __syncwarp();
         return it;
     };
@@ -252,10 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (next >= n_items) next = -1;
                     }
                 } else {
-                    ok = wait(bar(bars->sched_full[slot]), (sc / kSched) & 1);
+                    ok = wait_pair<true>(bar(bars->sched_full[slot]), (sc / kSched) & 1, bars, peer_abort, p.status);
                     if (!ok) break;
                     it = *reinterpret_cast<volatile int *>(&bars->sched_item[slot]);
-                    ptx::mbar_arrive_cluster(lead_bar(bars->sched_empty[slot]));
+                    ptx::mbar_arrive_remote(lead_bar(bars->sched_empty[slot]));
                 }
                 ++sc;
                 if (it < 0) break;
@@ -317,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             auto fwd = [&](uint64_t &b, uint32_t parity) -> bool {
                 if (!wait_pair_warp(bar(b), parity, bars, peer_abort, p.status)) return false;
-                if (lane == 0) ptx::mbar_arrive_cluster(lead_bar(b));
+                if (lane == 0) ptx::mbar_arrive_remote(lead_bar(b));
                 __syncwarp();
                 return true;
             };
@@ -332,6 +343,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t g = tg + j;
                     ok = fwd(bars->k_full[g % kTileBars], (g / kTileBars) & 1);
                     if (ok) ok = fwd(bars->v_full[g % kTileBars], (g / kTileBars) & 1);
+                }
+                tg += x.n_max;
+            }
+        } else if (warp >= 2 && leader) {
+            // ------------------------------------------------------------ helpers (leader)
+            // Warp 2 serves group 0, warp 3 group 1.  For every step j < n_t of a unit: once S_t(j)
+            // is ready (the MMA warp then has consumed the group's previous P-ready phase, so this
+            // arrival cannot fall into it), waits until key tile j's V and, if the group has a next
+            // tile, tile j + 1's K have landed in both CTAs (the leader's full barriers count the
+            // relay's arrivals), then arrives on the group's P-ready barrier.  All of this overlaps
+            // the group's softmax of step j.
+            const int t = warp - 2;
+            uint32_t ss = 0, tg = 0, sf = 0;
+            bool ok = true;
+            auto waitw = [&](uint32_t b, uint32_t parity) {
+                return wait_pair_warp(b, parity, bars, peer_abort, p.status);
+            };
+            while (ok) {
+                const int it = receive(ss++, ok);
+                if (!ok || it < 0) break;
+                const Item x = decode(p, it, num_units, kCausal, cta);
+                const int n_t = x.n[t];
+                for (int j = 0; j < n_t && ok; ++j) {
+                    const uint32_t g = tg + j;
+                    ok = waitw(bar(bars->s_full[t]), sf++ & 1);
+                    if (ok) ok = waitw(bar(bars->v_full[g % kTileBars]), (g / kTileBars) & 1);
+                    if (ok && j + 1 < n_t) ok = waitw(bar(bars->k_full[(g + 1) % kTileBars]), ((g + 1) / kTileBars) & 1);
+                    if (ok && lane == 0) ptx::mbar_arrive(bar(bars->p_full[t]));
+                    __syncwarp();
                 }
                 tg += x.n_max;
             }
@@ -423,19 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (x.n[1] == 1) commit(bars->q_empty[1]);
                 }
                 commit(bars->k_empty[tg % kTileBars]);
+                // Inside the unit the issuer waits for P-ready only: the helper has seen V_j and
+                // K_{j+1} land before its own arrival on the step's P-ready barriers.
                 for (int j = 0; j < x.n_max && ok; ++j) {
                     const uint32_t g = tg + j, kc = kTileChunks * g, vc = kc + kKChunks, kn = kc + kTileChunks;
-                    bool v_ready = false, k_next_ready = false;
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         if (ok && j < x.n[t]) {
                             uint32_t &pf = t ? pf1 : pf0;
                             uint32_t &oe = t ? oe1 : oe0;
                             ok = waitw(bar(bars->p_full[t]), pf++ & 1);
-                            if (ok && !v_ready) {
-                                ok = waitw(bar(bars->v_full[g % kTileBars]), (g / kTileBars) & 1);
-                                v_ready = true;
-                            }
                             if (ok && j == 0) ok = waitw(bar(bars->o_empty[t]), (oe++ & 1) ^ 1);
                             if (ok) {
                                 ptx::tc_fence_after();
@@ -445,16 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         if (ok && j + 1 < x.n[t]) {
-                            if (!k_next_ready) {
-                                ok = waitw(bar(bars->k_full[(g + 1) % kTileBars]), ((g + 1) / kTileBars) & 1);
-                                k_next_ready = true;
-                                if (ok) ptx::tc_fence_after();
-                            }
-                            if (ok) {
-                                issue_s(t, kn);
-                                if (j + 2 == x.n[t]) commit(bars->q_empty[t]);  // last S_t of the unit
-                                if (t == 1 || j + 1 >= x.n[1]) commit(bars->k_empty[(g + 1) % kTileBars]);
-                            }
+                            issue_s(t, kn);
+                            if (j + 2 == x.n[t]) commit(bars->q_empty[t]);  // last S_t of the unit
+                            if (t == 1 || j + 1 >= x.n[1]) commit(bars->k_empty[(g + 1) % kTileBars]);
                         }
                     }
                 }
@@ -484,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto arrive_warp = [&](uint32_t lead_addr) {
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster(lead_addr);
+            if (lane == 0) ptx::mbar_arrive_remote(lead_addr);
         };
         while (ok) {
             const int it = receive(ss++, ok);
@@ -550,16 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
                 const float2 sc2 = kPositiveScale ? make_float2(sl2, sl2) : make_float2(1.f, 1.f);
                 const float2 nm2 = make_float2(-m_use, -m_use);
-                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                 make_float2(0.f, 0.f)};
                 uint32_t pk[64];
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const float2 x2 = ptx::ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
-                    const float2 p2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
-                    acc[e & 3] = ptx::fadd2(acc[e & 3], p2);
-                    pk[e] = DType<T>::pack(p2.x, p2.y);
-                }
+                const float rowsum = exp_pack_sum<T>(s, sc2, nm2, pk);
                 ptx::tmem_st64(tS + kTmemPOff, pk);
                 // O_t holds P(j-1) V(j-1) already (the MMAs behind S_t(j) have completed);
                 // rescale it before P V(j) may start.
@@ -580,9 +602,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::tmem_st64(tO + c * 64, r);
                     }
                 }
-                const float2 acc01 = ptx::fadd2(acc[0], acc[1]), acc23 = ptx::fadd2(acc[2], acc[3]);
-                const float2 acc2 = ptx::fadd2(acc01, acc23);
-                const float rowsum = acc2.x + acc2.y;
                 ptx::tmem_wait_st();
                 arrive_warp(p_ready);
                 l_run = l_run * alpha + rowsum;

@@ -461,6 +461,24 @@ __device__ __forceinline__ float row_max(const float (&s)[kBN]) {
     return ptx::fmax3(ptx::fmax3(m[0], m[1], m[2]), ptx::fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
+// Exponentials of one row of a key tile: p = 2^(s * sc - m) for the 128 scores, packed to the
+// 16-bit P operand (pk) and summed in fp32 (returned): one packed FMA per pair, one MUFU ex2 per
+// element, four packed partial sums, one 16-bit pair conversion per pair.
+template <typename T>
+__device__ __forceinline__ float exp_pack_sum(const float (&s)[kBN], float2 sc2, float2 nm2, uint32_t (&pk)[kBN / 2]) {
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int e = 0; e < kBN / 2; ++e) {
+        const float2 x2 = ptx::ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+        const float2 p2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
+        acc[e & 3] = ptx::fadd2(acc[e & 3], p2);
+        pk[e] = DType<T>::pack(p2.x, p2.y);
+    }
+    const float2 acc01 = ptx::fadd2(acc[0], acc[1]), acc23 = ptx::fadd2(acc[2], acc[3]);
+    const float2 acc2 = ptx::fadd2(acc01, acc23);
+    return acc2.x + acc2.y;
+}
+
 // ---------------------------------------------------------------------------
 // Attention kernel
 // ---------------------------------------------------------------------------
@@ -940,20 +958,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_run = m_tile;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                // p = 2^(s * scale * log2 e - m): one packed FMA per pair, one MUFU op per element,
-                // packed partial sums, one 16-bit pair conversion per pair.
+                // p = 2^(s * scale * log2 e - m): one packed FMA per pair, packed partial sums,
+                // one 16-bit pair conversion per pair.
                 const float2 sc2 = kPositiveScale ? make_float2(sl2, sl2) : make_float2(1.f, 1.f);
                 const float2 nm2 = make_float2(-m_use, -m_use);
-                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                 make_float2(0.f, 0.f)};
                 uint32_t pk[64];
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const float2 x2 = ptx::ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
-                    const float2 p2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
-                    acc[e & 3] = ptx::fadd2(acc[e & 3], p2);
-                    pk[e] = DType<T>::pack(p2.x, p2.y);
-                }
+                const float rowsum = exp_pack_sum<T>(s, sc2, nm2, pk);
                 ptx::tmem_st64(tS + kTmemPOff, pk);
                 // O_t holds P(j-1) V(j-1) already (the MMAs behind S_t(j) have completed);
                 // rescale it before PV_t(j) may start.
@@ -974,9 +984,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::tmem_st64(tO + c * 64, r);
                     }
                 }
-                const float2 acc01 = ptx::fadd2(acc[0], acc[1]), acc23 = ptx::fadd2(acc[2], acc[3]);
-                const float2 acc2 = ptx::fadd2(acc01, acc23);
-                const float rowsum = acc2.x + acc2.y;
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(bar(bars->p_full[t]));

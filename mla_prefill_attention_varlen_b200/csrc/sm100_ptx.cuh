@@ -294,6 +294,14 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Arrive on an mbarrier given by its shared::cluster address (this CTA's or a peer's), with the
+// default semantics (release at CTA scope).  Used where the data the phase guards is ordered by
+// other means (tensor-memory stores by tcgen05.wait::st and the tcgen05 thread-sync fences,
+// shared-memory tiles by the TMA completion mechanism).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // One bounded probe with acquire semantics at cluster scope (phases completed by arrivals from
 // the peer CTA, or by a peer's writes that precede its release-arrival).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {

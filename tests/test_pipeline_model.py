@@ -228,12 +228,16 @@ def test_planted_protocol_mistakes_are_caught(bug):
 #                        K_g waits its own k_empty(g - 3), V_g its own v_empty(g - 3)
 #   relay (follower)     in the producer's order, waits for each of the follower's full
 #                        barriers and arrives on the leader's matching one
-#   MMA (leader)         as in the single-CTA kernel, waiting on the leader's full barriers
-#                        (two arrivals: the leader's own load, the relay); every release
-#                        (q_empty, k_empty, v_empty) and S-ready arrives in both CTAs; each
-#                        pair MMA reads both CTAs' halves
+#   helper t (leader)    one per group, for each step j < n_t of a unit: once S_t(j) is ready
+#                        (the leader's S-ready barrier; the MMA warp has then consumed the group's
+#                        previous P phase), waits the leader's v_full(j) and, if the group has a
+#                        next tile, k_full(j + 1) (two arrivals each: the leader's own load, the
+#                        relay), then arrives on P_t(j)
+#   MMA (leader)         per unit: waits q_full and k_full(first), issues S_0, S_1; per step:
+#                        waits P_t(j) only (three arrivals: each CTA's softmax and the helper),
+#                        P V_t(j), S_t(j + 1); every release (q_empty, k_empty, v_empty) and
+#                        S-ready arrives in both CTAs; each pair MMA reads both CTAs' halves
 #   softmax (each CTA)   group t: waits its own S_t(j), arrives on the leader's P_t(j)
-#                        (two arrivals: one per CTA)
 PAIR_RING = 16
 
 
@@ -257,7 +261,7 @@ def simulate_pair(units, seed, bug=None):
             mk("q_empty", cta, t)
             mk("s_full", cta, t)
     for t in range(2):
-        mk("p_full", 0, t, 2)
+        mk("p_full", 0, t, 3)
     owner = {}     # (cta, ring slot | ("Q", t)) -> operand last loaded there
     readers = {}   # operand -> MMAs issued and not yet completed
     landed = set()
@@ -324,6 +328,24 @@ def simulate_pair(units, seed, bug=None):
                 g += 1
                 yield
 
+    def helper(t):
+        tg, sf = 0, 0
+        for n in units:
+            for j in range(n[t]):
+                g = tg + j
+                if bug != "pair_helper_runs_ahead":
+                    while not ready(bars["s_full", 0, t], sf):
+                        yield
+                sf += 1
+                while not ready(b("v_full", 0, g), g // TILE_SETS):
+                    yield
+                if j + 1 < n[t] and bug != "pair_helper_skips_k":
+                    while not ready(b("k_full", 0, g + 1), (g + 1) // TILE_SETS):
+                        yield
+                bars["p_full", 0, t].arrive()
+                yield
+            tg += max(n)
+
     def issue(*operands):
         for op in operands:
             if op not in landed:
@@ -353,24 +375,15 @@ def simulate_pair(units, seed, bug=None):
             commit_both("k_empty", tg % TILE_SETS)
             for j in range(max(n)):
                 g = tg + j
-                v_ready = k_ready = False
                 for t in range(2):
                     if j < n[t]:
                         while not ready(bars["p_full", 0, t], pf[t]):
                             yield
                         pf[t] += 1
-                        if not v_ready:
-                            while not ready(b("v_full", 0, g), g // TILE_SETS):
-                                yield
-                            v_ready = True
                         issue((0, "V", g), (1, "V", g))
                         if t == 1 or j >= n[1]:
                             commit_both("v_empty", g % TILE_SETS)
                     if j + 1 < n[t]:
-                        if not k_ready:
-                            while not ready(b("k_full", 0, g + 1), (g + 1) // TILE_SETS):
-                                yield
-                            k_ready = True
                         issue((0, "Q", t, qn[t]), (1, "Q", t, qn[t]), (0, "K", g + 1), (1, "K", g + 1))
                         commit_both("s_full", t)
                         if j + 2 == n[t]:
@@ -393,7 +406,8 @@ def simulate_pair(units, seed, bug=None):
                 yield
                 bars["p_full", 0, t].arrive()
 
-    roles = [producer(0), producer(1), relay(), mma()] + [softmax(c, t) for c in range(2) for t in range(2)]
+    roles = [producer(0), producer(1), relay(), helper(0), helper(1), mma()] + \
+        [softmax(c, t) for c in range(2) for t in range(2)]
     alive = [True] * len(roles)
     for _ in range(800000):
         if not (any(alive) or tma or mma_queue):
@@ -431,9 +445,10 @@ def test_pair_protocol_holds_under_random_schedules():
 
 
 @pytest.mark.parametrize("bug", ["pair_lag_4", "pair_no_v_slot_wait", "pair_no_q_empty_wait", "pair_no_q_relay",
-                                 "pair_relay_skips_v"])
+                                 "pair_relay_skips_v", "pair_helper_skips_k", "pair_helper_runs_ahead"])
 def test_pair_planted_protocol_mistakes_are_caught(bug):
     rng = random.Random(11)
     with pytest.raises(ProtocolError):
         for trial in range(300):
             simulate_pair(random_units(rng), seed=trial, bug=bug)
+
