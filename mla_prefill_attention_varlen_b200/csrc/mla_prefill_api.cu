@@ -479,6 +479,8 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     p.out = pr.o.data;
     p.out_st = pr.o.st_tok;
     p.out_sh = pr.o.st_head;
+    p.out_v8 = (reinterpret_cast<uintptr_t>(pr.o.data) % 32 == 0) && (pr.o.st_tok * 2) % 32 == 0 &&
+               (pr.o.st_head * 2) % 32 == 0;
     p.head_num = pr.head_num;
     p.group = pr.head_num / pr.kv_head_num;
     // unit-major (longest-first) item order when all of K, K_rope and V fit in 48 MB of the L2

@@ -174,6 +174,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto lead_bar = [&](uint64_t &b) { return ptx::mapa_shared(ptx::smem_addr(&b), 0); };
     const uint32_t peer_abort = ptx::mapa_shared(ptx::smem_addr(&bars->abort), cta ^ 1u);
 
+    if (threadIdx.x == 32) {
+        // the tensor maps' descriptors are fetched while the CTA sets up (and, with programmatic
+        // dependent launch, while the plan kernel still runs)
+        ptx::tma_prefetch_desc(&tm_q);
+        ptx::tma_prefetch_desc(&tm_qr);
+        ptx::tma_prefetch_desc(&tm_k);
+        ptx::tma_prefetch_desc(&tm_kr);
+        ptx::tma_prefetch_desc(&tm_v);
+    }
     if (threadIdx.x == 0) {
         const uint32_t full_count = leader ? 2 : 1;
         for (int t = 0; t < 2; ++t) {
@@ -229,11 +238,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::regs_dec<kRegsLow>();
         if (warp == 0 && lane == 0) {
             // ------------------------------------------------------------ TMA producer (both CTAs)
-            ptx::tma_prefetch_desc(&tm_q);
-            ptx::tma_prefetch_desc(&tm_qr);
-            ptx::tma_prefetch_desc(&tm_k);
-            ptx::tma_prefetch_desc(&tm_kr);
-            ptx::tma_prefetch_desc(&tm_v);
             const uint64_t pol_q = ptx::policy_evict_first();
             const uint64_t pol_kv = ptx::policy_evict_last();
             auto wait = [&](uint32_t b, uint32_t parity) { return wait_pair(b, parity, bars, peer_abort, p.status); };
@@ -622,11 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     w[e] = DType<T>::pack(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
-                if (row_valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-                }
+                if (row_valid) store_row_chunk(orow + c * 32, w, p.out_v8);
             }
             arrive_warp(o_free);
         }

@@ -88,6 +88,7 @@ struct Params {
     int *status;           // sticky device status word
     void *out;
     long long out_st, out_sh;  // token / head strides of out, elements
+    int out_v8;                // every output row starts on a 32-byte boundary: 256-bit stores
     int head_num;
     int group;         // head_num / kv_head_num
     int lpt;           // 1: items unit-major (longest first across all heads); 0: kv-head-major
@@ -274,6 +275,20 @@ struct DType<__half> {
         return *reinterpret_cast<uint32_t *>(&v);
     }
 };
+
+// 32 output columns (64 bytes) of one row: two 256-bit stores when rows are 32-byte aligned,
+// else four 128-bit stores.
+template <typename T>
+__device__ __forceinline__ void store_row_chunk(T *dst, const uint32_t (&w)[16], int v8) {
+    if (v8) {
+        ptx::st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+        ptx::st_global_v8(dst + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+    } else {
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+    }
+}
 
 // ---------------------------------------------------------------------------
 // Plan kernel: one block of 1024 threads.  Clamps the seqlens to the tensor
@@ -502,6 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     auto bar = [&](uint64_t &b) { return ptx::smem_addr(&b); };
 
+    if (threadIdx.x == 32) {
+        // the tensor maps' descriptors are fetched while the CTA sets up (and, with programmatic
+        // dependent launch, while the plan kernel still runs)
+        ptx::tma_prefetch_desc(&tm_q);
+        ptx::tma_prefetch_desc(&tm_qr);
+        ptx::tma_prefetch_desc(&tm_k);
+        ptx::tma_prefetch_desc(&tm_kr);
+        ptx::tma_prefetch_desc(&tm_v);
+    }
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(bar(bars->q_full[t]), 1);
@@ -553,13 +577,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 auto wait = [&](uint32_t b, uint32_t parity) -> bool {
                     return kW ? wait_bar_warp(b, parity, bars, p.status) : wait_bar(b, parity, bars, p.status);
                 };
-                if (lead) {
-                    ptx::tma_prefetch_desc(&tm_q);
-                    ptx::tma_prefetch_desc(&tm_qr);
-                    ptx::tma_prefetch_desc(&tm_k);
-                    ptx::tma_prefetch_desc(&tm_kr);
-                    ptx::tma_prefetch_desc(&tm_v);
-                }
                 const uint64_t pol_q = ptx::policy_evict_first();
                 const uint64_t pol_kv = ptx::policy_evict_last();
                 uint32_t tk = 0, tv = 0;    // key tiles whose K / V loads have been issued
@@ -1027,11 +1044,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     w[e] = DType<T>::pack(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
-                if (row_valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-                }
+                if (row_valid) store_row_chunk(orow + c * 32, w, p.out_v8);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(bar(bars->o_empty[t]));

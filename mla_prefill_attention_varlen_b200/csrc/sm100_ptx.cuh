@@ -373,6 +373,16 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask)
         : "memory");
 }
 
+// ---------------------------------------------------------------- 256-bit global store
+// Eight 32-bit words to a 32-byte-aligned global address in one instruction: a warp's store then
+// writes whole 32-byte sectors, one per thread, whatever the distance between the threads' rows.
+__device__ __forceinline__ void st_global_v8(void *addr, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                             uint32_t w4, uint32_t w5, uint32_t w6, uint32_t w7) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(addr), "r"(w0), "r"(w1), "r"(w2),
+                 "r"(w3), "r"(w4), "r"(w5), "r"(w6), "r"(w7)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------- packed fp32 math
 // Two fp32 lanes per instruction (sm_100 f32x2 forms), and a three-input max.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {

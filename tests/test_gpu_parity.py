@@ -206,6 +206,14 @@ def test_strided_and_2d_views():
     run(x, H, G, 0.07, out=out2d)
     torch.cuda.synchronize()
     assert torch.equal(out2d.view(T, H, 128), ref_out)
+    # output rows on 16-byte but not 32-byte boundaries (the epilogue's 128-bit store path)
+    wide16 = torch.full((T, H, 160), 3.0, dtype=torch.bfloat16, device=DEV)
+    out16 = wide16[:, :, 8:136]
+    assert out16.data_ptr() % 32 == 16
+    run(x, H, G, 0.07, out=out16)
+    torch.cuda.synchronize()
+    assert torch.equal(out16, ref_out)
+    assert torch.all(wide16[:, :, :8] == 3.0) and torch.all(wide16[:, :, 136:] == 3.0)
 
 
 # ---------------------------------------------------------------------------
