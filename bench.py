@@ -67,6 +67,10 @@ def kernel_sources_hash():
     return h.hexdigest()
 
 
+# attention kernel of a prefill call (mla_prefill_last_kernel) -> its name
+KERNEL_NAMES = {1: "mla_prefill_sm100_kernel", 2: "mla_prefill_pair_kernel"}
+
+
 def measured_traffic(workload):
     """DRAM bytes per launch from the committed ncu figures (profiles/traffic.json), or None when
     there is no figure for this workload or it was taken on different kernel sources."""
@@ -578,11 +582,13 @@ def time_other_config(name, steps, warmup, peaks):
         raise RuntimeError("device status after %s: %s" % (name, mla.mla_status_string(st)))
     ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev[0], ev[1])]))
     kms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev[2], ev[3])]))
+    kernel_name = KERNEL_NAMES.get(mla.load_library().mla_prefill_last_kernel(), "none")
     flops = visible_triples(wl) * FLOPS_PER_TRIPLE
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     ab = algorithmic_bytes(wl)
-    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "kernel_ms": kms,
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms, "kernel": kernel_name,
+            "kernel_ms": kms,
             "kernel_tflops": flops / (kms * 1e-3) / 1e12, "frac": flops / (kms * 1e-3) / 1e12 / peak,
             "hbm_gbs": ab / (kms * 1e-3) / 1e9, "hbm_frac": ab / (kms * 1e-3) / 1e9 / hbm,
             "tokens_per_s": wl.t_q / (ms * 1e-3), "steps": steps, "warmup": warmup,
@@ -714,6 +720,7 @@ def main():
     ms = max_over_ranks(float(np.mean(step_ms)), world)
     kms = max_over_ranks(float(np.mean(kern_ms)), world)
     launches_per_step = mla.load_library().mla_prefill_last_launches()  # plan + attention (+ combine)
+    kernel_name = KERNEL_NAMES.get(mla.load_library().mla_prefill_last_kernel(), "none")
     st = mla.mla_prefill_device_status()
     if st != 0:
         raise RuntimeError("device status after timing: %s" % mla.mla_status_string(st))
@@ -841,7 +848,7 @@ def main():
                      "traffic": measured_traffic("%s_paged%d" % (wl.name, args.block_size) if paged else wl.name),
                      "peak_source": peak_src,
                      "peak_kind": "burst", "frac_of_sustained": kern_tflops / peak_sus,
-                     "kernel": "mla_prefill_sm100_kernel", "kernel_ms": kms,
+                     "kernel": kernel_name, "kernel_ms": kms,
                      "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": algo_bytes,
                      # the same launch against the HBM roofline (the bound near the ridge, e.g. `uniform`)
                      "hbm_achieved_gbs": algo_bytes / (kms * 1e-3) / 1e9, "hbm_peak_gbs": hbm_peak,

@@ -418,6 +418,10 @@ int mla_selftest_wait_timeout(int wait_ms, mla_stream_t stream);
  * enqueued: 2 (plan + attention), 3 with split-KV (+ combine), 0 if it launched nothing. */
 int mla_prefill_last_launches(void);
 
+/* Attention kernel the last mla_prefill / mla_prefill_ws / mla_prefill_paged / mla_prefill_noalloc
+ * call of this host thread launched: 1 the single-CTA kernel, 2 the CTA-pair kernel, 0 none. */
+int mla_prefill_last_kernel(void);
+
 /* Library version as 10000*major + 100*minor + patch. */
 int mla_prefill_version(void);
 

@@ -85,6 +85,8 @@ def load_library(path=None):
     lib.mla_selftest_wait_timeout.restype = ctypes.c_int
     lib.mla_prefill_last_launches.argtypes = []
     lib.mla_prefill_last_launches.restype = ctypes.c_int
+    lib.mla_prefill_last_kernel.argtypes = []
+    lib.mla_prefill_last_kernel.restype = ctypes.c_int
     lib.mla_prefill_set_kernel.argtypes = [ctypes.c_int]
     lib.mla_prefill_set_kernel.restype = ctypes.c_int
     lib.mla_prefill_set_split_tiles.argtypes = [ctypes.c_int]

@@ -37,6 +37,7 @@ thread_local cudaEvent_t t_prof_start = nullptr, t_prof_stop = nullptr;
 thread_local int t_split_tiles = -1;  // split-KV chunk in key tiles: -1 automatic, 0 off
 thread_local int t_kernel = -1;       // attention kernel: -1 automatic, 1 single-CTA, 2 CTA pair
 thread_local int t_last_launches = 0;  // kernels the last prefill call of this thread enqueued
+thread_local int t_last_kernel = 0;    // attention kernel of that call: 1 single-CTA, 2 CTA pair
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -446,8 +447,8 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
                                    pr.vc_block, pr.vc_slot, pr.vc_head, pr.bf16, rows_v)) != MLA_OK)
             return rc;
     } else {
-        // pair kernel: each CTA loads 64 keys of K per key tile
-        const int kbox = use_pair ? 64 : 128;
+        // pair kernel: each CTA loads 32 keys of K per 64-key tile
+        const int kbox = use_pair ? 32 : 128;
         if ((rc = encode_map(&maps[2], pr.k, pr.bf16, ws, kbox)) != MLA_OK) return rc;
         if ((rc = encode_map(&maps[3], pr.kr, pr.bf16, ws, kbox)) != MLA_OK) return rc;
         if ((rc = encode_map(&maps[4], pr.v, pr.bf16, ws, 64)) != MLA_OK) return rc;
@@ -513,6 +514,7 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
         }
 #undef MLA_PAIR
         t_last_launches = 2;  // plan + attention
+        t_last_kernel = 2;
         return rc;
     }
 
@@ -533,6 +535,7 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
 #undef MLA_PICK
 #undef MLA_LAUNCH
     t_last_launches = 2;  // plan + attention
+    t_last_kernel = 1;
     if (rc != MLA_OK || lay.split_tiles <= 0) return rc;
     t_last_launches = 3;  // + combine
     // split-KV: merge the chunks of every unit that has several
@@ -677,6 +680,7 @@ int mla_prefill(const mla_tensor *q, const mla_tensor *q_rope, const mla_tensor 
                 const mla_tensor *v, const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type,
                 int head_num, int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
     t_last_launches = 0;
+    t_last_kernel = 0;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     Problem pr;
     int rc = validate(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
@@ -741,6 +745,7 @@ int mla_prefill_ws(const mla_tensor *q, const mla_tensor *q_rope, const mla_tens
                    int head_num, int kv_head_num, float qk_scale, mla_tensor *out, void *workspace,
                    uint64_t workspace_bytes, mla_stream_t stream_) {
     t_last_launches = 0;
+    t_last_kernel = 0;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     Problem pr;
     WsLayout lay;
@@ -806,6 +811,8 @@ int mla_selftest_wait_timeout(int wait_ms, mla_stream_t stream_) {
 
 int mla_prefill_last_launches(void) { return t_last_launches; }
 
+int mla_prefill_last_kernel(void) { return t_last_kernel; }
+
 int mla_prefill_set_kernel(int kernel) {
     if (kernel != -1 && kernel != 1 && kernel != 2) return MLA_ERR_UNSUPPORTED;
     t_kernel = kernel;
@@ -838,6 +845,7 @@ extern "C" int mla_prefill_noalloc(const mla_tensor *q, const mla_tensor *q_rope
                                    const mla_tensor *kv_seqlen, int mask_type, int head_num, int kv_head_num,
                                    float qk_scale, mla_tensor *out, mla_stream_t stream_) {
     t_last_launches = 0;
+    t_last_kernel = 0;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     Problem pr;
     int rc = validate(q, q_rope, k, k_rope, v, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num, qk_scale, out,
@@ -1051,6 +1059,7 @@ extern "C" int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, 
                                  const mla_tensor *q_seqlen, const mla_tensor *kv_seqlen, int mask_type, int head_num,
                                  int kv_head_num, float qk_scale, mla_tensor *out, mla_stream_t stream_) {
     t_last_launches = 0;
+    t_last_kernel = 0;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (!key_cache || !value_cache || !block_tables) return MLA_ERR_NULL;
     Problem pr;

@@ -12,16 +12,22 @@
 // warp issues M = 256 tensor-core MMAs over the pair (tcgen05 cta_group::2): each CTA's tensor
 // memory receives its own 128 rows, the A operand (Q or P) comes from each CTA's own shared or
 // tensor memory, and the B operand (K for S, V for P V) is split along N: each CTA loads only
-// its half of every key tile -- 64 of the 128 keys of K, 64 of the 128 columns of V.  Per CTA
-// that halves the shared-memory bytes loaded per key tile and the B-operand bytes the tensor
-// core reads per FLOP, and a single thread issues the MMAs of two SMs.
+// its half of every key tile -- 32 of the 64 keys of K, 64 of the 128 columns of V.
+//
+// Key tiles are 64 keys, and each group has two S buffers in tensor memory: S of the group's
+// g-th tile (counted across units) goes to buffer g mod 2, and the softmax writes P over the
+// buffer it has just read.  The MMA warp issues S_t(j + 2) right after P V_t(j) -- into the
+// buffer P V_t(j) reads, which the in-order tensor pipe empties first -- so S of the next tile
+// is computed while the softmax still works on the current one: the softmax runs tile after
+// tile without waiting for P V and the next S, and the tensor pipe has the other group's work
+// and this group's next S to fill its time.
 //
 //   leader   warp 0: TMA loads of its halves; claims work items and hands them to both CTAs
 //            warp 1: MMA issuer for the pair
-//            warps 2, 3: helpers of groups 0, 1: for every step, once the group's S is ready,
-//                    wait until the key tile's V and the next tile's K have landed in both CTAs
-//                    and then arrive on the group's P-ready barrier, so that the MMA issuer waits
-//                    for nothing but P-ready between its MMAs
+//            warps 2, 3: helpers of groups 0, 1: for every tile, wait until the key tile's V
+//                    and the K of the group's tile two ahead have landed in both CTAs, then
+//                    arrive on the group's P-ready barrier, so that the MMA issuer waits for
+//                    nothing but P-ready between its MMAs
 //   follower warp 0: TMA loads of its halves (items received from the leader)
 //            warp 1: relay: once each of its loads has landed (its own barrier), arrives on the
 //                    leader's matching barrier, so the leader's MMAs see both halves
@@ -30,8 +36,8 @@
 //
 // Every TMA load completes on a barrier of the CTA it writes to, so each CTA can wait for its
 // own copies before it exits.  Commits of the pair MMAs arrive on the same barrier in both CTAs
-// (multicast); P-ready and O-free arrivals of the follower's softmax warps go to the leader's
-// barriers.  All waits are bounded; a timeout in either CTA aborts both.
+// (multicast); P-ready arrivals of the follower's softmax warps go to the leader's barriers.
+// All waits are bounded; a timeout in either CTA aborts both.
 #pragma once
 
 #include "mla_prefill_sm100.cuh"
@@ -39,37 +45,43 @@
 namespace mla {
 namespace pair {
 
-constexpr int kUnitRows = 512;          // query rows per work unit (two groups of 256)
-constexpr int kGroupRows = 256;         // rows of one pair MMA (128 per CTA)
-constexpr int kChunkBytes = 8192;       // one ring chunk: 64 rows x 128 B
-constexpr int kRing = 16;               // ring chunks per CTA (128 KB)
-constexpr int kKChunks = 3;             // this CTA's 64 keys: nope cols 0-63 | nope cols 64-127 | rope
-constexpr int kVChunks = 2;             // keys 0-63 | keys 64-127, this CTA's 64 V columns each
-constexpr int kTileChunks = kKChunks + kVChunks;
-constexpr int kQTileBytes = 3 * 16384;  // this CTA's 128 rows of a group: nope lo | nope hi | rope
-constexpr int kTileBars = 4;            // key-tile barrier sets
+constexpr int kUnitRows = 512;           // query rows per work unit (two groups of 256)
+constexpr int kGroupRows = 256;          // rows of one pair MMA (128 per CTA)
+constexpr int kKeys = 64;                // keys per key tile
+constexpr int kSlots = 6;                // key-tile slots in each CTA's ring
+constexpr int kKPart = 4096;             // this CTA's 32 keys x 64 channels (128 B rows)
+constexpr int kVBytes = 8192;            // 64 keys x this CTA's 64 V columns (128 B rows)
+constexpr int kSlotBytes = 3 * kKPart + kVBytes;  // K: nope 0-63 | nope 64-127 | rope, then V
+constexpr int kQTileBytes = 3 * 16384;   // this CTA's 128 rows of a group: nope lo | nope hi | rope
 constexpr int kSched = 4;
 
 constexpr int kSmemQ = 0;
 constexpr int kSmemRing = kSmemQ + 2 * kQTileBytes;
-constexpr int kSmemBar = kSmemRing + kRing * kChunkBytes;
+constexpr int kSmemBar = kSmemRing + kSlots * kSlotBytes;
 constexpr int kSmemBytes = kSmemBar + 512;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
+static_assert(kSlotBytes % 1024 == 0 && kKPart % 1024 == 0, "128-byte-swizzle atoms stay 1024-byte aligned");
+
+// Tensor memory (512 columns): O_t at 128 t; S_t buffer b at 256 + 128 t + 64 b, P_t of that
+// buffer's tile over its first 32 columns (64 16-bit values per row).
+constexpr uint32_t kTmemOBase = 0;
+constexpr uint32_t kTmemSBase = 256;
 
 // Arrivals the leader's sched_empty barrier collects per slot: its MMA warp, 2 helpers and 8
 // softmax warps, the follower's producer, relay and 8 softmax warps.
 constexpr int kSchedConsumers = 1 + 2 + 8 + 1 + 1 + 8;
-constexpr int kSoftmaxWarpsPerPair = 8;  // per-warp O-free arrivals of one group, both CTAs
-constexpr int kPReadyArrivals = kSoftmaxWarpsPerPair + 1;  // P_t(j) published by both CTAs, data seen by the helper
+constexpr int kSoftmaxWarpsPerPair = 8;  // per-warp arrivals of one group, both CTAs
+constexpr int kPReadyArrivals = kSoftmaxWarpsPerPair + 1;  // P_t(g) published by both CTAs, data seen by the helper
 
 struct Barriers {
     // full barriers: the leader's count its own producer's arrival (with the bytes it loads) and
     // the follower relay's arrival; the follower's count its own producer's arrival only
     uint64_t q_full[2], q_empty[2];
-    uint64_t k_full[kTileBars], v_full[kTileBars], k_empty[kTileBars], v_empty[kTileBars];
-    uint64_t s_full[2], p_full[2];
-    uint64_t o_full[2], o_empty[2];
+    uint64_t k_full[kSlots], v_full[kSlots], k_empty[kSlots], v_empty[kSlots];
+    // [group][tile parity]: S buffer full, P-ready, P V done of the group's tiles of that parity
+    uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];
+    uint64_t o_full[2];
     uint64_t sched_full[kSched], sched_empty[kSched];
     uint64_t drain;
     int sched_item[kSched];
@@ -124,9 +136,17 @@ struct Item {
     int q_tok0, k_tok0;  // first packed token of the unit / of the sequence's keys
     int lq, lk, off;     // off = Lk - Lq
     int rows[2];         // this CTA's valid rows in group 0 / 1
-    int n[2];            // key tiles of group 0 / 1: the larger of its two halves' counts
+    int n[2];            // 64-key tiles of group 0 / 1: the larger of its two halves' counts
     int n_max;
 };
+
+// 64-key tiles a 128-row query tile touches: the keys visible to its last row (causal) or all
+// keys; 0 when the tile has no rows or sees no key.
+__device__ __forceinline__ int key_tiles(int q0, int rows, int lq, int lk, bool causal) {
+    if (rows <= 0) return 0;
+    const int kv_end = causal ? min(q0 + rows + (lk - lq), lk) : lk;
+    return kv_end > 0 ? (kv_end + kKeys - 1) / kKeys : 0;
+}
 
 // Items are ordered as in the single-CTA kernel (kv-head-major, or unit-major when K/V fits in L2).
 __device__ __forceinline__ Item decode(const Params &p, int it, int num_units, bool causal, uint32_t cta) {
@@ -145,13 +165,47 @@ __device__ __forceinline__ Item decode(const Params &p, int it, int num_units, b
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int r0 = x.u0 + t * kGroupRows, r1 = r0 + kBM;
-        const int n0 = kv_tiles_for(r0, tile_rows(r0, s.z), s.z, s.w, causal);
-        const int n1 = kv_tiles_for(r1, tile_rows(r1, s.z), s.z, s.w, causal);
+        const int n0 = key_tiles(r0, tile_rows(r0, s.z), s.z, s.w, causal);
+        const int n1 = key_tiles(r1, tile_rows(r1, s.z), s.z, s.w, causal);
         x.n[t] = max(n0, n1);
         x.rows[t] = tile_rows(cta ? r1 : r0, s.z);
     }
     x.n_max = max(x.n[0], x.n[1]);
     return x;
+}
+
+// Max of a 64-element row: eight independent chains of three-input max, then a short tree.
+__device__ __forceinline__ float row_max64(const float (&s)[kKeys]) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = ptx::fmax3(s[i], s[i + 8], s[i + 16]);  // s[0..23]
+#pragma unroll
+    for (int c = 24; c + 16 <= kKeys; c += 16) {                               // s[24..55]
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = ptx::fmax3(m[i], s[c + i], s[c + 8 + i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], s[56 + i]);                 // s[56..63]
+    return ptx::fmax3(ptx::fmax3(m[0], m[1], m[2]), ptx::fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// Exponentials of one row of a key tile: p = 2^(s * sc - m) for the 64 scores, packed to the
+// 16-bit P operand (pk) and summed in fp32 (returned): one packed FMA per pair, one MUFU ex2 per
+// element, four packed partial sums, one 16-bit pair conversion per pair.
+template <typename T>
+__device__ __forceinline__ float exp_pack_sum64(const float (&s)[kKeys], float2 sc2, float2 nm2,
+                                                uint32_t (&pk)[kKeys / 2]) {
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int e = 0; e < kKeys / 2; ++e) {
+        const float2 x2 = ptx::ffma2(make_float2(s[2 * e], s[2 * e + 1]), sc2, nm2);
+        const float2 p2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
+        acc[e & 3] = ptx::fadd2(acc[e & 3], p2);
+        pk[e] = DType<T>::pack(p2.x, p2.y);
+    }
+    const float2 acc01 = ptx::fadd2(acc[0], acc[1]), acc23 = ptx::fadd2(acc[2], acc[3]);
+    const float2 acc2 = ptx::fadd2(acc01, acc23);
+    return acc2.x + acc2.y;
 }
 
 template <typename T, bool kCausal, bool kPositiveScale>
@@ -188,12 +242,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(bar(bars->q_full[t]), full_count);
             ptx::mbar_init(bar(bars->q_empty[t]), 1);
-            ptx::mbar_init(bar(bars->s_full[t]), 1);
-            ptx::mbar_init(bar(bars->p_full[t]), kPReadyArrivals);
+            for (int b = 0; b < 2; ++b) {
+                ptx::mbar_init(bar(bars->s_full[t][b]), 1);
+                ptx::mbar_init(bar(bars->p_full[t][b]), kPReadyArrivals);
+                ptx::mbar_init(bar(bars->pv_done[t][b]), 1);
+            }
             ptx::mbar_init(bar(bars->o_full[t]), 1);
-            ptx::mbar_init(bar(bars->o_empty[t]), kSoftmaxWarpsPerPair);
         }
-        for (int c = 0; c < kTileBars; ++c) {
+        for (int c = 0; c < kSlots; ++c) {
             ptx::mbar_init(bar(bars->k_full[c]), full_count);
             ptx::mbar_init(bar(bars->v_full[c]), full_count);
             ptx::mbar_init(bar(bars->k_empty[c]), 1);
@@ -241,13 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_q = ptx::policy_evict_first();
             const uint64_t pol_kv = ptx::policy_evict_last();
             auto wait = [&](uint32_t b, uint32_t parity) { return wait_pair(b, parity, bars, peer_abort, p.status); };
-            auto chunk = [&](uint32_t c) { return sRing + (c % kRing) * kChunkBytes; };
             uint32_t tk = 0, tv = 0, ql0 = 0, ql1 = 0;
             bool ok = true;
-            // Key tile g sits in ring chunks 5g .. 5g + 4 (mod 16).  K_g's chunks last held V_{g-4}'s
-            // second chunk and K_{g-3}'s first two; V_g's chunks last held K_{g-3}'s third and
-            // V_{g-3}'s first.  The commit releasing K_{g-3} follows every MMA reading V_{g-4}, so
-            // K_g waits for K_{g-3}'s release and V_g for V_{g-3}'s.
+            // Key tile g (counted across units) sits in slot g mod 6; its K waits for the release of
+            // tile g - 6's K, its V for that of tile g - 6's V.
             uint32_t sc = 0;
             int next = cluster_id < n_items ? cluster_id : -1;
             while (ok) {
@@ -292,26 +345,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++ql;
                 }
                 for (int j = 0; j < x.n_max && ok; ++j) {
-                    const int tok = x.k_tok0 + j * kBN;
-                    const uint32_t g = tk, c0 = kTileChunks * g;
-                    // K_j: this CTA's 64 keys, nope cols 0-63 | nope cols 64-127 | rope
-                    if (g >= 3 && !(ok = wait(bar(bars->k_empty[(g - 3) % kTileBars]), ((g - 3) / kTileBars) & 1)))
-                        break;
-                    uint32_t fb = bar(bars->k_full[g % kTileBars]);
-                    ptx::mbar_arrive_expect_tx(fb, kKChunks * kChunkBytes);
-                    const int ktok = tok + static_cast<int>(cta) * 64;
-                    ptx::tma_load_3d(chunk(c0), &tm_k, fb, 0, x.kh, ktok, pol_kv);
-                    ptx::tma_load_3d(chunk(c0 + 1), &tm_k, fb, 64, x.kh, ktok, pol_kv);
-                    ptx::tma_load_3d(chunk(c0 + 2), &tm_kr, fb, 0, x.kh, ktok, pol_kv);
+                    const int tok = x.k_tok0 + j * kKeys;
+                    const uint32_t g = tk, slot = g % kSlots, phase = ((g / kSlots) & 1) ^ 1;
+                    const uint32_t dst = sRing + slot * kSlotBytes;
+                    // K_g: this CTA's 32 keys, nope cols 0-63 | nope cols 64-127 | rope
+                    if (g >= kSlots && !(ok = wait(bar(bars->k_empty[slot]), phase))) break;
+                    uint32_t fb = bar(bars->k_full[slot]);
+                    ptx::mbar_arrive_expect_tx(fb, 3 * kKPart);
+                    const int ktok = tok + static_cast<int>(cta) * (kKeys / 2);
+                    ptx::tma_load_3d(dst, &tm_k, fb, 0, x.kh, ktok, pol_kv);
+                    ptx::tma_load_3d(dst + kKPart, &tm_k, fb, 64, x.kh, ktok, pol_kv);
+                    ptx::tma_load_3d(dst + 2 * kKPart, &tm_kr, fb, 0, x.kh, ktok, pol_kv);
                     ++tk;
-                    // V_j: keys 0-63 | keys 64-127, this CTA's 64 columns
-                    if (g >= 3 && !(ok = wait(bar(bars->v_empty[(g - 3) % kTileBars]), ((g - 3) / kTileBars) & 1)))
-                        break;
-                    fb = bar(bars->v_full[g % kTileBars]);
-                    ptx::mbar_arrive_expect_tx(fb, kVChunks * kChunkBytes);
-                    const int vcol = static_cast<int>(cta) * 64;
-                    ptx::tma_load_3d(chunk(c0 + 3), &tm_v, fb, vcol, x.kh, tok, pol_kv);
-                    ptx::tma_load_3d(chunk(c0 + 4), &tm_v, fb, vcol, x.kh, tok + 64, pol_kv);
+                    // V_g: the 64 keys, this CTA's 64 columns
+                    if (g >= kSlots && !(ok = wait(bar(bars->v_empty[slot]), phase))) break;
+                    fb = bar(bars->v_full[slot]);
+                    ptx::mbar_arrive_expect_tx(fb, kVBytes);
+                    ptx::tma_load_3d(dst + 3 * kKPart, &tm_v, fb, static_cast<int>(cta) * 64, x.kh, tok, pol_kv);
                     ++tv;
                 }
             }
@@ -320,10 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // arrival, which may never come after an abort: the wait is bounded either way.
             if (ql0) wait_landed(bar(bars->q_full[0]), (ql0 - 1) & 1);
             if (ql1) wait_landed(bar(bars->q_full[1]), (ql1 - 1) & 1);
-            for (uint32_t g = tk > kTileBars ? tk - kTileBars : 0; g < tk; ++g)
-                wait_landed(bar(bars->k_full[g % kTileBars]), (g / kTileBars) & 1);
-            for (uint32_t g = tv > kTileBars ? tv - kTileBars : 0; g < tv; ++g)
-                wait_landed(bar(bars->v_full[g % kTileBars]), (g / kTileBars) & 1);
+            for (uint32_t g = tk > kSlots ? tk - kSlots : 0; g < tk; ++g)
+                wait_landed(bar(bars->k_full[g % kSlots]), (g / kSlots) & 1);
+            for (uint32_t g = tv > kSlots ? tv - kSlots : 0; g < tv; ++g)
+                wait_landed(bar(bars->v_full[g % kSlots]), (g / kSlots) & 1);
         } else if (warp == 1 && !leader) {
             // ------------------------------------------------------------ relay (follower)
             // Follows the producer's order of loads: each time one of this CTA's loads has landed,
@@ -345,21 +395,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok && x.n[1]) ok = fwd(bars->q_full[1], qf1++ & 1);
                 for (int j = 0; j < x.n_max && ok; ++j) {
                     const uint32_t g = tg + j;
-                    ok = fwd(bars->k_full[g % kTileBars], (g / kTileBars) & 1);
-                    if (ok) ok = fwd(bars->v_full[g % kTileBars], (g / kTileBars) & 1);
+                    ok = fwd(bars->k_full[g % kSlots], (g / kSlots) & 1);
+                    if (ok) ok = fwd(bars->v_full[g % kSlots], (g / kSlots) & 1);
                 }
                 tg += x.n_max;
             }
         } else if (warp >= 2 && leader) {
             // ------------------------------------------------------------ helpers (leader)
-            // Warp 2 serves group 0, warp 3 group 1.  For every step j < n_t of a unit: once S_t(j)
-            // is ready (the MMA warp then has consumed the group's previous P-ready phase, so this
-            // arrival cannot fall into it), waits until key tile j's V and, if the group has a next
-            // tile, tile j + 1's K have landed in both CTAs (the leader's full barriers count the
-            // relay's arrivals), then arrives on the group's P-ready barrier.  All of this overlaps
-            // the group's softmax of step j.
+            // Warp 2 serves group 0, warp 3 group 1.  For the group's g-th tile (step j of a unit):
+            // waits until S_t(g) has completed -- it was issued after P V_t(g - 2), so the P-ready
+            // phase of tile g - 2 (the same barrier's previous one) is complete and this arrival
+            // cannot fall into it, and every slot checked next is within one phase of the tile
+            // asked for -- then until the tile's V and, if the group has a tile j + 2, that tile's
+            // K have landed in both CTAs (the leader's full barriers count the relay's arrivals),
+            // and arrives on the group's P-ready barrier of the tile's parity.  All of this
+            // overlaps the group's softmax of the tile.
             const int t = warp - 2;
-            uint32_t ss = 0, tg = 0, sf = 0;
+            uint32_t ss = 0, tg = 0, gt = 0;
             bool ok = true;
             auto waitw = [&](uint32_t b, uint32_t parity) {
                 return wait_pair_warp(b, parity, bars, peer_abort, p.status);
@@ -369,12 +421,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok || it < 0) break;
                 const Item x = decode(p, it, num_units, kCausal, cta);
                 const int n_t = x.n[t];
-                for (int j = 0; j < n_t && ok; ++j) {
-                    const uint32_t g = tg + j;
-                    ok = waitw(bar(bars->s_full[t]), sf++ & 1);
-                    if (ok) ok = waitw(bar(bars->v_full[g % kTileBars]), (g / kTileBars) & 1);
-                    if (ok && j + 1 < n_t) ok = waitw(bar(bars->k_full[(g + 1) % kTileBars]), ((g + 1) / kTileBars) & 1);
-                    if (ok && lane == 0) ptx::mbar_arrive(bar(bars->p_full[t]));
+                for (int j = 0; j < n_t && ok; ++j, ++gt) {
+                    const uint32_t kg = tg + j;
+                    ok = waitw(bar(bars->s_full[t][gt & 1]), (gt >> 1) & 1);
+                    if (ok) ok = waitw(bar(bars->v_full[kg % kSlots]), (kg / kSlots) & 1);
+                    if (ok && j + 2 < n_t)
+                        ok = waitw(bar(bars->k_full[(kg + 2) % kSlots]), ((kg + 2) / kSlots) & 1);
+                    if (ok && lane == 0) ptx::mbar_arrive(bar(bars->p_full[t][gt & 1]));
                     __syncwarp();
                 }
                 tg += x.n_max;
@@ -382,15 +435,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (warp == 1) {
             // ------------------------------------------------------------ MMA issuer (leader)
             constexpr bool kBf16 = DType<T>::kBf16;
-            constexpr uint32_t kIdQK = ptx::instr_desc_f16(kBf16, kGroupRows, kBN, false);
+            constexpr uint32_t kIdQK = ptx::instr_desc_f16(kBf16, kGroupRows, kKeys, false);
             constexpr uint32_t kIdPV = ptx::instr_desc_f16(kBf16, kGroupRows, kDn, true);
             constexpr uint32_t kHi = ptx::desc_hi_sw128(1024);
             constexpr uint16_t kBoth = 3;  // commits arrive in both CTAs
             const uint32_t q_lo = ptx::desc_lo(sQ, 16);
             const uint32_t ring_k_lo = ptx::desc_lo(sRing, 16);
-            const uint32_t ring_v_lo = ptx::desc_lo(sRing, kChunkBytes);
-            constexpr uint32_t kC = kChunkBytes >> 4;  // one ring chunk in descriptor units
-            uint32_t tg = 0, qf0 = 0, qf1 = 0, pf0 = 0, pf1 = 0, oe0 = 0, oe1 = 0;
+            const uint32_t ring_v_lo = ptx::desc_lo(sRing + 3 * kKPart, kVBytes);
+            constexpr uint32_t kSlotU = kSlotBytes >> 4;  // one slot in descriptor units
+            constexpr uint32_t kPartU = kKPart >> 4;
+            uint32_t tg = 0, qf0 = 0, qf1 = 0, gs0 = 0, gs1 = 0;
             bool ok = true;
             auto waitw = [&](uint32_t b, uint32_t parity) {
                 return wait_pair_warp(b, parity, bars, peer_abort, p.status);
@@ -399,13 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ptx::elect_one()) ptx::mma_commit_pair(bar(b), kBoth);
                 __syncwarp();
             };
-            // S_t = [Qn|Qr]_t [Kn|Kr]^T over the pair: 12 k-steps of 16 channels
-            auto issue_s = [&](int t, uint32_t kc) {
-                const uint32_t d = tmem + kTmemS + t * kBN;
+            // S_t = [Qn|Qr]_t [Kn|Kr]^T of key tile kg into S buffer sb: 12 k-steps of 16 channels
+            auto issue_s = [&](int t, uint32_t kg, uint32_t sb) {
+                const uint32_t d = tmem + kTmemSBase + t * 128 + sb * kKeys;
                 const uint32_t a0 = q_lo + ((t * kQTileBytes) >> 4);
-                const uint32_t b0 = ring_k_lo + ((kc + 0) % kRing) * kC;
-                const uint32_t b1 = ring_k_lo + ((kc + 1) % kRing) * kC;
-                const uint32_t b2 = ring_k_lo + ((kc + 2) % kRing) * kC;
+                const uint32_t b0 = ring_k_lo + (kg % kSlots) * kSlotU;
+                const uint32_t b1 = b0 + kPartU, b2 = b0 + 2 * kPartU;
                 if (ptx::elect_one()) {
                     constexpr uint32_t kQC = 16384 >> 4;  // one Q chunk (128 rows x 128 B)
                     ptx::mma2_ss_lo<kHi, kIdQK, 0>(d, a0 + 0, b0 + 0);
@@ -420,16 +473,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mma2_ss_lo<kHi, kIdQK, 1>(d, a0 + 2 * kQC + 2, b2 + 2);
                     ptx::mma2_ss_lo<kHi, kIdQK, 1>(d, a0 + 2 * kQC + 4, b2 + 4);
                     ptx::mma2_ss_lo<kHi, kIdQK, 1>(d, a0 + 2 * kQC + 6, b2 + 6);
-                    ptx::mma_commit_pair(bar(bars->s_full[t]), kBoth);
+                    ptx::mma_commit_pair(bar(bars->s_full[t][sb]), kBoth);
                 }
                 __syncwarp();
             };
-            // O_t (+)= P_t V over the pair: 8 k-steps of 16 keys, P from tensor memory
-            auto issue_pv = [&](int t, uint32_t vc, bool accumulate) {
-                const uint32_t d = tmem + kTmemO + t * kDn;
-                const uint32_t pa = tmem + kTmemS + t * kBN + kTmemPOff;
-                const uint32_t v0 = ring_v_lo + ((vc + 0) % kRing) * kC;
-                const uint32_t v1 = ring_v_lo + ((vc + 1) % kRing) * kC;
+            // O_t (+)= P_t V of key tile kg over the pair: 4 k-steps of 16 keys, P from S buffer sb
+            auto issue_pv = [&](int t, uint32_t kg, uint32_t sb, bool accumulate) {
+                const uint32_t d = tmem + kTmemOBase + t * kDn;
+                const uint32_t pa = tmem + kTmemSBase + t * 128 + sb * kKeys;
+                const uint32_t v0 = ring_v_lo + (kg % kSlots) * kSlotU;
                 if (ptx::elect_one()) {
                     // 16 keys x 128 B = 2048 B = 128 units per k-step; P advances 8 columns per k-step
                     if (accumulate) ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa, v0);
@@ -437,10 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa + 8, v0 + 128);
                     ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa + 16, v0 + 256);
                     ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa + 24, v0 + 384);
-                    ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa + 32, v1);
-                    ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa + 40, v1 + 128);
-                    ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa + 48, v1 + 256);
-                    ptx::mma2_ts_lo<kHi, kIdPV, 1>(d, pa + 56, v1 + 384);
+                    ptx::mma_commit_pair(bar(bars->pv_done[t][sb]), kBoth);
                 }
                 __syncwarp();
             };
@@ -452,47 +501,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (x.n_max == 0) continue;
                 if (x.n[0]) ok = waitw(bar(bars->q_full[0]), qf0++ & 1);
                 if (ok && x.n[1]) ok = waitw(bar(bars->q_full[1]), qf1++ & 1);
-                if (!ok) break;
-                // key tile g = tg + j: K_g in ring chunks 5g + {0,1,2}, V_g in 5g + {3,4}.  The last MMA
-                // reading a key tile is group 1's when group 1 reads it (issued after group 0's).
-                ok = waitw(bar(bars->k_full[tg % kTileBars]), (tg / kTileBars) & 1);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                if (x.n[0] > 0) {
-                    issue_s(0, kTileChunks * tg);
-                    if (x.n[0] == 1) commit(bars->q_empty[0]);
+                // S of the unit's first two key tiles.  Every release (k_empty, v_empty) is committed
+                // after the last MMA reading the tile: group 1's when group 1 reads it (its MMAs are
+                // issued after group 0's), else group 0's.
+                for (int j = 0; j < 2 && j < x.n_max && ok; ++j) {
+                    ok = waitw(bar(bars->k_full[(tg + j) % kSlots]), ((tg + j) / kSlots) & 1);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    if (j < x.n[0]) {
+                        issue_s(0, tg + j, (gs0 + j) & 1);
+                        if (j == x.n[0] - 1) commit(bars->q_empty[0]);
+                    }
+                    if (j < x.n[1]) {
+                        issue_s(1, tg + j, (gs1 + j) & 1);
+                        if (j == x.n[1] - 1) commit(bars->q_empty[1]);
+                    }
+                    commit(bars->k_empty[(tg + j) % kSlots]);
                 }
-                if (x.n[1] > 0) {
-                    issue_s(1, kTileChunks * tg);
-                    if (x.n[1] == 1) commit(bars->q_empty[1]);
-                }
-                commit(bars->k_empty[tg % kTileBars]);
-                // Inside the unit the issuer waits for P-ready only: the helper has seen V_j and
-                // K_{j+1} land before its own arrival on the step's P-ready barriers.
+                // Per step: P V_t(j) once P_t(j) is ready (the helper has seen V_j and K_{j+2} land
+                // before its own arrival), then S_t(j + 2) into the buffer P V_t(j) reads.
                 for (int j = 0; j < x.n_max && ok; ++j) {
-                    const uint32_t g = tg + j, kc = kTileChunks * g, vc = kc + kKChunks, kn = kc + kTileChunks;
+                    const uint32_t kg = tg + j;
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
+                        const uint32_t g = (t ? gs1 : gs0) + j, sb = g & 1;  // the group's g-th tile
                         if (ok && j < x.n[t]) {
-                            uint32_t &pf = t ? pf1 : pf0;
-                            uint32_t &oe = t ? oe1 : oe0;
-                            ok = waitw(bar(bars->p_full[t]), pf++ & 1);
-                            if (ok && j == 0) ok = waitw(bar(bars->o_empty[t]), (oe++ & 1) ^ 1);
+                            ok = waitw(bar(bars->p_full[t][sb]), (g >> 1) & 1);
                             if (ok) {
                                 ptx::tc_fence_after();
-                                issue_pv(t, vc, j > 0);
+                                issue_pv(t, kg, sb, j > 0);
                                 if (j == x.n[t] - 1) commit(bars->o_full[t]);
-                                if (t == 1 || j >= x.n[1]) commit(bars->v_empty[g % kTileBars]);  // last P V_g
+                                if (t == 1 || j >= x.n[1]) commit(bars->v_empty[kg % kSlots]);
                             }
                         }
-                        if (ok && j + 1 < x.n[t]) {
-                            issue_s(t, kn);
-                            if (j + 2 == x.n[t]) commit(bars->q_empty[t]);  // last S_t of the unit
-                            if (t == 1 || j + 1 >= x.n[1]) commit(bars->k_empty[(g + 1) % kTileBars]);
+                        if (ok && j + 2 < x.n[t]) {
+                            issue_s(t, kg + 2, sb);
+                            if (j + 3 == x.n[t]) commit(bars->q_empty[t]);  // last S_t of the unit
+                            if (t == 1 || j + 2 >= x.n[1]) commit(bars->k_empty[(kg + 2) % kSlots]);
                         }
                     }
                 }
                 if (!ok) break;
+                gs0 += x.n[0];
+                gs1 += x.n[1];
                 tg += x.n_max;
             }
             // Drain: wait until every MMA issued here has completed (commit to the leader only).
@@ -507,12 +558,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wq = warp & 3;         // TMEM lane quarter this warp may access
         const int row = wq * 32 + lane;  // row within this CTA's 128 rows of the group
         const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_addr + kTmemS + t * kBN;
-        const uint32_t tO = tmem + lane_addr + kTmemO + t * kDn;
-        const uint32_t p_ready = lead_bar(bars->p_full[t]);
-        const uint32_t o_free = lead_bar(bars->o_empty[t]);
+        const uint32_t tS0 = tmem + lane_addr + kTmemSBase + t * 128;
+        const uint32_t tO = tmem + lane_addr + kTmemOBase + t * kDn;
         const float sl2 = p.scale_log2;
-        uint32_t sf = 0, of = 0, ss = 0;
+        uint32_t gt = 0, of = 0, ss = 0;
         bool ok = true;
         // One arrival per warp on the leader's barrier, after this warp's tensor-memory accesses.
         auto arrive_warp = [&](uint32_t lead_addr) {
@@ -541,39 +590,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int lim_row = kCausal ? min(i + x.off + 1, x.lk) : x.lk;  // keys [0, lim_row) visible
             float m_run = -INFINITY, l_run = 0.f;
-            for (int j = 0; j < n_t; ++j) {
-                ok = wait_pair_warp(bar(bars->s_full[t]), sf & 1, bars, peer_abort, p.status);
-                ++sf;
+            for (int j = 0; j < n_t; ++j, ++gt) {
+                const uint32_t sb = gt & 1;
+                ok = wait_pair_warp(bar(bars->s_full[t][sb]), (gt >> 1) & 1, bars, peer_abort, p.status);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                float s[kBN];
+                const uint32_t tS = tS0 + sb * kKeys;
+                float s[kKeys];
                 {
-                    uint32_t r0[64], r1[64];
-                    ptx::tmem_ld64(tS, r0);
-                    ptx::tmem_ld64(tS + 64, r1);
-                    ptx::tmem_wait_ld_dep64(r0);
-                    ptx::tmem_wait_ld_dep64(r1);
+                    uint32_t r[64];
+                    ptx::tmem_ld64(tS, r);
+                    ptx::tmem_wait_ld_dep64(r);
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        s[e] = __uint_as_float(r0[e]);
-                        s[64 + e] = __uint_as_float(r1[e]);
-                    }
+                    for (int e = 0; e < 64; ++e) s[e] = __uint_as_float(r[e]);
                 }
-                const int kv0 = j * kBN;
-                const bool tile_masked = (kv0 + kBN > x.lk) || (kCausal && kv0 + kBN - 1 > tile_q0 + x.off);
+                const int kv0 = j * kKeys;
+                const bool tile_masked = (kv0 + kKeys > x.lk) || (kCausal && kv0 + kKeys - 1 > tile_q0 + x.off);
                 float m_tile;
                 if (kPositiveScale) {
                     if (tile_masked) {
                         const int lim = lim_row - kv0;
 #pragma unroll
-                        for (int c = 0; c < kBN; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+                        for (int c = 0; c < kKeys; ++c) s[c] = c < lim ? s[c] : -INFINITY;
                     }
-                    m_tile = row_max(s) * sl2;
+                    m_tile = row_max64(s) * sl2;
                 } else {
-                    const int lim = tile_masked ? lim_row - kv0 : kBN;
+                    const int lim = tile_masked ? lim_row - kv0 : kKeys;
 #pragma unroll
-                    for (int c = 0; c < kBN; ++c) s[c] = c < lim ? s[c] * sl2 : -INFINITY;
-                    m_tile = row_max(s);
+                    for (int c = 0; c < kKeys; ++c) s[c] = c < lim ? s[c] * sl2 : -INFINITY;
+                    m_tile = row_max64(s);
                 }
                 // Lazy rescaling: keep the old reference max unless the new one is 2^8 larger.
                 float alpha = 1.f;
@@ -584,12 +629,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
                 const float2 sc2 = kPositiveScale ? make_float2(sl2, sl2) : make_float2(1.f, 1.f);
                 const float2 nm2 = make_float2(-m_use, -m_use);
-                uint32_t pk[64];
-                const float rowsum = exp_pack_sum<T>(s, sc2, nm2, pk);
-                ptx::tmem_st64(tS + kTmemPOff, pk);
-                // O_t holds P(j-1) V(j-1) already (the MMAs behind S_t(j) have completed);
-                // rescale it before P V(j) may start.
+                uint32_t pk[kKeys / 2];
+                const float rowsum = exp_pack_sum64<T>(s, sc2, nm2, pk);
+                ptx::tmem_st32(tS, pk);  // P over the S values just read
+                // The running max moved: once P V_t of the group's previous tile has completed
+                // (O_t holds it), rescale O_t before P V of this tile may start.  That barrier's
+                // next phase needs this group's next tile's P-ready, so it is never two phases
+                // ahead of the one waited for, also when most tiles skip this wait.
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    const uint32_t gp = gt - 1;
+                    ok = wait_pair_warp(bar(bars->pv_done[t][gp & 1]), (gp >> 1) & 1, bars, peer_abort, p.status);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
                     const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
                     for (int c = 0; c < kDn / 64; ++c) {
@@ -607,11 +658,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 ptx::tmem_wait_st();
-                arrive_warp(p_ready);
+                arrive_warp(lead_bar(bars->p_full[t][sb]));
                 l_run = l_run * alpha + rowsum;
             }
             if (!ok) break;
-            // Epilogue: O / l -> 16-bit, one 256-byte row per thread.
+            // Epilogue: O / l -> 16-bit, one 256-byte row per thread.  The next unit's first P V_t,
+            // which overwrites O_t, waits for P-ready of that unit: every warp of the group arrives
+            // on it only after this read.
             ok = wait_pair_warp(bar(bars->o_full[t]), of & 1, bars, peer_abort, p.status);
             ++of;
             if (!ok) break;
@@ -628,7 +681,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     w[e] = DType<T>::pack(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
                 if (row_valid) store_row_chunk(orow + c * 32, w, p.out_v8);
             }
-            arrive_warp(o_free);
         }
     }
 

@@ -29,16 +29,20 @@ def gpu():
     torch.cuda.synchronize()
 
 
-# Every test of this module runs on both attention kernels: the single-CTA kernel (256-row units)
-# and the CTA-pair kernel (512-row units on clusters of two SMs).  Padded K/V always runs the
-# single-CTA kernel.
+# Every test of this module runs on both attention kernels: the single-CTA kernel (256-row units,
+# 128-key tiles) and the CTA-pair kernel (512-row units on clusters of two SMs, 64-key tiles).
+# Padded K/V always runs the single-CTA kernel.
 @pytest.fixture(autouse=True, params=[1, 2], ids=["single", "pair"])
 def kernel(request):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     mla.set_kernel(request.param)
+    _kernel[0] = request.param
     yield request.param
     mla.set_kernel(-1)
+
+
+_kernel = [-1]  # the kernel the running test selected
 
 
 def problem(lens_q, lens_k, H, G, dtype=torch.bfloat16, std=1.0, seed=0, extra_tokens=0):
@@ -49,6 +53,16 @@ def problem(lens_q, lens_k, H, G, dtype=torch.bfloat16, std=1.0, seed=0, extra_t
             pad = torch.randn(extra_tokens, *x[key].shape[1:], device=DEV).to(dtype)
             x[key] = torch.cat([x[key], pad])
     return wl, x
+
+
+def run_single(x, H, G, scale, mask=mla.MLA_MASK_CAUSAL):
+    """The packed problem on the single-CTA kernel: the kernel padded K/V runs on, with the same key
+    tiles, so the two layouts must agree bit for bit."""
+    mla.set_kernel(1)
+    try:
+        return run(x, H, G, scale, mask).clone()
+    finally:
+        mla.set_kernel(_kernel[0])
 
 
 def run(x, H, G, scale, mask=mla.MLA_MASK_CAUSAL, out=None, stream=None):
@@ -360,12 +374,13 @@ def _to_padded(x, lens_k, max_seq, G, fill=9.0):
 def test_padded_kv_layout_matches_packed(case):
     lq, lk, max_seq, H, G, dtype = case
     _, x = problem(lq, lk, H, G, dtype=dtype, seed=501)
-    packed = run(x, H, G, 0.07).clone()
+    packed = run(x, H, G, 0.07).clone()  # on this test's kernel
     y = dict(x, **_to_padded(x, lk, max_seq, G))
-    padded = run(y, H, G, 0.07)
+    padded = run(y, H, G, 0.07).clone()
     torch.cuda.synchronize()
-    assert torch.equal(packed, padded)  # same keys, same tiles: bit-identical
+    assert torch.equal(run_single(x, H, G, 0.07), padded)  # same keys, same tiles: bit-identical
     check_against_oracle(x, padded, H, G, 0.07)
+    check_against_oracle(x, packed, H, G, 0.07)
     assert status() == 0
 
 
@@ -374,11 +389,10 @@ def test_padded_kv_padding_never_reaches_the_result(fill):
     # padding rows past Lk_b share key tiles with real keys; P = 0 there, and 0 * NaN would be NaN
     lq, lk, H, G = [40, 130, 3], [100, 130, 77], 4, 2
     _, x = problem(lq, lk, H, G, seed=503)
-    packed = run(x, H, G, 0.07).clone()
     y = dict(x, **_to_padded(x, lk, 200, G, fill=fill))
     padded = run(y, H, G, 0.07)
     torch.cuda.synchronize()
-    assert torch.equal(packed, padded)
+    assert torch.equal(run_single(x, H, G, 0.07), padded)
     assert status() == 0
 
 

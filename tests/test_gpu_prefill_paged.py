@@ -35,9 +35,15 @@ def problem(lq, lk, H, G, dtype=torch.bfloat16, seed=0):
 
 
 def packed(x, H, G, scale, mask):
+    """Packed K/V on the single-CTA kernel, the kernel paged K/V runs on (same key tiles): the paged
+    result must match it bit for bit."""
     out = torch.full((x["q"].shape[0], H, 128), 7.0, dtype=x["q"].dtype, device=DEV)
-    mla.mla_prefill(x["q"], x["q_rope"], x["k"], x["k_rope"], x["v"], x["q_seqlen"], x["kv_seqlen"], mask, H, G,
-                    scale, out)
+    mla.set_kernel(1)
+    try:
+        mla.mla_prefill(x["q"], x["q_rope"], x["k"], x["k_rope"], x["v"], x["q_seqlen"], x["kv_seqlen"], mask, H, G,
+                        scale, out)
+    finally:
+        mla.set_kernel(-1)
     return out
 
 

@@ -219,30 +219,47 @@ def test_planted_protocol_mistakes_are_caught(bug):
 # ---------------------------------------------------------------------------
 # The CTA-pair kernel (mla_prefill_pair_sm100.cuh)
 # ---------------------------------------------------------------------------
-# Two CTAs (leader 0, follower 1) each stream their half of every key tile through their own
-# ring of sixteen 8 KB chunks: key tile g occupies chunks 5g .. 5g + 4 (mod 16), K_g in the
-# first three, V_g in the last two.  Each CTA also holds its 128 rows of Q for groups 0 and 1.
+# Two CTAs (leader 0, follower 1) each stream their half of every 64-key tile through their own
+# ring of six tile slots (K_g and V_g of key tile g in slot g mod 6, with a full and an empty
+# barrier per slot for K and for V).  Each CTA also holds its 128 rows of Q for groups 0 and 1.
+# Per group t, tensor memory holds O_t and two S buffers: S_t of the group's g-th tile (counted
+# across units) goes to buffer g mod 2, and the softmax writes P_t(g) over the same buffer.
 #
 #   producer (each CTA)  per unit: Q_t for each group with key tiles: waits its own
-#                        q_empty(t), arms its own q_full(t), loads; per key tile:
-#                        K_g waits its own k_empty(g - 3), V_g its own v_empty(g - 3)
+#                        q_empty(t), arms its own q_full(t), loads; per key tile g:
+#                        K_g waits its own k_empty(g - 6), V_g its own v_empty(g - 6)
 #   relay (follower)     in the producer's order, waits for each of the follower's full
 #                        barriers and arrives on the leader's matching one
-#   helper t (leader)    one per group, for each step j < n_t of a unit: once S_t(j) is ready
-#                        (the leader's S-ready barrier; the MMA warp has then consumed the group's
-#                        previous P phase), waits the leader's v_full(j) and, if the group has a
-#                        next tile, k_full(j + 1) (two arrivals each: the leader's own load, the
-#                        relay), then arrives on P_t(j)
-#   MMA (leader)         per unit: waits q_full and k_full(first), issues S_0, S_1; per step:
-#                        waits P_t(j) only (three arrivals: each CTA's softmax and the helper),
-#                        P V_t(j), S_t(j + 1); every release (q_empty, k_empty, v_empty) and
-#                        S-ready arrives in both CTAs; each pair MMA reads both CTAs' halves
-#   softmax (each CTA)   group t: waits its own S_t(j), arrives on the leader's P_t(j)
-PAIR_RING = 16
+#   helper t (leader)    for the group's g-th tile (unit step j): waits S_t(g) (issued after
+#                        P V_t(g - 2), so the P-ready phase of tile g - 2 is complete and this
+#                        arrival cannot fall into it; it also keeps the helper within one phase
+#                        of the slots it checks next), then the leader's v_full(j) and, if the
+#                        group has a tile j + 2, k_full(j + 2), then arrives on P_t[g mod 2]
+#   MMA (leader)         per unit: waits q_full; S_t(0), S_t(1) (after k_full of tiles 0, 1);
+#                        per step j and group t: waits P_t[g mod 2] (three arrivals: each CTA's
+#                        softmax and the helper), issues P V_t(j), commits pv_done_t[g mod 2],
+#                        then S_t(j + 2)
+#                        into the buffer P_t(j) occupies (in-order completion: after P V_t(j)
+#                        has read it) and commits s_full_t[buffer]; releases (q/k/v_empty)
+#                        arrive in both CTAs.  The
+#                        unit's first P V_t overwrites O_t with no O-free barrier: its P-ready
+#                        phase needs every softmax warp of the group, and each has read its rows
+#                        of O_t in the previous unit's epilogue before it starts the next unit
+#   softmax (each CTA)   group t, tile g: waits its own s_full_t[g mod 2], reads S_t(g), writes
+#                        P_t(g) over it; when its running max moved (modelled at random) waits
+#                        pv_done_t[(g - 1) mod 2] and rescales O_t; arrives on the leader's
+#                        P_t[g mod 2]; after the unit's last tile waits o_full_t and reads O_t.
+#                        The S, P-ready and P V-done barriers come in pairs (tile parity): a
+#                        barrier's next phase then needs this group's own next-but-one tile, so
+#                        no role can fall two phases behind one it waits for, even where the
+#                        softmax waits for P V-done only now and then
+# Tensor-memory contents are tracked too: a write over data still to be read, or a read of the
+# wrong tile's data, is a protocol error.
+PAIR_SLOTS = 6
 
 
 def simulate_pair(units, seed, bug=None):
-    """units: [(n0, n1)] key tiles of group 0 / 1 per 512-row unit (max > 0)."""
+    """units: [(n0, n1)] 64-key tiles of group 0 / 1 per 512-row unit (max > 0)."""
     rnd = random.Random(seed)
     bars = {}
 
@@ -251,7 +268,7 @@ def simulate_pair(units, seed, bug=None):
 
     for cta in range(2):
         full_count = 2 if cta == 0 else 1
-        for i in range(TILE_SETS):
+        for i in range(PAIR_SLOTS):
             mk("k_full", cta, i, full_count)
             mk("v_full", cta, i, full_count)
             mk("k_empty", cta, i)
@@ -259,17 +276,39 @@ def simulate_pair(units, seed, bug=None):
         for t in range(2):
             mk("q_full", cta, t, full_count)
             mk("q_empty", cta, t)
-            mk("s_full", cta, t)
+            mk("o_full", cta, t)
+            for buf in range(2):
+                mk("s_full", cta, 2 * t + buf)
+                mk("pv_done", cta, 2 * t + buf)
     for t in range(2):
-        mk("p_full", 0, t, 3)
-    owner = {}     # (cta, ring slot | ("Q", t)) -> operand last loaded there
+        for buf in range(2):
+            mk("p_full", 0, 2 * t + buf, 3)
+    owner = {}     # (cta, ring slot part | ("Q", t)) -> operand last loaded there
     readers = {}   # operand -> MMAs issued and not yet completed
     landed = set()
     tma = []       # (cta, barrier, operand)
     mma_queue = []
+    sbuf = {}      # (cta, t, buffer) -> ("S", g) | ("P", g) | ("X", g): written, P over it, P read
+    otile = {}     # (cta, t) -> ("O", g) after P V(g), ("R", g) rescaled for g + 1, ("D",) drained
 
     def b(kind, cta, g):
-        return bars[kind, cta, g % TILE_SETS]
+        return bars[kind, cta, g % PAIR_SLOTS]
+
+    def s_full(cta, t, g):
+        if bug == "pair_one_s_full":
+            return bars["s_full", cta, 2 * t]
+        return bars["s_full", cta, 2 * t + g % 2]
+
+    def p_full(t, g):
+        if bug == "pair_one_p_full":
+            return bars["p_full", 0, 2 * t]
+        return bars["p_full", 0, 2 * t + g % 2]
+
+    def pv_done(cta, t, g):
+        return bars["pv_done", cta, 2 * t + g % 2]
+
+    def phase(g):
+        return g if bug == "pair_one_p_full" else g // 2
 
     def fill(cta, key, operand):
         prev = owner.get((cta, key))
@@ -280,7 +319,7 @@ def simulate_pair(units, seed, bug=None):
     def producer(cta):
         g = 0
         ql = [0, 0]
-        lag = 4 if bug == "pair_lag_4" else 3
+        lag = 7 if bug == "pair_lag_7" else PAIR_SLOTS
         for n in units:
             for t in range(2):
                 if n[t] == 0:
@@ -293,16 +332,14 @@ def simulate_pair(units, seed, bug=None):
                 ql[t] += 1
             for _ in range(max(n)):
                 if g >= lag:
-                    while not ready(b("k_empty", cta, g - lag), (g - lag) // TILE_SETS):
+                    while not ready(b("k_empty", cta, g - lag), (g - lag) // PAIR_SLOTS):
                         yield
-                for c in (0, 1, 2):
-                    fill(cta, (5 * g + c) % PAIR_RING, (cta, "K", g))
+                fill(cta, ("K", g % PAIR_SLOTS), (cta, "K", g))
                 tma.append((cta, b("k_full", cta, g), (cta, "K", g)))
                 if g >= lag and bug != "pair_no_v_slot_wait":
-                    while not ready(b("v_empty", cta, g - lag), (g - lag) // TILE_SETS):
+                    while not ready(b("v_empty", cta, g - lag), (g - lag) // PAIR_SLOTS):
                         yield
-                for c in (3, 4):
-                    fill(cta, (5 * g + c) % PAIR_RING, (cta, "V", g))
+                fill(cta, ("V", g % PAIR_SLOTS), (cta, "V", g))
                 tma.append((cta, b("v_full", cta, g), (cta, "V", g)))
                 g += 1
                 yield
@@ -321,7 +358,7 @@ def simulate_pair(units, seed, bug=None):
                     bars["q_full", 0, t].arrive()
             for _ in range(max(n)):
                 for kind in ("k_full", "v_full"):
-                    while not ready(b(kind, 1, g), g // TILE_SETS):
+                    while not ready(b(kind, 1, g), g // PAIR_SLOTS):
                         yield
                     if not (bug == "pair_relay_skips_v" and kind == "v_full"):
                         b(kind, 0, g).arrive()
@@ -329,82 +366,128 @@ def simulate_pair(units, seed, bug=None):
                 yield
 
     def helper(t):
-        tg, sf = 0, 0
+        tg, gt = 0, 0
         for n in units:
             for j in range(n[t]):
-                g = tg + j
+                kg = tg + j
                 if bug != "pair_helper_runs_ahead":
-                    while not ready(bars["s_full", 0, t], sf):
+                    while not ready(s_full(0, t, gt), gt // 2):
                         yield
-                sf += 1
-                while not ready(b("v_full", 0, g), g // TILE_SETS):
+                while not ready(b("v_full", 0, kg), kg // PAIR_SLOTS):
                     yield
-                if j + 1 < n[t] and bug != "pair_helper_skips_k":
-                    while not ready(b("k_full", 0, g + 1), (g + 1) // TILE_SETS):
+                if j + 2 < n[t] and bug != "pair_helper_skips_k":
+                    while not ready(b("k_full", 0, kg + 2), (kg + 2) // PAIR_SLOTS):
                         yield
-                bars["p_full", 0, t].arrive()
+                p_full(t, gt).arrive()
+                gt += 1
                 yield
             tg += max(n)
 
-    def issue(*operands):
+    def issue(effect, *operands):
         for op in operands:
             if op not in landed:
                 raise ProtocolError("pair MMA reads %s before it landed" % (op,))
             readers[op] = readers.get(op, 0) + 1
-        mma_queue.append(("mma", operands))
+        mma_queue.append(("mma", (effect, operands)))
 
     def commit_both(kind, idx):
         mma_queue.append(("commit", [bars[kind, 0, idx], bars[kind, 1, idx]]))
 
+    def mma_effect(effect):
+        kind, t, g, first = effect
+        for cta in range(2):
+            key = (cta, t, g % 2)
+            if kind == "S":
+                prev = sbuf.get(key)
+                if prev is not None and prev != ("X", g - 2):
+                    raise ProtocolError("S_%d(%d) overwrites %s in buffer %d" % (t, g, prev, g % 2))
+                sbuf[key] = ("S", g)
+            else:
+                if sbuf.get(key) != ("P", g):
+                    raise ProtocolError("P V_%d(%d) reads %s" % (t, g, sbuf.get(key)))
+                sbuf[key] = ("X", g)
+                o = otile.get((cta, t))
+                want = [None, ("D",)] if first else [("O", g - 1), ("R", g - 1)]
+                if o not in want:
+                    raise ProtocolError("P V_%d(%d) on O_%d in state %s" % (t, g, t, o))
+                otile[(cta, t)] = ("O", g)
+
     def mma():
-        tg, pf, qf, qn = 0, [0, 0], [0, 0], [0, 0]
+        tg, qf, qn, gs = 0, [0, 0], [0, 0], [0, 0]
+        ahead = 3 if bug == "pair_s_lookahead_3" else 2
         for n in units:
             for t in range(2):
                 if n[t]:
                     while not ready(bars["q_full", 0, t], qf[t]):
                         yield
                     qf[t] += 1
-            while not ready(b("k_full", 0, tg), tg // TILE_SETS):
-                yield
-            for t in range(2):
-                if n[t] > 0:
-                    issue((0, "Q", t, qn[t]), (1, "Q", t, qn[t]), (0, "K", tg), (1, "K", tg))
-                    commit_both("s_full", t)
-                    if n[t] == 1:
-                        commit_both("q_empty", t)
-            commit_both("k_empty", tg % TILE_SETS)
+
+            def issue_s(t, j):
+                issue(("S", t, gs[t] + j, False), (0, "Q", t, qn[t]), (1, "Q", t, qn[t]), (0, "K", tg + j),
+                      (1, "K", tg + j))
+                mma_queue.append(("commit", [s_full(0, t, gs[t] + j), s_full(1, t, gs[t] + j)]))
+                if j == n[t] - 1:
+                    commit_both("q_empty", t)
+
+            for j0 in range(min(ahead, max(n))):
+                while not ready(b("k_full", 0, tg + j0), (tg + j0) // PAIR_SLOTS):
+                    yield
+                for t in range(2):
+                    if j0 < n[t]:
+                        issue_s(t, j0)
+                commit_both("k_empty", (tg + j0) % PAIR_SLOTS)
             for j in range(max(n)):
                 g = tg + j
                 for t in range(2):
                     if j < n[t]:
-                        while not ready(bars["p_full", 0, t], pf[t]):
+                        while not ready(p_full(t, gs[t] + j), phase(gs[t] + j)):
                             yield
-                        pf[t] += 1
-                        issue((0, "V", g), (1, "V", g))
+                        issue(("PV", t, gs[t] + j, j == 0), (0, "V", g), (1, "V", g))
+                        mma_queue.append(("commit", [pv_done(0, t, gs[t] + j), pv_done(1, t, gs[t] + j)]))
+                        if j == n[t] - 1:
+                            commit_both("o_full", t)
                         if t == 1 or j >= n[1]:
-                            commit_both("v_empty", g % TILE_SETS)
-                    if j + 1 < n[t]:
-                        issue((0, "Q", t, qn[t]), (1, "Q", t, qn[t]), (0, "K", g + 1), (1, "K", g + 1))
-                        commit_both("s_full", t)
-                        if j + 2 == n[t]:
-                            commit_both("q_empty", t)
-                        if t == 1 or j + 1 >= n[1]:
-                            commit_both("k_empty", (g + 1) % TILE_SETS)
+                            commit_both("v_empty", g % PAIR_SLOTS)
+                    if j + ahead < n[t]:
+                        issue_s(t, j + ahead)
+                        if t == 1 or j + ahead >= n[1]:
+                            commit_both("k_empty", (g + ahead) % PAIR_SLOTS)
                     yield
             for t in range(2):
                 if n[t]:
                     qn[t] += 1
+                gs[t] += n[t]
             tg += max(n)
 
     def softmax(cta, t):
-        sf = 0
+        gt, of = 0, 0
         for n in units:
-            for _ in range(n[t]):
-                while not ready(bars["s_full", cta, t], sf):
+            for j in range(n[t]):
+                while not ready(s_full(cta, t, gt), gt // 2 if bug != "pair_one_s_full" else gt):
                     yield
-                sf += 1
+                key = (cta, t, (gt + (bug == "pair_softmax_other_buffer")) % 2)
+                if sbuf.get(key) != ("S", gt):
+                    raise ProtocolError("softmax %d reads %s for S(%d)" % (t, sbuf.get(key), gt))
                 yield
-                bars["p_full", 0, t].arrive()
+                sbuf[key] = ("P", gt)
+                if j > 0 and rnd.random() < 0.3:  # the running max moved: rescale O_t
+                    if bug != "pair_softmax_no_pv_wait":
+                        while not ready(pv_done(cta, t, gt - 1), (gt - 1) // 2):
+                            yield
+                    o = otile.get((cta, t))
+                    if o != ("O", gt - 1):
+                        raise ProtocolError("rescale of O_%d(%d) sees %s" % (t, gt, o))
+                    otile[(cta, t)] = ("R", gt - 1)
+                p_full(t, gt).arrive()
+                gt += 1
+                yield
+            if n[t]:
+                while not ready(bars["o_full", cta, t], of):
+                    yield
+                of += 1
+                if otile.get((cta, t)) != ("O", gt - 1):
+                    raise ProtocolError("epilogue of O_%d sees %s" % (t, otile.get((cta, t))))
+                otile[(cta, t)] = ("D",)
 
     roles = [producer(0), producer(1), relay(), helper(0), helper(1), mma()] + \
         [softmax(c, t) for c in range(2) for t in range(2)]
@@ -430,7 +513,9 @@ def simulate_pair(units, seed, bug=None):
         else:
             op, x = mma_queue.pop(0)
             if op == "mma":
-                for operand in x:
+                effect, operands = x
+                mma_effect(effect)
+                for operand in operands:
                     readers[operand] -= 1
             else:
                 for bar in x:
@@ -444,11 +529,13 @@ def test_pair_protocol_holds_under_random_schedules():
         simulate_pair(random_units(rng), seed=trial)
 
 
-@pytest.mark.parametrize("bug", ["pair_lag_4", "pair_no_v_slot_wait", "pair_no_q_empty_wait", "pair_no_q_relay",
-                                 "pair_relay_skips_v", "pair_helper_skips_k", "pair_helper_runs_ahead"])
+@pytest.mark.parametrize("bug", ["pair_lag_7", "pair_no_v_slot_wait", "pair_no_q_empty_wait", "pair_no_q_relay",
+                                 "pair_relay_skips_v", "pair_helper_skips_k", "pair_helper_runs_ahead",
+                                 "pair_one_p_full",
+                                 "pair_softmax_no_pv_wait", "pair_one_s_full", "pair_s_lookahead_3",
+                                 "pair_softmax_other_buffer"])
 def test_pair_planted_protocol_mistakes_are_caught(bug):
     rng = random.Random(11)
     with pytest.raises(ProtocolError):
         for trial in range(300):
             simulate_pair(random_units(rng), seed=trial, bug=bug)
-
