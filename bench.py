@@ -435,10 +435,14 @@ def bench_prolog(args):
         mla.mla_prolog(*[inp[k] for k in order], H, qo, kvo, cqo, stream=stream)
 
     flops = 2.0 * t * (h * r + r * H * d + h * d)
+    q_flops = 2.0 * t * r * H * d  # the q projection (the fused kernel's work)
     norm_bytes = t * H * d * (4 + 2) + 2 * t * R * 2  # fp32 rows in, bf16 rows out, cos / sin
+    q_bytes = 2 * (t * r + r * H * d + t * H * d + 2 * t * R)  # c^Q, wq_b, q, cos / sin once
+    mla.set_prolog_path(args.prolog_path)
     for _ in range(args.warmup):
         call(x, q, kv, cq)
     torch.cuda.synchronize()
+    fused = mla.prolog_last_fused()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     k_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -518,12 +522,19 @@ def bench_prolog(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "prolog", "tokens": t, "hidden": h, "q_lora_rank": r, "num_heads": H, "head_dim": d,
                    "rope_dim": R, "weights": "random init", "l2": "inputs and outputs %.2f GB > 126 MB L2" % (
-                       (in_bytes + q.numel() * 2) / 1e9)},
-        "roofline": {"bound": "hbm", "achieved": norm_bytes / (kms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
-                     "frac": norm_bytes / (kms * 1e-3) / 1e9 / hbm, "traffic": None, "peak_source": peak_src,
-                     "kernel": "rms_norm_rope_kernel (q rows)", "kernel_ms": kms,
-                     "algorithmic_bytes_per_launch": norm_bytes,
-                     "step_tensor_frac": value / world / peak},
+                       (in_bytes + q.numel() * 2) / 1e9),
+                   "q_path": "fused tcgen05 q kernel" if fused else "library GEMM + row kernel"},
+        "roofline": ({"bound": "tensor", "achieved": q_flops / (kms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                      "frac": q_flops / (kms * 1e-3) / 1e12 / peak, "traffic": None, "peak_source": peak_src,
+                      "kernel": "mla_prolog_q_kernel (q projection + per-head RmsNorm + RoPE)", "kernel_ms": kms,
+                      "algorithmic_flops_per_launch": q_flops, "algorithmic_bytes_per_launch": q_bytes,
+                      "hbm_achieved_gbs": q_bytes / (kms * 1e-3) / 1e9, "step_tensor_frac": value / world / peak}
+                     if fused else
+                     {"bound": "hbm", "achieved": norm_bytes / (kms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                      "frac": norm_bytes / (kms * 1e-3) / 1e9 / hbm, "traffic": None, "peak_source": peak_src,
+                      "kernel": "rms_norm_rope_kernel (q rows)", "kernel_ms": kms,
+                      "algorithmic_bytes_per_launch": norm_bytes,
+                      "step_tensor_frac": value / world / peak}),
         "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": smi.summary(),
     }
     if rank == 0:
@@ -618,6 +629,8 @@ def main():
     ap.add_argument("--other-configs", default="varlen_gqa,chunked,uniform",
                     help="prefill on the default workload: more workloads timed in the same run and reported "
                          "under other_configs (comma-separated; empty for none)")
+    ap.add_argument("--prolog-path", type=int, default=-1, choices=[-1, 0],
+                    help="prolog: q projection -1 fused kernel where the sizes allow (default), 0 library GEMM")
     ap.add_argument("--kernel", type=int, default=-1, choices=[-1, 1, 2],
                     help="attention kernel: -1 automatic (default), 1 single-CTA, 2 CTA pair")
     ap.add_argument("--heads", type=int, default=0,

@@ -335,17 +335,32 @@ int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, const mla_t
  * 16-byte aligned bases; vectors are contiguous.  Outputs must not overlap each
  * other or any input.
  *
- * The projections run as bf16 GEMMs with fp32 results (cuBLAS); nothing is
- * rounded before the norms except c^Q, which is rounded to bf16 once before
- * the q projection.  Scratch (fp32 projections of up to 4096 tokens at a time)
- * lives in the per-GPU workspace shared with mla_prefill: order calls on one
- * stream.  Argument errors return before any launch.  Returns MLA_OK or an
- * mla_status error code.
+ * The q projection c^Q wq_b runs in this library's tcgen05 kernel with the
+ * per-head RmsNorm and RoPE as its epilogue (the head's d channels of 256
+ * tokens accumulate in fp32 in tensor memory and are written once, as bf16)
+ * when d is a multiple of 128 up to 512, r a multiple of 64 and R even -- the
+ * page's sizes among them; otherwise it runs as a library GEMM (fp32 result)
+ * followed by a row kernel.  x wq_a and x wkv are library GEMMs (cuBLAS, fp32
+ * results) followed by the row kernel.  Nothing is rounded before the norms
+ * except c^Q, which is rounded to bf16 once before the q projection.  Scratch
+ * (fp32 projections of up to 4096 tokens at a time) lives in the per-GPU
+ * workspace shared with mla_prefill: order calls on one stream.  Argument
+ * errors return before any launch.  Returns MLA_OK or an mla_status error code.
  */
 int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, const mla_tensor *wq_b, const mla_tensor *wkv,
                const mla_tensor *rope_cos, const mla_tensor *rope_sin, const mla_tensor *gamma_cq,
                const mla_tensor *gamma_ckv, int num_heads, float eps, mla_tensor *q_out, mla_tensor *kv_out,
                mla_tensor *cq_out, mla_stream_t stream);
+
+/* How this host thread's mla_prolog calls run the q projection: -1 (default)
+ * the fused tcgen05 kernel wherever the sizes allow it, 0 always the library
+ * GEMM followed by the row kernel (for comparison).  Returns MLA_OK, or
+ * MLA_ERR_UNSUPPORTED for any other value. */
+int mla_prolog_set_path(int path);
+
+/* 1 if the last mla_prolog call of this host thread ran the fused q kernel,
+ * else 0. */
+int mla_prolog_last_fused(void);
 
 /* A static, human-readable name for a status code (never NULL). */
 const char *mla_status_string(int status);

@@ -87,6 +87,10 @@ def load_library(path=None):
     lib.mla_prefill_last_launches.restype = ctypes.c_int
     lib.mla_prefill_last_kernel.argtypes = []
     lib.mla_prefill_last_kernel.restype = ctypes.c_int
+    lib.mla_prolog_set_path.argtypes = [ctypes.c_int]
+    lib.mla_prolog_set_path.restype = ctypes.c_int
+    lib.mla_prolog_last_fused.argtypes = []
+    lib.mla_prolog_last_fused.restype = ctypes.c_int
     lib.mla_prefill_set_kernel.argtypes = [ctypes.c_int]
     lib.mla_prefill_set_kernel.restype = ctypes.c_int
     lib.mla_prefill_set_split_tiles.argtypes = [ctypes.c_int]
@@ -274,6 +278,19 @@ def set_kernel(kernel):
     rc = load_library().mla_prefill_set_kernel(int(kernel))
     if rc != 0:
         raise MlaError(rc, "mla_prefill_set_kernel")
+
+
+def set_prolog_path(path):
+    """q projection of later mla_prolog calls on this thread: -1 the fused tcgen05 kernel where the
+    sizes allow it (default), 0 the library GEMM + row kernel."""
+    rc = load_library().mla_prolog_set_path(int(path))
+    if rc != 0:
+        raise MlaError(rc, "mla_prolog_set_path")
+
+
+def prolog_last_fused():
+    """True if the last mla_prolog call of this thread ran the fused q kernel."""
+    return bool(load_library().mla_prolog_last_fused())
 
 
 def set_profile_events(start=None, stop=None):

@@ -16,6 +16,7 @@
 #include "mla_prefill_sm100.cuh"
 #include "paged_cache_load.cuh"
 #include "prolog_norm_rope.cuh"
+#include "prolog_q_sm100.cuh"
 
 namespace {
 
@@ -30,12 +31,16 @@ struct DeviceState {
     size_t ws_bytes = 0;
     bool attr_set[32] = {};  // dynamic shared memory opt-in done, per kernel instantiation
     int pair_clusters = 0;   // co-resident clusters of two CTAs of the pair kernel (0: not yet queried)
+    bool prolog_attr = false;  // dynamic shared memory opt-in of the fused q-projection kernel
+    int prolog_clusters = 0;   // its co-resident clusters (0: not yet queried)
 };
 
 std::mutex g_mu;
 thread_local cudaEvent_t t_prof_start = nullptr, t_prof_stop = nullptr;
 thread_local int t_split_tiles = -1;  // split-KV chunk in key tiles: -1 automatic, 0 off
 thread_local int t_kernel = -1;       // attention kernel: -1 automatic, 1 single-CTA, 2 CTA pair
+thread_local int t_prolog_path = -1;  // MLA Prolog q path: -1 automatic (fused where the sizes allow), 0 library
+thread_local int t_prolog_fused = 0;  // the last mla_prolog call of this thread ran the fused q kernel
 thread_local int t_last_launches = 0;  // kernels the last prefill call of this thread enqueued
 thread_local int t_last_kernel = 0;    // attention kernel of that call: 1 single-CTA, 2 CTA pair
 DeviceState g_dev[kMaxDevices];
@@ -1185,6 +1190,55 @@ int gemm_rowmajor(cublasHandle_t h, int64_t M, int64_t N, int64_t K, const void 
     return s == CUBLAS_STATUS_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// 2-D map over a bf16 matrix {cols, rows} (row stride row_bytes) with a {64, box_rows} box and
+// 128-byte swizzle.
+int encode_map2d(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, int64_t row_bytes, int box_rows) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_UNSUPPORTED;
+}
+
+// The fused q projection + per-head RmsNorm + RoPE (prolog_q_sm100.cuh): clusters of two CTAs, one
+// per SM, static tiles of 256 tokens x one head.
+int launch_prolog_q(DeviceState *ds, cudaStream_t stream, const CUtensorMap &tm_a, const CUtensorMap &tm_b,
+                    const mla::prolog::QParams &qp) {
+    auto kern = mla::prolog::mla_prolog_q_kernel;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(mla::prolog::kThreads);
+    cfg.dynamicSmemBytes = mla::prolog::kSmemAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (!ds->prolog_attr) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::prolog::kSmemAlloc) !=
+            cudaSuccess)
+            return MLA_ERR_CUDA;
+        ds->prolog_attr = true;
+    }
+    if (ds->prolog_clusters <= 0) {
+        int n = 0;
+        cfg.gridDim = dim3(2);
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return MLA_ERR_CUDA;
+        ds->prolog_clusters = n;
+    }
+    const int64_t tiles = static_cast<int64_t>((qp.tokens + mla::prolog::kTileTokens - 1) / mla::prolog::kTileTokens) *
+                          qp.heads;
+    const int64_t clusters = tiles < ds->prolog_clusters ? tiles : ds->prolog_clusters;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+    if (cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, qp) != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_OK;
+}
+
 int launch_norm(const mla::NormParams &np, int sm_count, cudaStream_t stream) {
     const long long rows = np.job[0].rows + (np.njobs > 1 ? np.job[1].rows : 0);
     if (rows == 0) return MLA_OK;
@@ -1236,10 +1290,15 @@ extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, con
     }
     if (t == 0) return MLA_OK;
 
-    // scratch per slab: [S, r + d] fp32 (x wq_a | x wkv), [S, H d] fp32 (c^Q wq_b), [S, r] bf16 c^Q
+    // The q projection runs fused with its norm and rotation (prolog_q_sm100.cuh) where the sizes fit
+    // the kernel's tiles: head_dim a multiple of 128 up to 512 (the accumulator of a head row in
+    // tensor memory), q_lora_rank a multiple of 64 (its k-stages), an even rope_dim.
+    const bool fused = t_prolog_path != 0 && d % 128 == 0 && d <= 512 && r % 64 == 0 && R % 2 == 0;
+    // scratch per slab: [S, r + d] fp32 (x wq_a | x wkv), [S, H d] fp32 (c^Q wq_b; library path
+    // only), [S, r] bf16 c^Q
     const int64_t slab = t < kPrologSlab ? t : kPrologSlab;
     const size_t pre_bytes = align_up(static_cast<size_t>(slab * (r + d)) * 4, 256);
-    const size_t q_bytes = align_up(static_cast<size_t>(slab * H * d) * 4, 256);
+    const size_t q_bytes = fused ? 0 : align_up(static_cast<size_t>(slab * H * d) * 4, 256);
     const size_t cq_bytes = cq_out ? 0 : align_up(static_cast<size_t>(slab * r) * 2, 256);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
@@ -1259,6 +1318,12 @@ extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, con
     const auto bf = [](const void *p, int64_t elems) {
         return reinterpret_cast<__nv_bfloat16 *>(const_cast<uint8_t *>(static_cast<const uint8_t *>(p)) + elems * 2);
     };
+    CUtensorMap tm_b;
+    if (fused) {
+        if ((rc = ensure_encode()) != MLA_OK) return rc;
+        if ((rc = encode_map2d(&tm_b, wb.data, H * d, r, wb.ld * 2, 64)) != MLA_OK) return rc;
+    }
+    t_prolog_fused = fused ? 1 : 0;
 
     for (int64_t s0 = 0; s0 < t; s0 += slab) {
         const int64_t S = t - s0 < slab ? t - s0 : slab;
@@ -1278,6 +1343,33 @@ extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, con
                                  bf(sn.data, s0 * sn.ld), cs.ld, sn.ld, static_cast<int>(d), static_cast<int>(R), 1,
                                  S};
         if ((rc = launch_norm(np, ds->sm_count, stream)) != MLA_OK) return rc;
+        if (fused) {
+            // c^Q wq_b with the per-head RmsNorm and rope as the epilogue, straight into q_out
+            CUtensorMap tm_a;
+            if ((rc = encode_map2d(&tm_a, cq, r, S, cq_ld * 2, 128)) != MLA_OK) return rc;
+            mla::prolog::QParams qp{};
+            qp.out = bf(qo.data, s0 * qo.st_tok);
+            qp.out_tok = qo.st_tok;
+            qp.out_head = qo.st_head;
+            qp.cos = bf(cs.data, s0 * cs.ld);
+            qp.sin = bf(sn.data, s0 * sn.ld);
+            qp.cos_tok = cs.ld;
+            qp.sin_tok = sn.ld;
+            qp.tokens = static_cast<int>(S);
+            qp.heads = static_cast<int>(H);
+            qp.d = static_cast<int>(d);
+            qp.nc = d % 256 == 0 ? 256 : 128;
+            qp.rope = static_cast<int>(R);
+            qp.k_stages = static_cast<int>(r / 64);
+            qp.eps = eps;
+            qp.out_v8 = (reinterpret_cast<uintptr_t>(qp.out) % 32 == 0 && qo.st_tok % 16 == 0 && qo.st_head % 16 == 0)
+                            ? 1 : 0;
+            qp.status = ds->status;
+            if (t_prof_start && cudaEventRecord(t_prof_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
+            if ((rc = launch_prolog_q(ds, stream, tm_a, tm_b, qp)) != MLA_OK) return rc;
+            if (t_prof_stop && cudaEventRecord(t_prof_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
+            continue;
+        }
         // c^Q wq_b -> qpre [S, H d]; per-head RmsNorm (weight 1) and rope into q_out
         if ((rc = gemm_rowmajor(bl, S, H * d, r, cq, cq_ld, wb.data, wb.ld, qpre, H * d)) != MLA_OK) return rc;
         mla::NormParams nq{};
@@ -1292,3 +1384,11 @@ extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, con
     }
     return MLA_OK;
 }
+
+extern "C" int mla_prolog_set_path(int path) {
+    if (path != -1 && path != 0) return MLA_ERR_UNSUPPORTED;
+    t_prolog_path = path;
+    return MLA_OK;
+}
+
+extern "C" int mla_prolog_last_fused(void) { return t_prolog_fused; }

@@ -1,0 +1,332 @@
+// q projection of the MLA Prolog with its per-head RmsNorm and RoPE as the GEMM's epilogue (sm_100a,
+// clusters of two CTAs).  The "MlaProlog" page of cann-recipes-infer (计算公式 section) defines, for
+// each token row c of c^Q [t, r] and head h of wq_b [r, H*d]:
+//   v        = c wq_b[:, h*d : (h+1)*d]                    (d channels, fp32 accumulation)
+//   q[h]     = v / sqrt(mean(v^2) + eps)                   (RmsNorm, weight 1)
+//   q[h, d-R+2i], q[h, d-R+2i+1] = the interleaved rotation of that pair by the token's cos / sin rows
+//   rope_cos / rope_sin [t, R]:  y[2i] = v[2i] cos[2i] - v[2i+1] sin[2i],  y[2i+1] = v[2i+1] cos[2i+1] + v[2i] sin[2i+1]
+// and q is written as bf16.  The norm needs the whole head row, so a tile is 256 tokens x one head:
+// each CTA of the pair holds 128 token rows x d fp32 accumulators in its tensor memory (d <= 512
+// columns), and the row never leaves the SM in fp32.
+//
+// Operands: A = c^Q rows (K-major: r contiguous), B = wq_b (MN-major: the head's d columns
+// contiguous).  The MMAs are tcgen05 cta_group::2 with M = 256 (128 rows in each CTA) and N = nc
+// (256 when d is a multiple of 256, else 128): B is split along N, so for N-chunk c each CTA loads
+// its nc/2 columns c*nc + rank*nc/2 + [0, nc/2).  A k-stage is 64 channels of r: per CTA 16 KB of A
+// (128 rows x 128 B) and d/128 blocks of 8 KB of B (64 rows of r x 64 columns, 128-byte swizzled);
+// four stages in flight.
+//
+//   leader   warp 0: TMA loads of its A rows and B halves; warp 1: MMA issuer for the pair
+//   follower warp 0: TMA loads of its halves; warp 1: relay of its full barriers to the leader's
+//   both     warps 4-11: epilogue, two warps per tensor-memory lane quarter, each one half of the
+//            head's d channels of 32 rows: sum of squares over its half, the two halves added
+//            through shared memory (an mbarrier per lane quarter), then scale, rotate, convert and
+//            store its half
+// Tiles are static (tile = cluster + i * clusters, head-major so that concurrent clusters share a
+// head's wq_b columns in L2).  The accumulator fills tensor memory: the next tile's MMAs wait for
+// the epilogue (an acc-empty barrier), while the producers already load its first stages.
+// Every wait is bounded; a timeout sets the status word and aborts both CTAs.
+#pragma once
+
+#include "mla_prefill_sm100.cuh"
+
+namespace mla {
+namespace prolog {
+
+constexpr int kThreads = 384;
+constexpr int kTileTokens = 256;   // rows of one pair MMA (128 per CTA)
+constexpr int kStageK = 64;        // channels of r per stage (one 128-byte swizzle row of A)
+constexpr int kStages = 4;
+constexpr int kABytes = 128 * kStageK * 2;  // 16 KB: this CTA's 128 rows of the stage
+constexpr int kBBlock = 64 * kStageK * 2;   // 8 KB: 64 columns of wq_b x the stage's 64 rows
+constexpr int kMaxBBlocks = 4;              // d <= 512: d / 128 blocks per CTA and stage
+constexpr int kStageBytes = kABytes + kMaxBBlocks * kBBlock;
+constexpr int kSmemStages = 0;
+constexpr int kSmemBar = kSmemStages + kStages * kStageBytes;
+constexpr int kSmemXss = kSmemBar + 256;      // per-row partial sums of squares, one per half
+constexpr int kSmemBytes = kSmemXss + 2 * 128 * 4;
+constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
+static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
+constexpr int kEpiWarps = 8;
+constexpr int kAccEmptyArrivals = 2 * kEpiWarps;  // every epilogue warp of both CTAs
+constexpr uint64_t kWaitLimitNs = 200000000ull;   // 200 ms
+
+struct QParams {
+    __nv_bfloat16 *out;          // q_out rows: token * out_tok + head * out_head
+    long long out_tok, out_head;
+    const __nv_bfloat16 *cos, *sin;  // [tokens, R] with row strides cos_tok / sin_tok
+    long long cos_tok, sin_tok;
+    int tokens;      // rows of this launch
+    int heads;       // H
+    int d;           // head_dim: a multiple of 128, <= 512
+    int nc;          // MMA N per chunk: 256 or 128
+    int rope;        // R (even, <= d)
+    int k_stages;    // r / 64
+    float eps;
+    int out_v8;      // output rows allow 32-byte stores
+    int *status;
+};
+
+struct Bars {
+    uint64_t full[kStages], empty[kStages];
+    uint64_t acc_full, acc_empty;
+    uint64_t xready[4];  // per lane quarter: both halves' sums of squares are in shared memory
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block too large");
+
+// Bounded wait on a phase; on timeout records the status, raises both CTAs' abort flags.
+__device__ __forceinline__ bool qwait(uint32_t bar, uint32_t parity, Bars *bars, uint32_t peer_abort, int *status) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*reinterpret_cast<volatile int *>(&bars->abort)) return false;
+            if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+                *reinterpret_cast<volatile int *>(&bars->abort) = 1;
+                ptx::st_shared_cluster_u32(peer_abort, 1u);
+                atomicCAS(status, 0, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool qwait_warp(uint32_t bar, uint32_t parity, Bars *bars, uint32_t peer_abort,
+                                           int *status) {
+    const bool ok = qwait(bar, parity, bars, peer_abort, status);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void qwait_landed(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, parity))
+        if (ptx::globaltimer_ns() - t0 > 100000000ull) return;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    mla_prolog_q_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                        const QParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars *bars = reinterpret_cast<Bars *>(smem + kSmemBar);
+    float *xss = reinterpret_cast<float *>(smem + kSmemXss);
+    const uint32_t sStages = ptx::smem_addr(smem + kSmemStages);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t cta = ptx::cluster_ctarank();
+    const bool leader = cta == 0;
+    auto bar = [&](uint64_t &b) { return ptx::smem_addr(&b); };
+    auto lead_bar = [&](uint64_t &b) { return ptx::mapa_shared(ptx::smem_addr(&b), 0); };
+    const uint32_t peer_abort = ptx::mapa_shared(ptx::smem_addr(&bars->abort), cta ^ 1u);
+
+    if (threadIdx.x == 32) {
+        ptx::tma_prefetch_desc(&tm_a);
+        ptx::tma_prefetch_desc(&tm_b);
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(bar(bars->full[s]), leader ? 2 : 1);
+            ptx::mbar_init(bar(bars->empty[s]), 1);
+        }
+        ptx::mbar_init(bar(bars->acc_full), 1);
+        ptx::mbar_init(bar(bars->acc_empty), kAccEmptyArrivals);
+        for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(bars->xready[q]), 2);
+        bars->abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(ptx::smem_addr(&bars->tmem_base), kTmemCols);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync_all();
+    ptx::tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    const int n_tblocks = (p.tokens + kTileTokens - 1) / kTileTokens;
+    const int n_tiles = n_tblocks * p.heads;
+    const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+    const int b_blocks = p.d / 128;        // this CTA's 8 KB B blocks per stage
+    const int chunk_blocks = p.nc / 128;   // of which per N-chunk
+    const int chunks = p.d / p.nc;
+    const uint32_t stage_tx = kABytes + b_blocks * kBBlock;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ TMA producer (both CTAs)
+            const uint64_t pol_a = ptx::policy_evict_last();  // c^Q rows: read by every head
+            const uint64_t pol_b = ptx::policy_evict_last();  // wq_b columns: read by every token block
+            uint32_t it = 0;  // stages issued
+            bool ok = true;
+            for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters) {
+                const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
+                const int row0 = tb * kTileTokens + static_cast<int>(cta) * 128;
+                for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+                    const uint32_t s = it % kStages;
+                    if (it >= kStages && !(ok = qwait(bar(bars->empty[s]), ((it / kStages) & 1) ^ 1, bars, peer_abort,
+                                                      p.status)))
+                        break;
+                    const uint32_t fb = bar(bars->full[s]);
+                    const uint32_t dst = sStages + s * kStageBytes;
+                    ptx::mbar_arrive_expect_tx(fb, stage_tx);
+                    ptx::tma_load_2d(dst, &tm_a, fb, ks * kStageK, row0, pol_a);
+                    for (int c = 0; c < chunks; ++c)
+                        for (int b = 0; b < chunk_blocks; ++b) {
+                            const int col = h * p.d + c * p.nc + static_cast<int>(cta) * (p.nc / 2) + 64 * b;
+                            ptx::tma_load_2d(dst + kABytes + (c * chunk_blocks + b) * kBBlock, &tm_b, fb, col,
+                                             ks * kStageK, pol_b);
+                        }
+                }
+            }
+            // every copy into this CTA lands before it may exit
+            for (uint32_t i = it > kStages ? it - kStages : 0; i < it; ++i)
+                qwait_landed(bar(bars->full[i % kStages]), (i / kStages) & 1);
+        }
+    } else if (warp == 1 && !leader) {
+        // ------------------------------------------------------------ relay (follower)
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters)
+            for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+                const uint32_t s = it % kStages;
+                ok = qwait_warp(bar(bars->full[s]), (it / kStages) & 1, bars, peer_abort, p.status);
+                if (ok && lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->full[s]));
+                __syncwarp();
+            }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        constexpr uint32_t kHi = ptx::desc_hi_sw128(1024);
+        constexpr uint32_t kId256 = ptx::instr_desc_f16(true, kTileTokens, 256, true);
+        constexpr uint32_t kId128 = ptx::instr_desc_f16(true, kTileTokens, 128, true);
+        constexpr uint16_t kBoth = 3;
+        const uint32_t a_lo = ptx::desc_lo(sStages, 16);
+        const uint32_t b_lo = ptx::desc_lo(sStages + kABytes, kBBlock);  // LBO: the chunk's next 64 columns
+        constexpr uint32_t kStageU = kStageBytes >> 4;
+        constexpr uint32_t kBlockU = kBBlock >> 4;
+        uint32_t it = 0, tl = 0;
+        bool ok = true;
+        for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters, ++tl) {
+            // the epilogue of the previous tile has read the accumulator
+            ok = qwait_warp(bar(bars->acc_empty), (tl & 1) ^ 1, bars, peer_abort, p.status);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+                const uint32_t s = it % kStages;
+                ok = qwait_warp(bar(bars->full[s]), (it / kStages) & 1, bars, peer_abort, p.status);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                if (ptx::elect_one()) {
+                    const uint32_t a = a_lo + s * kStageU;
+#pragma unroll
+                    for (int k = 0; k < kStageK / 16; ++k) {
+                        // 16 channels of r per MMA: 32 B along A's swizzled rows, 16 rows (2 KB) of B
+                        for (int c = 0; c < chunks; ++c) {
+                            const uint32_t d = tmem + static_cast<uint32_t>(c * p.nc);
+                            const uint32_t b = b_lo + s * kStageU + c * chunk_blocks * kBlockU + 128 * k;
+                            const bool acc = ks > 0 || k > 0;
+                            if (p.nc == 256) {
+                                if (acc) ptx::mma2_ss_lo<kHi, kId256, 1>(d, a + 2 * k, b);
+                                else ptx::mma2_ss_lo<kHi, kId256, 0>(d, a + 2 * k, b);
+                            } else {
+                                if (acc) ptx::mma2_ss_lo<kHi, kId128, 1>(d, a + 2 * k, b);
+                                else ptx::mma2_ss_lo<kHi, kId128, 0>(d, a + 2 * k, b);
+                            }
+                        }
+                    }
+                    ptx::mma_commit_pair(bar(bars->empty[s]), kBoth);  // the stage's operands are read
+                    if (ks == p.k_stages - 1) ptx::mma_commit_pair(bar(bars->acc_full), kBoth);
+                }
+                __syncwarp();
+            }
+        }
+        // drain: every MMA issued here has completed before tensor memory is freed
+        if (ok) {
+            const uint32_t last = tl;  // acc_full phases committed
+            if (last > 0) qwait_warp(bar(bars->acc_full), (last - 1) & 1, bars, peer_abort, p.status);
+        }
+    } else if (warp >= 4) {
+        // ---------------------------------------------------------------- epilogue (both CTAs)
+        const int wq = warp & 3;         // tensor-memory lane quarter
+        const int half = (warp - 4) >> 2;  // which half of the head's channels
+        const int row = wq * 32 + lane;  // row within this CTA's 128
+        const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+        const int hd = p.d / 2;          // channels per half
+        const int c0 = half * hd;
+        const int rope0 = p.d - p.rope;  // first rotated channel
+        const float inv_d = 1.f / static_cast<float>(p.d);
+        uint32_t tl = 0;
+        bool ok = true;
+        for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters, ++tl) {
+            const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
+            const int token = tb * kTileTokens + static_cast<int>(cta) * 128 + row;
+            ok = qwait_warp(bar(bars->acc_full), tl & 1, bars, peer_abort, p.status);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t tA = tmem + lane_addr + static_cast<uint32_t>(c0);
+            // sum of squares over this half of the row
+            float ss = 0.f;
+            for (int c = 0; c < hd; c += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tA + c, r);
+                ptx::tmem_wait_ld_dep(r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float v = __uint_as_float(r[e]);
+                    ss = fmaf(v, v, ss);
+                }
+            }
+            // the other half of these rows is summed by the partner warp (same lane quarter)
+            xss[half * 128 + row] = ss;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(bars->xready[wq]));
+            ok = qwait_warp(bar(bars->xready[wq]), tl & 1, bars, peer_abort, p.status);
+            if (!ok) break;
+            const float total = xss[row] + xss[128 + row];
+            const float inv = rsqrtf(total * inv_d + p.eps);
+            const bool valid = token < p.tokens;
+            __nv_bfloat16 *orow = p.out + static_cast<long long>(token) * p.out_tok +
+                                  static_cast<long long>(h) * p.out_head + c0;
+            const __nv_bfloat16 *cs = p.cos + static_cast<long long>(valid ? token : 0) * p.cos_tok;
+            const __nv_bfloat16 *sn = p.sin + static_cast<long long>(valid ? token : 0) * p.sin_tok;
+            for (int c = 0; c < hd; c += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tA + c, r);
+                ptx::tmem_wait_ld_dep(r);
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float x = __uint_as_float(r[2 * e]) * inv, y = __uint_as_float(r[2 * e + 1]) * inv;
+                    const int ch = c0 + c + 2 * e;  // even channel of the pair
+                    if (ch >= rope0 && valid) {
+                        const int j = ch - rope0;
+                        const float2 cc = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(cs + j));
+                        const float2 ssn = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sn + j));
+                        const float x2 = x * cc.x - y * ssn.x, y2 = y * cc.y + x * ssn.y;
+                        x = x2;
+                        y = y2;
+                    }
+                    w[e] = DType<__nv_bfloat16>::pack(x, y);
+                }
+                if (valid) store_row_chunk(orow + c, w, p.out_v8);
+            }
+            // this warp's reads of the accumulator are done
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->acc_empty));
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync_all();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+}  // namespace prolog
+}  // namespace mla

@@ -94,6 +94,41 @@ def test_small_full_against_oracle():
     s = W.prolog_shapes()["prolog_small"]
     x = W.make_prolog_inputs(s, device=DEV)
     q, kv, cq = run(x, s)
+    assert mla.prolog_last_fused()  # head_dim 256, q_lora_rank 256: the fused q kernel
+    check_all(x, s, np.arange(s.tokens), q, kv, cq)
+
+
+def test_library_q_path_against_oracle_and_fused():
+    # the same problem with the q projection forced onto the library GEMM + row kernel
+    s = W.prolog_shapes()["prolog_small"]
+    x = W.make_prolog_inputs(s, device=DEV)
+    fq, fkv, fcq = run(x, s)
+    mla.set_prolog_path(0)
+    try:
+        q, kv, cq = run(x, s)
+        assert not mla.prolog_last_fused()
+    finally:
+        mla.set_prolog_path(-1)
+    check_all(x, s, np.arange(s.tokens), q, kv, cq)
+    assert torch.equal(cq, fcq) and torch.equal(kv, fkv)  # only the q projection differs
+    # two fp32 accumulation orders of the same products, each rounded once to bf16: at most one ulp apart
+    d = (q.float() - fq.float()).abs()
+    assert torch.all(d <= 2 * torch.from_numpy(half_ulp(fq.float().cpu().double().numpy(), torch.bfloat16)).to(DEV)
+                     + 2.0 ** -20)
+
+
+@pytest.mark.parametrize("shape", [
+    # head_dim 384: three N = 128 chunks per k-step; a ragged last tile of tokens
+    dict(tokens=300, hidden=256, q_lora_rank=192, num_heads=3, head_dim=384, rope_dim=64, seed=65),
+    # head_dim 128 with rope over all of it: both halves of the epilogue rotate
+    dict(tokens=130, hidden=128, q_lora_rank=64, num_heads=2, head_dim=128, rope_dim=128, seed=66),
+])
+def test_fused_kernel_shapes(shape):
+    s = W.PrologShape("prolog_fused", **shape)
+    x = W.make_prolog_inputs(s, device=DEV, positions=np.random.default_rng(shape["seed"]).integers(0, 4096,
+                                                                                                    s.tokens))
+    q, kv, cq = run(x, s)
+    assert mla.prolog_last_fused()
     check_all(x, s, np.arange(s.tokens), q, kv, cq)
 
 
@@ -102,6 +137,7 @@ def test_page_configuration_sampled_tokens():
     s = W.prolog_shapes()["prolog"]
     x = W.make_prolog_inputs(s, device=DEV)
     q, kv, cq = run(x, s)
+    assert mla.prolog_last_fused()
     rows = np.unique(np.concatenate([[0, 1, 127, 128, 2047, 4094, 4095],
                                      np.random.default_rng(5).choice(s.tokens, 25, replace=False)]))
     check_all(x, s, rows, q, kv, cq)
@@ -140,6 +176,14 @@ def test_strided_views_and_guards():
     q, kv, _ = run(y, s, q_out=qbuf[:, :, :d], kv_out=kvbuf[:, :d])
     assert torch.equal(q, ref_q) and torch.equal(kv, ref_kv)
     assert torch.all(qbuf[:, :, d:] == 5.0) and torch.all(kvbuf[:, d:] == 5.0)
+    # q rows on 16-byte but not 32-byte boundaries (the fused epilogue's 128-bit store path)
+    qbuf16 = torch.full((t, H, d + 16), 5.0, dtype=torch.bfloat16, device=DEV)
+    q16 = qbuf16[:, :, 8:8 + d]
+    assert q16.data_ptr() % 32 == 16
+    run(x, s, q_out=q16)
+    assert mla.prolog_last_fused()
+    assert torch.equal(q16, ref_q)
+    assert torch.all(qbuf16[:, :, :8] == 5.0) and torch.all(qbuf16[:, :, 8 + d:] == 5.0)
 
 
 def test_repeatable():
@@ -151,9 +195,10 @@ def test_repeatable():
 
 
 def test_head_dim_outside_the_fused_kernel():
-    # head_dim 96 is not a tensor-memory accumulator size: the library GEMM + row kernel path
+    # head_dim 96 is not a multiple of 128 (the fused kernel's N chunks): the library GEMM + row kernel path
     s = W.PrologShape("prolog_d96", tokens=50, hidden=256, q_lora_rank=96, num_heads=3, head_dim=96, rope_dim=32,
                       seed=64)
     x = W.make_prolog_inputs(s, device=DEV)
     q, kv, cq = run(x, s)
+    assert not mla.prolog_last_fused()
     check_all(x, s, np.arange(s.tokens), q, kv, cq)
