@@ -338,7 +338,8 @@ int mla_prefill_paged(const mla_tensor *q, const mla_tensor *q_rope, const mla_t
  * The q projection c^Q wq_b runs in this library's tcgen05 kernel with the
  * per-head RmsNorm and RoPE as its epilogue (the head's d channels of 256
  * tokens accumulate in fp32 in tensor memory and are written once, as bf16)
- * when d is a multiple of 128 up to 512, r a multiple of 64 and R even -- the
+ * when d is a multiple of 128 up to 512, r a multiple of 64 and R a multiple
+ * of 32 -- the
  * page's sizes among them; otherwise it runs as a library GEMM (fp32 result)
  * followed by a row kernel.  x wq_a and x wkv are library GEMMs (cuBLAS, fp32
  * results) followed by the row kernel.  Nothing is rounded before the norms

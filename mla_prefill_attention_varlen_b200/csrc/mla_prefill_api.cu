@@ -1203,10 +1203,25 @@ int encode_map2d(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, i
     return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_UNSUPPORTED;
 }
 
+// q_out rows of a slab {d, H, tokens} for the fused q kernel's TMA stores: a {32, 1, 128} box with
+// 64-byte swizzle (its staging buffers' layout).
+int encode_out_map(CUtensorMap *m, const View3 &v) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(v.width), static_cast<cuuint64_t>(v.heads),
+                                static_cast<cuuint64_t>(v.tokens)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>((v.heads > 1 ? v.st_head : v.width) * 2),
+                                   static_cast<cuuint64_t>((v.tokens > 1 ? v.st_tok : v.heads * v.width) * 2)};
+    const cuuint32_t box[3] = {32, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v.data, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_UNSUPPORTED;
+}
+
 // The fused q projection + per-head RmsNorm + RoPE (prolog_q_sm100.cuh): clusters of two CTAs, one
 // per SM, static tiles of 256 tokens x one head.
 int launch_prolog_q(DeviceState *ds, cudaStream_t stream, const CUtensorMap &tm_a, const CUtensorMap &tm_b,
-                    const mla::prolog::QParams &qp) {
+                    const CUtensorMap &tm_o, const mla::prolog::QParams &qp) {
     auto kern = mla::prolog::mla_prolog_q_kernel;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(mla::prolog::kThreads);
@@ -1235,7 +1250,7 @@ int launch_prolog_q(DeviceState *ds, cudaStream_t stream, const CUtensorMap &tm_
                           qp.heads;
     const int64_t clusters = tiles < ds->prolog_clusters ? tiles : ds->prolog_clusters;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
-    if (cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, qp) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, tm_o, qp) != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;
 }
 
@@ -1292,8 +1307,9 @@ extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, con
 
     // The q projection runs fused with its norm and rotation (prolog_q_sm100.cuh) where the sizes fit
     // the kernel's tiles: head_dim a multiple of 128 up to 512 (the accumulator of a head row in
-    // tensor memory), q_lora_rank a multiple of 64 (its k-stages), an even rope_dim.
-    const bool fused = t_prolog_path != 0 && d % 128 == 0 && d <= 512 && r % 64 == 0 && R % 2 == 0;
+    // tensor memory), q_lora_rank a multiple of 64 (its k-stages), rope_dim a multiple of 32 (the
+    // epilogue's column chunks are rotated whole).
+    const bool fused = t_prolog_path != 0 && d % 128 == 0 && d <= 512 && r % 64 == 0 && R % 32 == 0;
     // scratch per slab: [S, r + d] fp32 (x wq_a | x wkv), [S, H d] fp32 (c^Q wq_b; library path
     // only), [S, r] bf16 c^Q
     const int64_t slab = t < kPrologSlab ? t : kPrologSlab;
@@ -1345,12 +1361,13 @@ extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, con
         if ((rc = launch_norm(np, ds->sm_count, stream)) != MLA_OK) return rc;
         if (fused) {
             // c^Q wq_b with the per-head RmsNorm and rope as the epilogue, straight into q_out
-            CUtensorMap tm_a;
+            CUtensorMap tm_a, tm_o;
             if ((rc = encode_map2d(&tm_a, cq, r, S, cq_ld * 2, 128)) != MLA_OK) return rc;
+            View3 qs = qo;  // this slab's rows of q_out
+            qs.data = bf(qo.data, s0 * qo.st_tok);
+            qs.tokens = S;
+            if ((rc = encode_out_map(&tm_o, qs)) != MLA_OK) return rc;
             mla::prolog::QParams qp{};
-            qp.out = bf(qo.data, s0 * qo.st_tok);
-            qp.out_tok = qo.st_tok;
-            qp.out_head = qo.st_head;
             qp.cos = bf(cs.data, s0 * cs.ld);
             qp.sin = bf(sn.data, s0 * sn.ld);
             qp.cos_tok = cs.ld;
@@ -1362,11 +1379,9 @@ extern "C" int mla_prolog(const mla_tensor *token_x, const mla_tensor *wq_a, con
             qp.rope = static_cast<int>(R);
             qp.k_stages = static_cast<int>(r / 64);
             qp.eps = eps;
-            qp.out_v8 = (reinterpret_cast<uintptr_t>(qp.out) % 32 == 0 && qo.st_tok % 16 == 0 && qo.st_head % 16 == 0)
-                            ? 1 : 0;
             qp.status = ds->status;
             if (t_prof_start && cudaEventRecord(t_prof_start, stream) != cudaSuccess) return MLA_ERR_CUDA;
-            if ((rc = launch_prolog_q(ds, stream, tm_a, tm_b, qp)) != MLA_OK) return rc;
+            if ((rc = launch_prolog_q(ds, stream, tm_a, tm_b, tm_o, qp)) != MLA_OK) return rc;
             if (t_prof_stop && cudaEventRecord(t_prof_stop, stream) != cudaSuccess) return MLA_ERR_CUDA;
             continue;
         }

@@ -14,14 +14,18 @@
 // (256 when d is a multiple of 256, else 128): B is split along N, so for N-chunk c each CTA loads
 // its nc/2 columns c*nc + rank*nc/2 + [0, nc/2).  A k-stage is 64 channels of r: per CTA 16 KB of A
 // (128 rows x 128 B) and d/128 blocks of 8 KB of B (64 rows of r x 64 columns, 128-byte swizzled);
-// four stages in flight.
+// four stages in flight.  The epilogue writes q through shared memory: each 32-column block of a
+// half (128 rows x 64 B, 64-byte swizzled; two buffers per half) is stored by a TMA tensor store,
+// so the output leaves in whole 64-byte row segments, a store overlaps the next block's work, and
+// rows past the last token are clipped by the store.
 //
 //   leader   warp 0: TMA loads of its A rows and B halves; warp 1: MMA issuer for the pair
 //   follower warp 0: TMA loads of its halves; warp 1: relay of its full barriers to the leader's
 //   both     warps 4-11: epilogue, two warps per tensor-memory lane quarter, each one half of the
 //            head's d channels of 32 rows: sum of squares over its half, the two halves added
-//            through shared memory (an mbarrier per lane quarter), then scale, rotate, convert and
-//            store its half
+//            through shared memory (an mbarrier per lane quarter), then per 32-column block scale,
+//            rotate, convert and stage it
+//            warps 2, 3: TMA stores of the staged blocks of half 0 / 1
 // Tiles are static (tile = cluster + i * clusters, head-major so that concurrent clusters share a
 // head's wq_b columns in L2).  The accumulator fills tensor memory: the next tile's MMAs wait for
 // the epilogue (an acc-empty barrier), while the producers already load its first stages.
@@ -41,8 +45,11 @@ constexpr int kABytes = 128 * kStageK * 2;  // 16 KB: this CTA's 128 rows of the
 constexpr int kBBlock = 64 * kStageK * 2;   // 8 KB: 64 columns of wq_b x the stage's 64 rows
 constexpr int kMaxBBlocks = 4;              // d <= 512: d / 128 blocks per CTA and stage
 constexpr int kStageBytes = kABytes + kMaxBBlocks * kBBlock;
+constexpr int kOutCols = 32;                   // output block: 32 columns (64 B) x 128 rows
+constexpr int kStageOut = 128 * kOutCols * 2;   // 8 KB
 constexpr int kSmemStages = 0;
-constexpr int kSmemBar = kSmemStages + kStages * kStageBytes;
+constexpr int kSmemOut = kSmemStages + kStages * kStageBytes;  // two output blocks per half
+constexpr int kSmemBar = kSmemOut + 4 * kStageOut;
 constexpr int kSmemXss = kSmemBar + 256;      // per-row partial sums of squares, one per half
 constexpr int kSmemBytes = kSmemXss + 2 * 128 * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
@@ -52,18 +59,15 @@ constexpr int kAccEmptyArrivals = 2 * kEpiWarps;  // every epilogue warp of both
 constexpr uint64_t kWaitLimitNs = 200000000ull;   // 200 ms
 
 struct QParams {
-    __nv_bfloat16 *out;          // q_out rows: token * out_tok + head * out_head
-    long long out_tok, out_head;
     const __nv_bfloat16 *cos, *sin;  // [tokens, R] with row strides cos_tok / sin_tok
     long long cos_tok, sin_tok;
     int tokens;      // rows of this launch
     int heads;       // H
     int d;           // head_dim: a multiple of 128, <= 512
     int nc;          // MMA N per chunk: 256 or 128
-    int rope;        // R (even, <= d)
+    int rope;        // R (a multiple of 32, <= d)
     int k_stages;    // r / 64
     float eps;
-    int out_v8;      // output rows allow 32-byte stores
     int *status;
 };
 
@@ -71,6 +75,7 @@ struct Bars {
     uint64_t full[kStages], empty[kStages];
     uint64_t acc_full, acc_empty;
     uint64_t xready[4];  // per lane quarter: both halves' sums of squares are in shared memory
+    uint64_t st_full[2][2], st_empty[2][2];  // [half][buffer]: staged by the half's 4 warps / read by its store
     uint32_t tmem_base;
     int abort;
 };
@@ -108,12 +113,13 @@ __device__ __forceinline__ void qwait_landed(uint32_t bar, uint32_t parity) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     mla_prolog_q_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                        const QParams p) {
+                        const __grid_constant__ CUtensorMap tm_o /* q_out {d, H, tokens} */, const QParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bars = reinterpret_cast<Bars *>(smem + kSmemBar);
     float *xss = reinterpret_cast<float *>(smem + kSmemXss);
     const uint32_t sStages = ptx::smem_addr(smem + kSmemStages);
+    const uint32_t sOut = ptx::smem_addr(smem + kSmemOut);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t cta = ptx::cluster_ctarank();
@@ -125,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 32) {
         ptx::tma_prefetch_desc(&tm_a);
         ptx::tma_prefetch_desc(&tm_b);
+        ptx::tma_prefetch_desc(&tm_o);
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -134,6 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(bar(bars->acc_full), 1);
         ptx::mbar_init(bar(bars->acc_empty), kAccEmptyArrivals);
         for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(bars->xready[q]), 2);
+        for (int hh = 0; hh < 2; ++hh)
+            for (int b = 0; b < 2; ++b) {
+                ptx::mbar_init(bar(bars->st_full[hh][b]), 4);
+                ptx::mbar_init(bar(bars->st_empty[hh][b]), 1);
+            }
         bars->abort = 0;
         ptx::fence_mbar_init();
     }
@@ -257,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c0 = half * hd;
         const int rope0 = p.d - p.rope;  // first rotated channel
         const float inv_d = 1.f / static_cast<float>(p.d);
-        uint32_t tl = 0;
+        uint32_t tl = 0, kb = 0;  // tiles; output blocks staged by this half
         bool ok = true;
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters, ++tl) {
             const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
@@ -286,37 +298,100 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             const float total = xss[row] + xss[128 + row];
             const float inv = rsqrtf(total * inv_d + p.eps);
-            const bool valid = token < p.tokens;
-            __nv_bfloat16 *orow = p.out + static_cast<long long>(token) * p.out_tok +
-                                  static_cast<long long>(h) * p.out_head + c0;
-            const __nv_bfloat16 *cs = p.cos + static_cast<long long>(valid ? token : 0) * p.cos_tok;
-            const __nv_bfloat16 *sn = p.sin + static_cast<long long>(valid ? token : 0) * p.sin_tok;
-            for (int c = 0; c < hd; c += 32) {
-                uint32_t r[32];
-                ptx::tmem_ld32(tA + c, r);
-                ptx::tmem_wait_ld_dep(r);
+            const int tok_c = token < p.tokens ? token : 0;  // rows past the end: any valid cos / sin row
+            const __nv_bfloat16 *cs = p.cos + static_cast<long long>(tok_c) * p.cos_tok;
+            const __nv_bfloat16 *sn = p.sin + static_cast<long long>(tok_c) * p.sin_tok;
+            // per 32-column block: scale (and rotate), pack to bf16 and stage row `row` in one of the
+            // half's two 64-byte-swizzled buffers; the half's first warp stores the block with TMA.
+            // The next block's tensor-memory load is issued before this block is processed.
+            const int nblk = hd / kOutCols;  // even: hd is a multiple of 64
+            // one block: cur holds its accumulator columns; the next block's load goes to nxt
+            auto block = [&](int k, const uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
+                const int cc = c0 + k * kOutCols;  // first channel of the block
+                const bool rot = cc >= rope0;
+                uint4 cv[4], sv[4];
+                if (rot) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        cv[v] = __ldg(reinterpret_cast<const uint4 *>(cs + (cc - rope0)) + v);
+                        sv[v] = __ldg(reinterpret_cast<const uint4 *>(sn + (cc - rope0)) + v);
+                    }
+                }
+                if (k + 1 < nblk) {
+                    ptx::tmem_ld32(tA + (k + 1) * kOutCols, nxt);
+                } else {  // this warp's last accumulator read of the tile has completed
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->acc_empty));
+                }
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    float x = __uint_as_float(r[2 * e]) * inv, y = __uint_as_float(r[2 * e + 1]) * inv;
-                    const int ch = c0 + c + 2 * e;  // even channel of the pair
-                    if (ch >= rope0 && valid) {
-                        const int j = ch - rope0;
-                        const float2 cc = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(cs + j));
-                        const float2 ssn = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(sn + j));
-                        const float x2 = x * cc.x - y * ssn.x, y2 = y * cc.y + x * ssn.y;
+                    float x = __uint_as_float(cur[2 * e]) * inv, y = __uint_as_float(cur[2 * e + 1]) * inv;
+                    if (rot) {
+                        const uint32_t cw = reinterpret_cast<const uint32_t *>(&cv[e >> 2])[e & 3];
+                        const uint32_t sw = reinterpret_cast<const uint32_t *>(&sv[e >> 2])[e & 3];
+                        const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&cw));
+                        const float2 s2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&sw));
+                        const float x2 = x * c2.x - y * s2.x, y2 = y * c2.y + x * s2.y;
                         x = x2;
                         y = y2;
                     }
                     w[e] = DType<__nv_bfloat16>::pack(x, y);
                 }
-                if (valid) store_row_chunk(orow + c, w, p.out_v8);
+                const uint32_t b = kb & 1, use = kb >> 1;
+                const uint32_t buf = sOut + static_cast<uint32_t>((half * 2 + b) * kStageOut);
+                // the buffer is free once the store of its previous block has read it
+                if (use > 0 &&
+                    !(ok = qwait_warp(bar(bars->st_empty[half][b]), (use - 1) & 1, bars, peer_abort, p.status)))
+                    return;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {  // 16-byte chunk v of the row's 64 bytes, swizzled by (row / 2) mod 4
+                    const uint32_t chunk = static_cast<uint32_t>(v ^ ((row >> 1) & 3));
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + row * 64 + chunk * 16),
+                                 "r"(w[4 * v]), "r"(w[4 * v + 1]), "r"(w[4 * v + 2]), "r"(w[4 * v + 3])
+                                 : "memory");
+                }
+                ptx::fence_proxy_async_smem();  // visible to the TMA store
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar(bars->st_full[half][b]));
+                ++kb;
+                if (k + 1 < nblk) ptx::tmem_wait_ld_dep(nxt);
+            };
+            uint32_t r0[32], r1[32];
+            ptx::tmem_ld32(tA, r0);
+            ptx::tmem_wait_ld_dep(r0);
+            for (int k = 0; k < nblk && ok; k += 2) {
+                block(k, r0, r1);
+                if (ok) block(k + 1, r1, r0);
             }
-            // this warp's reads of the accumulator are done
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->acc_empty));
         }
+    } else if (warp >= 2) {
+        // ---------------------------------------------------------------- q stores (both CTAs)
+        // Warp 2 stores half 0's blocks, warp 3 half 1's, in the epilogue's order: once the half's
+        // four warps have staged a block, one TMA tensor store; once the store before it has read
+        // its buffer, that buffer is released.
+        const int half = warp - 2;
+        const int hd = p.d / 2, nblk = hd / kOutCols;
+        uint32_t kb = 0;
+        bool ok = true;
+        for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters) {
+            const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
+            for (int k = 0; k < nblk && ok; ++k, ++kb) {
+                const uint32_t b = kb & 1, use = kb >> 1;
+                ok = qwait_warp(bar(bars->st_full[half][b]), use & 1, bars, peer_abort, p.status);
+                if (!ok) break;
+                if (lane == 0) {
+                    ptx::tma_store_3d(&tm_o, sOut + static_cast<uint32_t>((half * 2 + b) * kStageOut),
+                                      half * hd + k * kOutCols, h, tb * kTileTokens + static_cast<int>(cta) * 128);
+                    ptx::bulk_commit_group();
+                    ptx::bulk_wait_group_read1();  // the previous block's store has read its buffer
+                    if (kb > 0) ptx::mbar_arrive(bar(bars->st_empty[half][b ^ 1]));
+                }
+                __syncwarp();
+            }
+        }
+        if (lane == 0) ptx::bulk_wait_group0();  // this CTA's q stores have completed
     }
 
     ptx::tc_fence_before();

@@ -176,7 +176,7 @@ def test_strided_views_and_guards():
     q, kv, _ = run(y, s, q_out=qbuf[:, :, :d], kv_out=kvbuf[:, :d])
     assert torch.equal(q, ref_q) and torch.equal(kv, ref_kv)
     assert torch.all(qbuf[:, :, d:] == 5.0) and torch.all(kvbuf[:, d:] == 5.0)
-    # q rows on 16-byte but not 32-byte boundaries (the fused epilogue's 128-bit store path)
+    # q rows on 16-byte but not 32-byte boundaries (the fused epilogue's TMA store of a strided view)
     qbuf16 = torch.full((t, H, d + 16), 5.0, dtype=torch.bfloat16, device=DEV)
     q16 = qbuf16[:, :, 8:8 + d]
     assert q16.data_ptr() % 32 == 16
