@@ -12,23 +12,25 @@
 // Operands: A = c^Q rows (K-major: r contiguous), B = wq_b (MN-major: the head's d columns
 // contiguous).  The MMAs are tcgen05 cta_group::2 with M = 256 (128 rows in each CTA) and N = nc
 // (256 when d is a multiple of 256, else 128): B is split along N, so for N-chunk c each CTA loads
-// its nc/2 columns c*nc + rank*nc/2 + [0, nc/2).  A k-stage is 64 channels of r: per CTA 16 KB of A
-// (128 rows x 128 B) and d/128 blocks of 8 KB of B (64 rows of r x 64 columns, 128-byte swizzled);
-// four stages in flight.  The epilogue writes q through shared memory: each 32-column block of a
+// its nc/2 columns c*nc + rank*nc/2 + [0, nc/2).  A stage is 64 channels of r for one N-chunk: per
+// CTA 16 KB of A (128 rows x 128 B) and nc/128 blocks of 8 KB of B (64 rows of r x 64 columns,
+// 128-byte swizzled); six stages in flight.  A tile runs chunk by chunk (A is read once per chunk),
+// and the head's two channel halves have their own accumulated / read-back barriers, so the next
+// tile's first chunk starts as soon as the epilogue has read the first half.  The epilogue writes q through shared memory: each 32-column block of a
 // half (128 rows x 64 B, 64-byte swizzled; two buffers per half) is stored by a TMA tensor store,
 // so the output leaves in whole 64-byte row segments, a store overlaps the next block's work, and
 // rows past the last token are clipped by the store.
 //
 //   leader   warp 0: TMA loads of its A rows and B halves; warp 1: MMA issuer for the pair
 //   follower warp 0: TMA loads of its halves; warp 1: relay of its full barriers to the leader's
-//   both     warps 4-11: epilogue, two warps per tensor-memory lane quarter, each one half of the
-//            head's d channels of 32 rows: sum of squares over its half, the two halves added
-//            through shared memory (an mbarrier per lane quarter), then per 32-column block scale,
-//            rotate, convert and stage it
+//   both     warps 4-11: epilogue, two warps per tensor-memory lane quarter: each sums the squares
+//            of one half of the head's d channels of 32 rows, the two sums meet through shared
+//            memory (an mbarrier per lane quarter); then both finish the first half (a quarter of
+//            the head each), release it, and do the second: per 32-column block scale, rotate,
+//            convert and stage
 //            warps 2, 3: TMA stores of the staged blocks of half 0 / 1
 // Tiles are static (tile = cluster + i * clusters, head-major so that concurrent clusters share a
-// head's wq_b columns in L2).  The accumulator fills tensor memory: the next tile's MMAs wait for
-// the epilogue (an acc-empty barrier), while the producers already load its first stages.
+// head's wq_b columns in L2).
 // Every wait is bounded; a timeout sets the status word and aborts both CTAs.
 #pragma once
 
@@ -40,10 +42,10 @@ namespace prolog {
 constexpr int kThreads = 384;
 constexpr int kTileTokens = 256;   // rows of one pair MMA (128 per CTA)
 constexpr int kStageK = 64;        // channels of r per stage (one 128-byte swizzle row of A)
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kABytes = 128 * kStageK * 2;  // 16 KB: this CTA's 128 rows of the stage
 constexpr int kBBlock = 64 * kStageK * 2;   // 8 KB: 64 columns of wq_b x the stage's 64 rows
-constexpr int kMaxBBlocks = 4;              // d <= 512: d / 128 blocks per CTA and stage
+constexpr int kMaxBBlocks = 2;              // one N-chunk per stage: nc / 128 blocks per CTA
 constexpr int kStageBytes = kABytes + kMaxBBlocks * kBBlock;
 constexpr int kOutCols = 32;                   // output block: 32 columns (64 B) x 128 rows
 constexpr int kStageOut = 128 * kOutCols * 2;   // 8 KB
@@ -55,7 +57,7 @@ constexpr int kSmemBytes = kSmemXss + 2 * 128 * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 constexpr int kEpiWarps = 8;
-constexpr int kAccEmptyArrivals = 2 * kEpiWarps;  // every epilogue warp of both CTAs
+constexpr int kHalfFreeArrivals = 2 * kEpiWarps;  // every epilogue warp of both CTAs reads part of each half
 constexpr uint64_t kWaitLimitNs = 200000000ull;   // 200 ms
 
 struct QParams {
@@ -73,7 +75,7 @@ struct QParams {
 
 struct Bars {
     uint64_t full[kStages], empty[kStages];
-    uint64_t acc_full, acc_empty;
+    uint64_t half_full[2], half_free[2];  // the head's channel halves: accumulated / read by the epilogue
     uint64_t xready[4];  // per lane quarter: both halves' sums of squares are in shared memory
     uint64_t st_full[2][2], st_empty[2][2];  // [half][buffer]: staged by the half's 4 warps / read by its store
     uint32_t tmem_base;
@@ -138,8 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(bars->full[s]), leader ? 2 : 1);
             ptx::mbar_init(bar(bars->empty[s]), 1);
         }
-        ptx::mbar_init(bar(bars->acc_full), 1);
-        ptx::mbar_init(bar(bars->acc_empty), kAccEmptyArrivals);
+        for (int hh = 0; hh < 2; ++hh) {
+            ptx::mbar_init(bar(bars->half_full[hh]), 1);
+            ptx::mbar_init(bar(bars->half_free[hh]), kHalfFreeArrivals);
+        }
         for (int q = 0; q < 4; ++q) ptx::mbar_init(bar(bars->xready[q]), 2);
         for (int hh = 0; hh < 2; ++hh)
             for (int b = 0; b < 2; ++b) {
@@ -161,10 +165,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tblocks = (p.tokens + kTileTokens - 1) / kTileTokens;
     const int n_tiles = n_tblocks * p.heads;
     const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
-    const int b_blocks = p.d / 128;        // this CTA's 8 KB B blocks per stage
-    const int chunk_blocks = p.nc / 128;   // of which per N-chunk
+    const int chunk_blocks = p.nc / 128;   // this CTA's 8 KB B blocks per stage (one N-chunk)
     const int chunks = p.d / p.nc;
-    const uint32_t stage_tx = kABytes + b_blocks * kBBlock;
+    const int hd = p.d / 2;                // channels per half of the head
+    const uint32_t stage_tx = kABytes + chunk_blocks * kBBlock;
+    // Per tile the stages run N-chunk by N-chunk (all of r for chunk 0, then chunk 1, ...), so the
+    // columns of the head's first half are accumulated, and can be handed back by the epilogue,
+    // before those of its second half.
+    const int stages_per_tile = chunks * p.k_stages;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -176,22 +184,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters) {
                 const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
                 const int row0 = tb * kTileTokens + static_cast<int>(cta) * 128;
-                for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
-                    const uint32_t s = it % kStages;
-                    if (it >= kStages && !(ok = qwait(bar(bars->empty[s]), ((it / kStages) & 1) ^ 1, bars, peer_abort,
-                                                      p.status)))
-                        break;
-                    const uint32_t fb = bar(bars->full[s]);
-                    const uint32_t dst = sStages + s * kStageBytes;
-                    ptx::mbar_arrive_expect_tx(fb, stage_tx);
-                    ptx::tma_load_2d(dst, &tm_a, fb, ks * kStageK, row0, pol_a);
-                    for (int c = 0; c < chunks; ++c)
+                for (int c = 0; c < chunks && ok; ++c)
+                    for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+                        const uint32_t s = it % kStages;
+                        if (it >= kStages && !(ok = qwait(bar(bars->empty[s]), ((it / kStages) & 1) ^ 1, bars,
+                                                          peer_abort, p.status)))
+                            break;
+                        const uint32_t fb = bar(bars->full[s]);
+                        const uint32_t dst = sStages + s * kStageBytes;
+                        ptx::mbar_arrive_expect_tx(fb, stage_tx);
+                        ptx::tma_load_2d(dst, &tm_a, fb, ks * kStageK, row0, pol_a);
                         for (int b = 0; b < chunk_blocks; ++b) {
                             const int col = h * p.d + c * p.nc + static_cast<int>(cta) * (p.nc / 2) + 64 * b;
-                            ptx::tma_load_2d(dst + kABytes + (c * chunk_blocks + b) * kBBlock, &tm_b, fb, col,
-                                             ks * kStageK, pol_b);
+                            ptx::tma_load_2d(dst + kABytes + b * kBBlock, &tm_b, fb, col, ks * kStageK, pol_b);
                         }
-                }
+                    }
             }
             // every copy into this CTA lands before it may exit
             for (uint32_t i = it > kStages ? it - kStages : 0; i < it; ++i)
@@ -202,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters)
-            for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+            for (int k = 0; k < stages_per_tile && ok; ++k, ++it) {
                 const uint32_t s = it % kStages;
                 ok = qwait_warp(bar(bars->full[s]), (it / kStages) & 1, bars, peer_abort, p.status);
                 if (ok && lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->full[s]));
@@ -217,68 +224,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_lo = ptx::desc_lo(sStages, 16);
         const uint32_t b_lo = ptx::desc_lo(sStages + kABytes, kBBlock);  // LBO: the chunk's next 64 columns
         constexpr uint32_t kStageU = kStageBytes >> 4;
-        constexpr uint32_t kBlockU = kBBlock >> 4;
         uint32_t it = 0, tl = 0;
         bool ok = true;
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters, ++tl) {
-            // the epilogue of the previous tile has read the accumulator
-            ok = qwait_warp(bar(bars->acc_empty), (tl & 1) ^ 1, bars, peer_abort, p.status);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
-                const uint32_t s = it % kStages;
-                ok = qwait_warp(bar(bars->full[s]), (it / kStages) & 1, bars, peer_abort, p.status);
+            int waited = 0;  // halves whose previous-tile release this tile has waited for
+            for (int c = 0; c < chunks && ok; ++c) {
+                // the halves chunk c writes must have been read by the previous tile's epilogue
+                const int h_lo = (c * p.nc) / hd, h_hi = ((c + 1) * p.nc - 1) / hd;
+                for (int hh = h_lo; hh <= h_hi && ok; ++hh)
+                    if (!(waited & (1 << hh))) {
+                        ok = qwait_warp(bar(bars->half_free[hh]), (tl & 1) ^ 1, bars, peer_abort, p.status);
+                        waited |= 1 << hh;
+                    }
                 if (!ok) break;
                 ptx::tc_fence_after();
-                if (ptx::elect_one()) {
-                    const uint32_t a = a_lo + s * kStageU;
+                const uint32_t d = tmem + static_cast<uint32_t>(c * p.nc);
+                for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+                    const uint32_t s = it % kStages;
+                    ok = qwait_warp(bar(bars->full[s]), (it / kStages) & 1, bars, peer_abort, p.status);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    if (ptx::elect_one()) {
+                        const uint32_t a = a_lo + s * kStageU, b = b_lo + s * kStageU;
 #pragma unroll
-                    for (int k = 0; k < kStageK / 16; ++k) {
-                        // 16 channels of r per MMA: 32 B along A's swizzled rows, 16 rows (2 KB) of B
-                        for (int c = 0; c < chunks; ++c) {
-                            const uint32_t d = tmem + static_cast<uint32_t>(c * p.nc);
-                            const uint32_t b = b_lo + s * kStageU + c * chunk_blocks * kBlockU + 128 * k;
+                        for (int k = 0; k < kStageK / 16; ++k) {
+                            // 16 channels of r per MMA: 32 B along A's swizzled rows, 16 rows (2 KB) of B
                             const bool acc = ks > 0 || k > 0;
                             if (p.nc == 256) {
-                                if (acc) ptx::mma2_ss_lo<kHi, kId256, 1>(d, a + 2 * k, b);
-                                else ptx::mma2_ss_lo<kHi, kId256, 0>(d, a + 2 * k, b);
+                                if (acc) ptx::mma2_ss_lo<kHi, kId256, 1>(d, a + 2 * k, b + 128 * k);
+                                else ptx::mma2_ss_lo<kHi, kId256, 0>(d, a + 2 * k, b + 128 * k);
                             } else {
-                                if (acc) ptx::mma2_ss_lo<kHi, kId128, 1>(d, a + 2 * k, b);
-                                else ptx::mma2_ss_lo<kHi, kId128, 0>(d, a + 2 * k, b);
+                                if (acc) ptx::mma2_ss_lo<kHi, kId128, 1>(d, a + 2 * k, b + 128 * k);
+                                else ptx::mma2_ss_lo<kHi, kId128, 0>(d, a + 2 * k, b + 128 * k);
                             }
                         }
+                        ptx::mma_commit_pair(bar(bars->empty[s]), kBoth);  // the stage's operands are read
+                        if (ks == p.k_stages - 1)  // halves whose last chunk this is are complete
+                            for (int hh = h_lo; hh <= h_hi; ++hh)
+                                if ((hh + 1) * hd <= (c + 1) * p.nc) ptx::mma_commit_pair(bar(bars->half_full[hh]), kBoth);
                     }
-                    ptx::mma_commit_pair(bar(bars->empty[s]), kBoth);  // the stage's operands are read
-                    if (ks == p.k_stages - 1) ptx::mma_commit_pair(bar(bars->acc_full), kBoth);
+                    __syncwarp();
                 }
-                __syncwarp();
             }
-        }
-        // drain: every MMA issued here has completed before tensor memory is freed
-        if (ok) {
-            const uint32_t last = tl;  // acc_full phases committed
-            if (last > 0) qwait_warp(bar(bars->acc_full), (last - 1) & 1, bars, peer_abort, p.status);
         }
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- epilogue (both CTAs)
-        const int wq = warp & 3;         // tensor-memory lane quarter
-        const int half = (warp - 4) >> 2;  // which half of the head's channels
-        const int row = wq * 32 + lane;  // row within this CTA's 128
+        const int wq = warp & 3;           // tensor-memory lane quarter
+        const int half = (warp - 4) >> 2;  // half of the head summed in the first pass
+        const int row = wq * 32 + lane;    // row within this CTA's 128
         const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-        const int hd = p.d / 2;          // channels per half
         const int c0 = half * hd;
         const int rope0 = p.d - p.rope;  // first rotated channel
         const float inv_d = 1.f / static_cast<float>(p.d);
-        uint32_t tl = 0, kb = 0;  // tiles; output blocks staged by this half
+        const int nb = p.d / 64;         // output blocks of 32 columns per warp and tile (even)
+        uint32_t tl = 0, kb = 0;         // tiles; output blocks staged by this warp's buffers
         bool ok = true;
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters, ++tl) {
             const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
             const int token = tb * kTileTokens + static_cast<int>(cta) * 128 + row;
-            ok = qwait_warp(bar(bars->acc_full), tl & 1, bars, peer_abort, p.status);
+            ok = qwait_warp(bar(bars->half_full[half]), tl & 1, bars, peer_abort, p.status);
             if (!ok) break;
             ptx::tc_fence_after();
+            // sum of squares over this warp's half of the row
             const uint32_t tA = tmem + lane_addr + static_cast<uint32_t>(c0);
-            // sum of squares over this half of the row
             float ss = 0.f;
             for (int c = 0; c < hd; c += 32) {
                 uint32_t r[32];
@@ -298,16 +306,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             const float total = xss[row] + xss[128 + row];
             const float inv = rsqrtf(total * inv_d + p.eps);
+            // the second pass reads both halves (the partner's half too): its accumulation is complete
+            ok = qwait_warp(bar(bars->half_full[half ^ 1]), tl & 1, bars, peer_abort, p.status);
+            if (!ok) break;
+            ptx::tc_fence_after();
             const int tok_c = token < p.tokens ? token : 0;  // rows past the end: any valid cos / sin row
             const __nv_bfloat16 *cs = p.cos + static_cast<long long>(tok_c) * p.cos_tok;
             const __nv_bfloat16 *sn = p.sin + static_cast<long long>(tok_c) * p.sin_tok;
-            // per 32-column block: scale (and rotate), pack to bf16 and stage row `row` in one of the
-            // half's two 64-byte-swizzled buffers; the half's first warp stores the block with TMA.
-            // The next block's tensor-memory load is issued before this block is processed.
-            const int nblk = hd / kOutCols;  // even: hd is a multiple of 64
-            // one block: cur holds its accumulator columns; the next block's load goes to nxt
+            // second pass: the two warps of a lane quarter finish the head's first half (each a
+            // quarter of the head), hand it back to the MMA warp, then do the second half.  Per
+            // 32-column block: scale (and rotate), pack to bf16 and stage row `row` in one of this
+            // warp's two 64-byte-swizzled buffers; the store warps write it with TMA.  The next
+            // block's tensor-memory load is issued before this block is processed.
+            auto col_of = [&](int k) { return (k < nb / 2 ? 0 : hd) + half * (hd / 2) + (k % (nb / 2)) * kOutCols; };
             auto block = [&](int k, const uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
-                const int cc = c0 + k * kOutCols;  // first channel of the block
+                const int cc = col_of(k);
                 const bool rot = cc >= rope0;
                 uint4 cv[4], sv[4];
                 if (rot) {
@@ -317,13 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sv[v] = __ldg(reinterpret_cast<const uint4 *>(sn + (cc - rope0)) + v);
                     }
                 }
-                if (k + 1 < nblk) {
-                    ptx::tmem_ld32(tA + (k + 1) * kOutCols, nxt);
-                } else {  // this warp's last accumulator read of the tile has completed
+                if (k == nb / 2 - 1 || k == nb - 1) {  // this warp's last read of a half has completed
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->acc_empty));
+                    if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->half_free[k == nb - 1 ? 1 : 0]));
                 }
+                if (k + 1 < nb) ptx::tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(col_of(k + 1)), nxt);
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -356,34 +368,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar(bars->st_full[half][b]));
                 ++kb;
-                if (k + 1 < nblk) ptx::tmem_wait_ld_dep(nxt);
+                if (k + 1 < nb) ptx::tmem_wait_ld_dep(nxt);
             };
             uint32_t r0[32], r1[32];
-            ptx::tmem_ld32(tA, r0);
+            ptx::tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(col_of(0)), r0);
             ptx::tmem_wait_ld_dep(r0);
-            for (int k = 0; k < nblk && ok; k += 2) {
+            for (int k = 0; k < nb && ok; k += 2) {
                 block(k, r0, r1);
                 if (ok) block(k + 1, r1, r0);
             }
         }
     } else if (warp >= 2) {
         // ---------------------------------------------------------------- q stores (both CTAs)
-        // Warp 2 stores half 0's blocks, warp 3 half 1's, in the epilogue's order: once the half's
-        // four warps have staged a block, one TMA tensor store; once the store before it has read
-        // its buffer, that buffer is released.
+        // Warp 2 stores the blocks of the epilogue warps 4-7, warp 3 those of warps 8-11, in their
+        // order: once the four warps have staged a block, one TMA tensor store; once the store
+        // before it has read its buffer, that buffer is released.
         const int half = warp - 2;
-        const int hd = p.d / 2, nblk = hd / kOutCols;
+        const int nb = p.d / 64;
         uint32_t kb = 0;
         bool ok = true;
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters) {
             const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
-            for (int k = 0; k < nblk && ok; ++k, ++kb) {
+            for (int k = 0; k < nb && ok; ++k, ++kb) {
                 const uint32_t b = kb & 1, use = kb >> 1;
                 ok = qwait_warp(bar(bars->st_full[half][b]), use & 1, bars, peer_abort, p.status);
                 if (!ok) break;
                 if (lane == 0) {
-                    ptx::tma_store_3d(&tm_o, sOut + static_cast<uint32_t>((half * 2 + b) * kStageOut),
-                                      half * hd + k * kOutCols, h, tb * kTileTokens + static_cast<int>(cta) * 128);
+                    const int cc = (k < nb / 2 ? 0 : hd) + half * (hd / 2) + (k % (nb / 2)) * kOutCols;
+                    ptx::tma_store_3d(&tm_o, sOut + static_cast<uint32_t>((half * 2 + b) * kStageOut), cc, h,
+                                      tb * kTileTokens + static_cast<int>(cta) * 128);
                     ptx::bulk_commit_group();
                     ptx::bulk_wait_group_read1();  // the previous block's store has read its buffer
                     if (kb > 0) ptx::mbar_arrive(bar(bars->st_empty[half][b ^ 1]));
