@@ -1,4 +1,4 @@
-"""Host model of the attention kernel's shared-memory ring protocol (no GPU).
+"""Host models of the barrier protocols of the attention kernels and the fused prolog q kernel (no GPU).
 
 The attention kernel (mla_prefill_sm100.cuh) streams key tiles through a ring of eight
 16 KB chunks: key tile g, counted per CTA across its work units, occupies chunks
@@ -539,3 +539,252 @@ def test_pair_planted_protocol_mistakes_are_caught(bug):
     with pytest.raises(ProtocolError):
         for trial in range(300):
             simulate_pair(random_units(rng), seed=trial, bug=bug)
+
+
+# ---------------------------------------------------------------------------
+# The fused MLA Prolog q kernel (prolog_q_sm100.cuh)
+# ---------------------------------------------------------------------------
+# Two CTAs (leader 0, follower 1).  Per tile (256 tokens x one head) the stages run N-chunk by
+# N-chunk: chunk c takes k_stages stages of a ring of S slots; the accumulator's two channel halves
+# (tensor memory) have their own barriers.
+#
+#   producer (each CTA)  stage i: waits its own empty(i - S), arms full(i), loads A and chunk c's B
+#   relay (follower)     forwards each of the follower's full barriers to the leader's
+#   MMA (leader)         before chunk c of a tile: waits half_free(h) of the previous tile for each
+#                        half h the chunk writes (first time in the tile); per stage: waits full,
+#                        MMAs, commits empty (both CTAs); after the chunk's last stage commits
+#                        half_full(h) for the halves whose last chunk it is
+#   epilogue half w      (the four warps summing half w's squares, modelled as one role per CTA):
+#                        waits half_full(w), reads half w (pass 1), exchanges with the other half
+#                        (xready), waits half_full(1 - w) (implied by the exchange, whose other side
+#                        waited for it; the kernel waits too, for the tensor-memory ordering of its
+#                        own reads), then per output block: reads its slice of
+#                        the accumulator (first its share of half 0, then of half 1), releasing
+#                        half_free(0) / (1) (leader, both CTAs' roles count) after its last read of
+#                        the half; waits st_empty of the block's buffer, stages it, arrives st_full
+#   store w (each CTA)   per block: waits st_full, issues the store (its read of the buffer happens
+#                        later, at a random point); once every store but the newest has read its
+#                        buffer, arrives the previous buffer's st_empty
+# Tensor-memory halves and staging buffers are tracked: an MMA over a half the previous tile's
+# epilogue still reads, a read of a half before its chunk completed, a staged buffer overwritten
+# before its store read it, or a store of a buffer not yet staged are errors.
+
+
+def simulate_prolog(n_tiles, chunks, halves_of_chunk, last_chunk_of_half, k_stages, blocks_per_half, seed,
+                    slots=6, bug=None):
+    rnd = random.Random(seed)
+    bars = {}
+
+    def mk(kind, cta, i, count=1):
+        bars[kind, cta, i] = Barrier("%s[%d]@%d" % (kind, i, cta), count)
+
+    for cta in range(2):
+        for i in range(slots):
+            mk("full", cta, i, 2 if cta == 0 else 1)
+            mk("empty", cta, i)
+        for h in range(2):
+            mk("half_full", cta, h)
+            mk("xready", cta, h, 2) if h == 0 else None
+            for b in range(2):
+                mk("st_full", cta, 2 * h + b)
+                mk("st_empty", cta, 2 * h + b)
+    for h in range(2):
+        mk("half_free", 0, h, 4)  # both epilogue halves of both CTAs read part of every half
+    owner, readers, landed, tma, mma_queue = {}, {}, set(), [], []
+    acc = {}   # (cta, half) -> ("acc", tile, MMA stages done) | ("read", tile, readers left) | ("free", tile)
+    buf = {}   # (cta, w, b) -> ("staged", block id) | ("free",)
+    stage_order = [(t, c, ks) for t in range(n_tiles) for c in range(chunks) for ks in range(k_stages)]
+
+    def producer(cta):
+        for i, (t, c, ks) in enumerate(stage_order):
+            lag = slots + 1 if bug == "prolog_lag" else slots
+            if i >= slots:
+                while not ready(bars["empty", cta, (i - lag) % slots if bug == "prolog_lag" else i % slots],
+                                (i - slots) // slots):
+                    yield
+            prev = owner.get((cta, i % slots))
+            if prev is not None and readers.get(prev, 0):
+                raise ProtocolError("stage slot %d refilled while an MMA reads %s" % (i % slots, prev))
+            owner[(cta, i % slots)] = (cta, i)
+            tma.append((cta, bars["full", cta, i % slots], (cta, i)))
+            yield
+
+    def relay():
+        for i in range(len(stage_order)):
+            while not ready(bars["full", 1, i % slots], i // slots):
+                yield
+            bars["full", 0, i % slots].arrive()
+            yield
+
+    def mma():
+        i = 0
+        for t in range(n_tiles):
+            waited = set()
+            for c in range(chunks):
+                for h in halves_of_chunk[c]:
+                    if h not in waited and bug != "prolog_no_half_free_wait":
+                        if t >= 1:
+                            while not ready(bars["half_free", 0, h], t - 1):
+                                yield
+                        waited.add(h)
+                for ks in range(k_stages):
+                    while not ready(bars["full", 0, i % slots], i // slots):
+                        yield
+                    for op in ((0, i), (1, i)):
+                        if op not in landed:
+                            raise ProtocolError("MMA reads stage %s before it landed" % (op,))
+                        readers[op] = readers.get(op, 0) + 1
+                    mma_queue.append(("mma", (t, c, (0, i), (1, i))))
+                    mma_queue.append(("commit", [bars["empty", 0, i % slots], bars["empty", 1, i % slots]]))
+                    if ks == k_stages - 1:
+                        for h in halves_of_chunk[c]:
+                            if last_chunk_of_half[h] == c or (bug == "prolog_early_half_full" and h == 1):
+                                mma_queue.append(("commit", [bars["half_full", 0, h], bars["half_full", 1, h]]))
+                    i += 1
+                    yield
+
+    def mma_effect(t, c):
+        for cta in range(2):
+            for h in halves_of_chunk[c]:
+                st = acc.get((cta, h))
+                if st is not None and not (st[0] == "acc" and st[1] == t) and not (st[0] == "free" and st[1] == t - 1):
+                    raise ProtocolError("chunk %d of tile %d writes half %d in state %s" % (c, t, h, st))
+                done = st[2] + 1 if st is not None and st[0] == "acc" and st[1] == t else 1
+                acc[(cta, h)] = ("acc", t, done)
+
+    def epilogue(cta, w):
+        kb = 0
+        for t in range(n_tiles):
+            while not ready(bars["half_full", cta, w], t):
+                yield
+            need = k_stages * sum(1 for c in range(chunks) if w in halves_of_chunk[c])  # MMA stages
+            st = acc.get((cta, w))
+            if st != ("acc", t, need) and not (st is not None and st[0] == "read" and st[1] == t):
+                raise ProtocolError("pass 1 of half %d, tile %d sees %s" % (w, t, st))
+            yield
+            bars["xready", cta, 0].arrive()
+            while not ready(bars["xready", cta, 0], t):
+                yield
+            while not ready(bars["half_full", cta, 1 - w], t):
+                yield
+            for part in (0, 1):  # this role's share of half 0, then of half 1
+                other = acc.get((cta, part))
+                if other is None or other[1] != t or other[0] not in ("acc", "read"):
+                    raise ProtocolError("pass 2 of tile %d reads half %d in state %s" % (t, part, other))
+                if other[0] == "acc":
+                    need_p = k_stages * sum(1 for c in range(chunks) if part in halves_of_chunk[c])
+                    if other[2] != need_p:
+                        raise ProtocolError("pass 2 of tile %d reads half %d before its chunks completed" % (t, part))
+                    acc[(cta, part)] = ("read", t, 2)
+                for _ in range(blocks_per_half):
+                    b = kb & 1
+                    if kb >= 2 and bug != "prolog_no_st_empty_wait":
+                        while not ready(bars["st_empty", cta, 2 * w + b], (kb >> 1) - 1):
+                            yield
+                    if buf.get((cta, w, b), ("free",))[0] == "staged":
+                        raise ProtocolError("staging buffer %s overwritten before its store read it" % ((cta, w, b),))
+                    buf[(cta, w, b)] = ("staged", kb)
+                    bars["st_full", cta, 2 * w + b].arrive()
+                    kb += 1
+                    yield
+                st = acc[(cta, part)]
+                left = st[2] - 1
+                acc[(cta, part)] = ("read", t, left) if left else ("free", t)
+                bars["half_free", 0, part].arrive()
+                yield
+
+    store_reads = []  # TMA stores whose shared-memory read has not happened yet
+
+    def store(cta, w):
+        kb, inflight = 0, []
+        for t in range(n_tiles):
+            for _ in range(2 * blocks_per_half):
+                b = kb & 1
+                while not ready(bars["st_full", cta, 2 * w + b], kb >> 1):
+                    yield
+                if buf.get((cta, w, b)) != ("staged", kb):
+                    raise ProtocolError("store of block %d sees buffer %s" % (kb, buf.get((cta, w, b))))
+                ev = {"buf": (cta, w, b), "block": kb, "done": False}
+                store_reads.append(ev)
+                inflight.append(ev)
+                if bug == "prolog_release_current":
+                    buf[(cta, w, b)] = ("free",)
+                    bars["st_empty", cta, 2 * w + b].arrive()
+                else:
+                    # wait_group.read 1: every store but the newest has read its buffer
+                    while any(not e["done"] for e in inflight[:-1]):
+                        yield
+                    if len(inflight) > 1:
+                        prev = inflight.pop(0)
+                        buf[prev["buf"]] = ("free",)
+                        bars["st_empty", cta, 2 * w + (prev["block"] & 1)].arrive()
+                kb += 1
+                yield
+
+    roles = [producer(0), producer(1), relay(), mma()] + [epilogue(c, w) for c in range(2) for w in range(2)] + \
+        [store(c, w) for c in range(2) for w in range(2)]
+    alive = [True] * len(roles)
+    for _ in range(400000):
+        if not (any(alive) or tma or mma_queue or store_reads):
+            return
+        acts = [("role", i) for i, a in enumerate(alive) if a]
+        if tma:
+            acts.append(("tma", rnd.randrange(len(tma))))
+        if mma_queue:
+            acts.append(("mma", 0))
+        if store_reads:
+            acts.append(("read", rnd.randrange(len(store_reads))))
+        act, arg = rnd.choice(acts)
+        if act == "role":
+            try:
+                next(roles[arg])
+            except StopIteration:
+                alive[arg] = False
+        elif act == "tma":
+            cta, bar, operand = tma.pop(arg)
+            landed.add(operand)
+            bar.arrive()
+        elif act == "read":
+            ev = store_reads.pop(arg)
+            if buf.get(ev["buf"]) != ("staged", ev["block"]):
+                raise ProtocolError("store of block %d reads buffer %s" % (ev["block"], buf.get(ev["buf"])))
+            ev["done"] = True
+        else:
+            op, x = mma_queue.pop(0)
+            if op == "mma":
+                t, c, o0, o1 = x
+                mma_effect(t, c)
+                readers[o0] -= 1
+                readers[o1] -= 1
+            else:
+                for bar in x:
+                    bar.arrive()
+    raise ProtocolError("deadlock")
+
+
+# (chunks, halves each chunk writes, last chunk of each half) for the head sizes the kernel takes
+PROLOG_SHAPES = {
+    512: (2, [[0], [1]], [0, 1]),          # nc = 256: chunk c is half c
+    384: (3, [[0], [0, 1], [1]], [1, 2]),  # nc = 128: the middle chunk straddles the halves
+    256: (1, [[0, 1]], [0, 0]),
+    128: (1, [[0, 1]], [0, 0]),
+}
+
+
+@pytest.mark.parametrize("d", sorted(PROLOG_SHAPES))
+def test_prolog_protocol_holds_under_random_schedules(d):
+    chunks, hoc, loh = PROLOG_SHAPES[d]
+    rng = random.Random(d)
+    for trial in range(60):
+        simulate_prolog(rng.randint(1, 4), chunks, hoc, loh, rng.randint(1, 4), d // 128, seed=trial)
+
+
+@pytest.mark.parametrize("bug", ["prolog_lag", "prolog_no_half_free_wait", "prolog_early_half_full",
+                                 "prolog_release_current", "prolog_no_st_empty_wait"])
+def test_prolog_planted_protocol_mistakes_are_caught(bug):
+    rng = random.Random(3)
+    with pytest.raises(ProtocolError):
+        for trial in range(200):
+            d = rng.choice(sorted(PROLOG_SHAPES))
+            chunks, hoc, loh = PROLOG_SHAPES[d]
+            simulate_prolog(rng.randint(2, 4), chunks, hoc, loh, rng.randint(1, 3), d // 128, seed=trial, bug=bug)
