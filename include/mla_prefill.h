@@ -270,8 +270,11 @@ int mla_paged_cache_load(const mla_tensor *key_cache, const mla_tensor *value_ca
  * block-paged caches through a block table: the composition of the
  * PagedCacheLoadOperation page's gather (ND format, plain lengths, no
  * seqStarts) with the MLA Prefill page's attention, without the packed copy.
- * Its result is bit-identical to mla_paged_cache_load into packed key / value
- * tensors followed by mla_prefill on them.
+ * It runs the single-CTA attention kernel; its result is bit-identical to
+ * mla_paged_cache_load into packed key / value tensors followed by mla_prefill
+ * on them on that kernel (mla_prefill_set_kernel(1); the CTA-pair kernel that
+ * mla_prefill picks by itself for long sequences agrees within the bound, not
+ * bit for bit).
  *
  *   q, q_rope, q_seqlen, kv_seqlen, mask_type, head_num, kv_head_num,
  *   qk_scale, out   exactly as in mla_prefill.
@@ -383,7 +386,9 @@ int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *
 /*
  * mla_prefill_set_kernel -- attention-kernel choice for later mla_prefill,
  * mla_prefill_ws and mla_prefill_noalloc calls on this host thread (no
- * counterpart on the pages; the result is the same operation either way).
+ * counterpart on the pages; the result is the same operation either way, each
+ * within the stated bound of the exact result, the two kernels' bits differing
+ * where their key tiles do).
  *   kernel = -1  automatic (the default): the CTA-pair kernel for packed,
  *                unsplit K/V with long sequences (on average 3072 keys or
  *                more per sequence) once its 512-row work units give at least
@@ -394,7 +399,10 @@ int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *
  *                single-CTA kernel.
  * The CTA-pair kernel runs each 512-row unit on a cluster of two SMs: M = 256
  * tensor-core MMAs across the pair (tcgen05 cta_group::2), each SM loading half
- * of every key tile.  Returns MLA_OK, or MLA_ERR_UNSUPPORTED for other values.
+ * of every 64-key tile, with two score buffers per 256-row group so that the
+ * next tile's scores are computed during the current tile's softmax; the
+ * single-CTA kernel uses 128-key tiles.  Returns MLA_OK, or MLA_ERR_UNSUPPORTED
+ * for other values.
  */
 int mla_prefill_set_kernel(int kernel);
 
