@@ -20,7 +20,10 @@
 // buffer P V_t(j) reads, which the in-order tensor pipe empties first -- so S of the next tile
 // is computed while the softmax still works on the current one: the softmax runs tile after
 // tile without waiting for P V and the next S, and the tensor pipe has the other group's work
-// and this group's next S to fill its time.
+// and this group's next S to fill its time.  The S-full, P-ready and P V-done barriers come in
+// pairs by tile parity: a barrier's next phase then needs the group's next-but-one tile, so no
+// role can fall two phases behind one it waits for, and the softmax waits for P V only when it
+// has to rescale O.
 //
 //   leader   warp 0: TMA loads of its halves; claims work items and hands them to both CTAs
 //            warp 1: MMA issuer for the pair
