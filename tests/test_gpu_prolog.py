@@ -184,6 +184,11 @@ def test_strided_views_and_guards():
     assert mla.prolog_last_fused()
     assert torch.equal(q16, ref_q)
     assert torch.all(qbuf16[:, :, :8] == 5.0) and torch.all(qbuf16[:, :, 8 + d:] == 5.0)
+    # q_out as the page's 2-D [t, H * d] layout
+    q2d = torch.full((t, H * d), 5.0, dtype=torch.bfloat16, device=DEV)
+    run(x, s, q_out=q2d)
+    assert mla.prolog_last_fused()
+    assert torch.equal(q2d.view(t, H, d), ref_q)
 
 
 def test_repeatable():
