@@ -31,8 +31,8 @@ struct DeviceState {
     size_t ws_bytes = 0;
     bool attr_set[32] = {};  // dynamic shared memory opt-in done, per kernel instantiation
     int pair_clusters = 0;   // co-resident clusters of two CTAs of the pair kernel (0: not yet queried)
-    bool prolog_attr = false;  // dynamic shared memory opt-in of the fused q-projection kernel
-    int prolog_clusters = 0;   // its co-resident clusters (0: not yet queried)
+    bool prolog_attr[4] = {};     // dynamic shared memory opt-in of the fused q-projection kernel, per d / 128 - 1
+    int prolog_clusters[4] = {};  // its co-resident clusters (0: not yet queried)
 };
 
 std::mutex g_mu;
@@ -1219,10 +1219,12 @@ int encode_out_map(CUtensorMap *m, const View3 &v) {
 }
 
 // The fused q projection + per-head RmsNorm + RoPE (prolog_q_sm100.cuh): clusters of two CTAs, one
-// per SM, static tiles of 256 tokens x one head.
-int launch_prolog_q(DeviceState *ds, cudaStream_t stream, const CUtensorMap &tm_a, const CUtensorMap &tm_b,
-                    const CUtensorMap &tm_o, const mla::prolog::QParams &qp) {
-    auto kern = mla::prolog::mla_prolog_q_kernel;
+// per SM, static tiles of 256 tokens x one head; one instantiation per head size.
+template <int kD>
+int launch_prolog_q_d(DeviceState *ds, cudaStream_t stream, const CUtensorMap &tm_a, const CUtensorMap &tm_b,
+                      const CUtensorMap &tm_o, const mla::prolog::QParams &qp) {
+    constexpr int di = kD / 128 - 1;
+    auto kern = mla::prolog::mla_prolog_q_kernel<kD>;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(mla::prolog::kThreads);
     cfg.dynamicSmemBytes = mla::prolog::kSmemAlloc;
@@ -1234,24 +1236,35 @@ int launch_prolog_q(DeviceState *ds, cudaStream_t stream, const CUtensorMap &tm_
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (!ds->prolog_attr) {
+    if (!ds->prolog_attr[di]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::prolog::kSmemAlloc) !=
             cudaSuccess)
             return MLA_ERR_CUDA;
-        ds->prolog_attr = true;
+        ds->prolog_attr[di] = true;
     }
-    if (ds->prolog_clusters <= 0) {
+    if (ds->prolog_clusters[di] <= 0) {
         int n = 0;
         cfg.gridDim = dim3(2);
         if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return MLA_ERR_CUDA;
-        ds->prolog_clusters = n;
+        ds->prolog_clusters[di] = n;
     }
     const int64_t tiles = static_cast<int64_t>((qp.tokens + mla::prolog::kTileTokens - 1) / mla::prolog::kTileTokens) *
                           qp.heads;
-    const int64_t clusters = tiles < ds->prolog_clusters ? tiles : ds->prolog_clusters;
+    const int64_t clusters = tiles < ds->prolog_clusters[di] ? tiles : ds->prolog_clusters[di];
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
     if (cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, tm_o, qp) != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;
+}
+
+int launch_prolog_q(DeviceState *ds, cudaStream_t stream, const CUtensorMap &tm_a, const CUtensorMap &tm_b,
+                    const CUtensorMap &tm_o, const mla::prolog::QParams &qp) {
+    switch (qp.d) {
+        case 128: return launch_prolog_q_d<128>(ds, stream, tm_a, tm_b, tm_o, qp);
+        case 256: return launch_prolog_q_d<256>(ds, stream, tm_a, tm_b, tm_o, qp);
+        case 384: return launch_prolog_q_d<384>(ds, stream, tm_a, tm_b, tm_o, qp);
+        case 512: return launch_prolog_q_d<512>(ds, stream, tm_a, tm_b, tm_o, qp);
+        default: return MLA_ERR_UNSUPPORTED;
+    }
 }
 
 int launch_norm(const mla::NormParams &np, int sm_count, cudaStream_t stream) {

@@ -23,14 +23,15 @@
 //
 //   leader   warp 0: TMA loads of its A rows and B halves; warp 1: MMA issuer for the pair
 //   follower warp 0: TMA loads of its halves; warp 1: relay of its full barriers to the leader's
-//   both     warps 4-11: epilogue, two warps per tensor-memory lane quarter: each sums the squares
-//            of one half of the head's d channels of 32 rows, the two sums meet through shared
-//            memory (an mbarrier per lane quarter); then both finish the first half (a quarter of
-//            the head each), release it, and do the second: per 32-column block scale, rotate,
-//            convert and stage
-//            warps 2, 3: TMA stores of the staged blocks of half 0 / 1
+//   both     warps 4-11: epilogue, two warps per tensor-memory lane quarter, each owning a quarter
+//            of the head's d channels of its 32 rows (d/4 columns of each half): it sums their
+//            squares half by half as each half's accumulation completes (64-column tensor-memory
+//            loads issued together), the two warps' sums meet through shared memory (an mbarrier per
+//            lane quarter); then per half, per 64 columns: load, scale (and rotate), convert and
+//            stage two 32-column blocks; a half is released after the warp's last load of it
+//            warps 2, 3: TMA stores of the staged blocks of warps 4-7 / 8-11
 // Tiles are static (tile = cluster + i * clusters, head-major so that concurrent clusters share a
-// head's wq_b columns in L2).
+// head's wq_b columns in L2).  The kernel is instantiated per head size (d = 128, 256, 384, 512).
 // Every wait is bounded; a timeout sets the status word and aborts both CTAs.
 #pragma once
 
@@ -113,6 +114,82 @@ __device__ __forceinline__ void qwait_landed(uint32_t bar, uint32_t parity) {
         if (ptx::globaltimer_ns() - t0 > 100000000ull) return;
 }
 
+// One 32-column output block of a row: scale by the row's norm (two lanes per multiply) and, for
+// kRot, rotate the interleaved pairs by the row's cos / sin values (cs, sn: the block's 32 entries);
+// pack to bf16.
+template <bool kRot>
+__device__ __forceinline__ void scale_block(const uint32_t *cur, float inv, const __nv_bfloat16 *cs,
+                                            const __nv_bfloat16 *sn, uint32_t (&w)[16]) {
+    const float2 inv2 = make_float2(inv, inv);
+    if constexpr (kRot) {
+        uint4 cv[4], sv[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            cv[v] = __ldg(reinterpret_cast<const uint4 *>(cs) + v);
+            sv[v] = __ldg(reinterpret_cast<const uint4 *>(sn) + v);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float2 xy = ptx::fmul2(make_float2(__uint_as_float(cur[2 * e]), __uint_as_float(cur[2 * e + 1])), inv2);
+            const uint32_t cw = reinterpret_cast<const uint32_t *>(&cv[e >> 2])[e & 3];
+            const uint32_t sw = reinterpret_cast<const uint32_t *>(&sv[e >> 2])[e & 3];
+            const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&cw));
+            const float2 s2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&sw));
+            w[e] = DType<__nv_bfloat16>::pack(xy.x * c2.x - xy.y * s2.x, xy.y * c2.y + xy.x * s2.y);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float2 xy = ptx::fmul2(make_float2(__uint_as_float(cur[2 * e]), __uint_as_float(cur[2 * e + 1])), inv2);
+            w[e] = DType<__nv_bfloat16>::pack(xy.x, xy.y);
+        }
+    }
+}
+
+// Sum of squares of kCols consecutive fp32 columns of this warp's 32 lanes (one row per thread),
+// all loads in flight together.
+template <int kCols>
+__device__ __forceinline__ float sum_squares(uint32_t taddr) {
+    static_assert(kCols == 32 || kCols == 64 || kCols == 96 || kCols == 128, "columns per warp and half");
+    float ss = 0.f;
+    auto add = [&](const uint32_t *r, int n) {
+#pragma unroll
+        for (int e = 0; e < n; ++e) {
+            const float v = __uint_as_float(r[e]);
+            ss = fmaf(v, v, ss);
+        }
+    };
+    if constexpr (kCols == 32) {
+        uint32_t a[32];
+        ptx::tmem_ld32(taddr, a);
+        ptx::tmem_wait_ld_dep(a);
+        add(a, 32);
+    } else if constexpr (kCols == 64) {
+        uint32_t a[64];
+        ptx::tmem_ld64(taddr, a);
+        ptx::tmem_wait_ld_dep64(a);
+        add(a, 64);
+    } else if constexpr (kCols == 96) {
+        uint32_t a[64], b[32];
+        ptx::tmem_ld64(taddr, a);
+        ptx::tmem_ld32(taddr + 64, b);
+        ptx::tmem_wait_ld_dep64(a);
+        ptx::tmem_wait_ld_dep(b);
+        add(a, 64);
+        add(b, 32);
+    } else {
+        uint32_t a[64], b[64];
+        ptx::tmem_ld64(taddr, a);
+        ptx::tmem_ld64(taddr + 64, b);
+        ptx::tmem_wait_ld_dep64(a);
+        ptx::tmem_wait_ld_dep64(b);
+        add(a, 64);
+        add(b, 64);
+    }
+    return ss;
+}
+
+template <int kD>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_prolog_q_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_o /* q_out {d, H, tokens} */, const QParams p) {
@@ -162,12 +239,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
+    static_assert(kD % 128 == 0 && kD >= 128 && kD <= 512, "head_dim");
+    constexpr int kNc = kD % 256 == 0 ? 256 : 128;  // MMA N per chunk
+    constexpr int chunk_blocks = kNc / 128;          // this CTA's 8 KB B blocks per stage (one N-chunk)
+    constexpr int chunks = kD / kNc;
+    constexpr int hd = kD / 2;                       // channels per half of the head
     const int n_tblocks = (p.tokens + kTileTokens - 1) / kTileTokens;
     const int n_tiles = n_tblocks * p.heads;
     const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
-    const int chunk_blocks = p.nc / 128;   // this CTA's 8 KB B blocks per stage (one N-chunk)
-    const int chunks = p.d / p.nc;
-    const int hd = p.d / 2;                // channels per half of the head
     const uint32_t stage_tx = kABytes + chunk_blocks * kBBlock;
     // Per tile the stages run N-chunk by N-chunk (all of r for chunk 0, then chunk 1, ...), so the
     // columns of the head's first half are accumulated, and can be handed back by the epilogue,
@@ -195,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::mbar_arrive_expect_tx(fb, stage_tx);
                         ptx::tma_load_2d(dst, &tm_a, fb, ks * kStageK, row0, pol_a);
                         for (int b = 0; b < chunk_blocks; ++b) {
-                            const int col = h * p.d + c * p.nc + static_cast<int>(cta) * (p.nc / 2) + 64 * b;
+                            const int col = h * kD + c * kNc + static_cast<int>(cta) * (kNc / 2) + 64 * b;
                             ptx::tma_load_2d(dst + kABytes + b * kBBlock, &tm_b, fb, col, ks * kStageK, pol_b);
                         }
                     }
@@ -230,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int waited = 0;  // halves whose previous-tile release this tile has waited for
             for (int c = 0; c < chunks && ok; ++c) {
                 // the halves chunk c writes must have been read by the previous tile's epilogue
-                const int h_lo = (c * p.nc) / hd, h_hi = ((c + 1) * p.nc - 1) / hd;
+                const int h_lo = (c * kNc) / hd, h_hi = ((c + 1) * kNc - 1) / hd;
                 for (int hh = h_lo; hh <= h_hi && ok; ++hh)
                     if (!(waited & (1 << hh))) {
                         ok = qwait_warp(bar(bars->half_free[hh]), (tl & 1) ^ 1, bars, peer_abort, p.status);
@@ -238,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 if (!ok) break;
                 ptx::tc_fence_after();
-                const uint32_t d = tmem + static_cast<uint32_t>(c * p.nc);
+                const uint32_t d = tmem + static_cast<uint32_t>(c * kNc);
                 for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
                     const uint32_t s = it % kStages;
                     ok = qwait_warp(bar(bars->full[s]), (it / kStages) & 1, bars, peer_abort, p.status);
@@ -250,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < kStageK / 16; ++k) {
                             // 16 channels of r per MMA: 32 B along A's swizzled rows, 16 rows (2 KB) of B
                             const bool acc = ks > 0 || k > 0;
-                            if (p.nc == 256) {
+                            if constexpr (kNc == 256) {
                                 if (acc) ptx::mma2_ss_lo<kHi, kId256, 1>(d, a + 2 * k, b + 128 * k);
                                 else ptx::mma2_ss_lo<kHi, kId256, 0>(d, a + 2 * k, b + 128 * k);
                             } else {
@@ -261,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::mma_commit_pair(bar(bars->empty[s]), kBoth);  // the stage's operands are read
                         if (ks == p.k_stages - 1)  // halves whose last chunk this is are complete
                             for (int hh = h_lo; hh <= h_hi; ++hh)
-                                if ((hh + 1) * hd <= (c + 1) * p.nc) ptx::mma_commit_pair(bar(bars->half_full[hh]), kBoth);
+                                if ((hh + 1) * hd <= (c + 1) * kNc) ptx::mma_commit_pair(bar(bars->half_full[hh]), kBoth);
                     }
                     __syncwarp();
                 }
@@ -269,93 +348,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- epilogue (both CTAs)
+        constexpr int kQ = hd / 2;         // columns of each half this warp owns (32 .. 128)
+        constexpr int kBlocks = kQ / 32;   // its 32-column output blocks per half
         const int wq = warp & 3;           // tensor-memory lane quarter
-        const int half = (warp - 4) >> 2;  // half of the head summed in the first pass
+        const int part = (warp - 4) >> 2;  // which quarter of each half: columns part * kQ + [0, kQ)
         const int row = wq * 32 + lane;    // row within this CTA's 128
-        const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-        const int c0 = half * hd;
-        const int rope0 = p.d - p.rope;  // first rotated channel
-        const float inv_d = 1.f / static_cast<float>(p.d);
-        const int nb = p.d / 64;         // output blocks of 32 columns per warp and tile (even)
-        uint32_t tl = 0, kb = 0;         // tiles; output blocks staged by this warp's buffers
+        const uint32_t tcol = tmem + (static_cast<uint32_t>(wq * 32) << 16) + static_cast<uint32_t>(part * kQ);
+        const int rope0 = kD - p.rope;     // first rotated channel
+        constexpr float inv_d = 1.f / static_cast<float>(kD);
+        uint32_t tl = 0, kb = 0;           // tiles; output blocks staged by this warp's buffers
         bool ok = true;
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters, ++tl) {
-            const int h = tile / n_tblocks, tb = tile - h * n_tblocks;
+            const int tb = tile % n_tblocks;
             const int token = tb * kTileTokens + static_cast<int>(cta) * 128 + row;
-            ok = qwait_warp(bar(bars->half_full[half]), tl & 1, bars, peer_abort, p.status);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            // sum of squares over this warp's half of the row
-            const uint32_t tA = tmem + lane_addr + static_cast<uint32_t>(c0);
+            // sums of squares over this warp's columns, half by half as each is accumulated
             float ss = 0.f;
-            for (int c = 0; c < hd; c += 32) {
-                uint32_t r[32];
-                ptx::tmem_ld32(tA + c, r);
-                ptx::tmem_wait_ld_dep(r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float v = __uint_as_float(r[e]);
-                    ss = fmaf(v, v, ss);
-                }
+            for (int hh = 0; hh < 2 && ok; ++hh) {
+                ok = qwait_warp(bar(bars->half_full[hh]), tl & 1, bars, peer_abort, p.status);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                ss += sum_squares<kQ>(tcol + static_cast<uint32_t>(hh * hd));
             }
-            // the other half of these rows is summed by the partner warp (same lane quarter)
-            xss[half * 128 + row] = ss;
+            if (!ok) break;
+            // the partner warp (same lane quarter) holds the other two quarters of these rows
+            xss[part * 128 + row] = ss;
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar(bars->xready[wq]));
             ok = qwait_warp(bar(bars->xready[wq]), tl & 1, bars, peer_abort, p.status);
             if (!ok) break;
             const float total = xss[row] + xss[128 + row];
             const float inv = rsqrtf(total * inv_d + p.eps);
-            // the second pass reads both halves (the partner's half too): its accumulation is complete
-            ok = qwait_warp(bar(bars->half_full[half ^ 1]), tl & 1, bars, peer_abort, p.status);
-            if (!ok) break;
-            ptx::tc_fence_after();
             const int tok_c = token < p.tokens ? token : 0;  // rows past the end: any valid cos / sin row
             const __nv_bfloat16 *cs = p.cos + static_cast<long long>(tok_c) * p.cos_tok;
             const __nv_bfloat16 *sn = p.sin + static_cast<long long>(tok_c) * p.sin_tok;
-            // second pass: the two warps of a lane quarter finish the head's first half (each a
-            // quarter of the head), hand it back to the MMA warp, then do the second half.  Per
-            // 32-column block: scale (and rotate), pack to bf16 and stage row `row` in one of this
-            // warp's two 64-byte-swizzled buffers; the store warps write it with TMA.  The next
-            // block's tensor-memory load is issued before this block is processed.
-            auto col_of = [&](int k) { return (k < nb / 2 ? 0 : hd) + half * (hd / 2) + (k % (nb / 2)) * kOutCols; };
-            auto block = [&](int k, const uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
-                const int cc = col_of(k);
-                const bool rot = cc >= rope0;
-                uint4 cv[4], sv[4];
-                if (rot) {
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        cv[v] = __ldg(reinterpret_cast<const uint4 *>(cs + (cc - rope0)) + v);
-                        sv[v] = __ldg(reinterpret_cast<const uint4 *>(sn + (cc - rope0)) + v);
-                    }
-                }
-                if (k == nb / 2 - 1 || k == nb - 1) {  // this warp's last read of a half has completed
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->half_free[k == nb - 1 ? 1 : 0]));
-                }
-                if (k + 1 < nb) ptx::tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(col_of(k + 1)), nxt);
+            // one 32-column block at column cc: scale (and rotate), pack, stage for the store warp
+            auto emit = [&](int cc, const uint32_t *cur) {
                 uint32_t w[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float x = __uint_as_float(cur[2 * e]) * inv, y = __uint_as_float(cur[2 * e + 1]) * inv;
-                    if (rot) {
-                        const uint32_t cw = reinterpret_cast<const uint32_t *>(&cv[e >> 2])[e & 3];
-                        const uint32_t sw = reinterpret_cast<const uint32_t *>(&sv[e >> 2])[e & 3];
-                        const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&cw));
-                        const float2 s2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&sw));
-                        const float x2 = x * c2.x - y * s2.x, y2 = y * c2.y + x * s2.y;
-                        x = x2;
-                        y = y2;
-                    }
-                    w[e] = DType<__nv_bfloat16>::pack(x, y);
-                }
+                if (cc >= rope0) scale_block<true>(cur, inv, cs + (cc - rope0), sn + (cc - rope0), w);
+                else scale_block<false>(cur, inv, cs, sn, w);
                 const uint32_t b = kb & 1, use = kb >> 1;
-                const uint32_t buf = sOut + static_cast<uint32_t>((half * 2 + b) * kStageOut);
+                const uint32_t buf = sOut + static_cast<uint32_t>((part * 2 + b) * kStageOut);
                 // the buffer is free once the store of its previous block has read it
                 if (use > 0 &&
-                    !(ok = qwait_warp(bar(bars->st_empty[half][b]), (use - 1) & 1, bars, peer_abort, p.status)))
+                    !(ok = qwait_warp(bar(bars->st_empty[part][b]), (use - 1) & 1, bars, peer_abort, p.status)))
                     return;
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {  // 16-byte chunk v of the row's 64 bytes, swizzled by (row / 2) mod 4
@@ -366,25 +401,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::fence_proxy_async_smem();  // visible to the TMA store
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(bars->st_full[half][b]));
+                if (lane == 0) ptx::mbar_arrive(bar(bars->st_full[part][b]));
                 ++kb;
-                if (k + 1 < nb) ptx::tmem_wait_ld_dep(nxt);
             };
-            uint32_t r0[32], r1[32];
-            ptx::tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(col_of(0)), r0);
-            ptx::tmem_wait_ld_dep(r0);
-            for (int k = 0; k < nb && ok; k += 2) {
-                block(k, r0, r1);
-                if (ok) block(k + 1, r1, r0);
+            // the warp's last tensor-memory read of half hh has completed: hand the half back
+            auto release = [&](int hh) {
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->half_free[hh]));
+            };
+            // per half, 64 columns (two blocks) per load; half 0 first, as the next tile's first
+            // N-chunk waits for it
+            for (int hh = 0; hh < 2 && ok; ++hh) {
+                const int c0 = hh * hd + part * kQ;
+#pragma unroll
+                for (int j = 0; j < kBlocks; j += 2) {
+                    if (!ok) break;
+                    if (j + 1 < kBlocks) {
+                        uint32_t r[64];
+                        ptx::tmem_ld64(tcol + static_cast<uint32_t>(hh * hd + 32 * j), r);
+                        ptx::tmem_wait_ld_dep64(r);
+                        if (j + 2 >= kBlocks) release(hh);
+                        emit(c0 + 32 * j, r);
+                        if (ok) emit(c0 + 32 * (j + 1), r + 32);
+                    } else {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(tcol + static_cast<uint32_t>(hh * hd + 32 * j), r);
+                        ptx::tmem_wait_ld_dep(r);
+                        release(hh);
+                        emit(c0 + 32 * j, r);
+                    }
+                }
             }
         }
+        ptx::tmem_wait_ld();  // a load left in flight by an aborted tile lands before the columns are freed
     } else if (warp >= 2) {
         // ---------------------------------------------------------------- q stores (both CTAs)
         // Warp 2 stores the blocks of the epilogue warps 4-7, warp 3 those of warps 8-11, in their
         // order: once the four warps have staged a block, one TMA tensor store; once the store
         // before it has read its buffer, that buffer is released.
         const int half = warp - 2;
-        const int nb = p.d / 64;
+        constexpr int nb = kD / 64;
         uint32_t kb = 0;
         bool ok = true;
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters) {

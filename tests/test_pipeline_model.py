@@ -654,44 +654,59 @@ def simulate_prolog(n_tiles, chunks, halves_of_chunk, last_chunk_of_half, k_stag
 
     def epilogue(cta, w):
         kb = 0
-        for t in range(n_tiles):
-            while not ready(bars["half_full", cta, w], t):
-                yield
-            need = k_stages * sum(1 for c in range(chunks) if w in halves_of_chunk[c])  # MMA stages
-            st = acc.get((cta, w))
-            if st != ("acc", t, need) and not (st is not None and st[0] == "read" and st[1] == t):
-                raise ProtocolError("pass 1 of half %d, tile %d sees %s" % (w, t, st))
+
+        def check_read(t, part, what):
+            st = acc.get((cta, part))
+            need = k_stages * sum(1 for c in range(chunks) if part in halves_of_chunk[c])  # MMA stages
+            if st is None or st[1] != t or st[0] not in ("acc", "read") or (st[0] == "acc" and st[2] != need):
+                raise ProtocolError("%s of tile %d reads half %d in state %s" % (what, t, part, st))
+            if st[0] == "acc":
+                acc[(cta, part)] = ("read", t, 2)
+
+        def release(t, part):
+            st = acc[(cta, part)]
+            left = st[2] - 1
+            acc[(cta, part)] = ("read", t, left) if left else ("free", t)
+            bars["half_free", 0, part].arrive()
+
+        def stage():
+            nonlocal kb
+            b = kb & 1
+            if kb >= 2 and bug != "prolog_no_st_empty_wait":
+                while not ready(bars["st_empty", cta, 2 * w + b], (kb >> 1) - 1):
+                    yield
+            if buf.get((cta, w, b), ("free",))[0] == "staged":
+                raise ProtocolError("staging buffer %s overwritten before its store read it" % ((cta, w, b),))
+            buf[(cta, w, b)] = ("staged", kb)
+            bars["st_full", cta, 2 * w + b].arrive()
+            kb += 1
             yield
+
+        for t in range(n_tiles):
+            # pass 1: this role's share of each half, as each half's accumulation completes
+            for part in (0, 1):
+                if not (bug == "prolog_sum_before_full" and part == 1):
+                    while not ready(bars["half_full", cta, part], t):
+                        yield
+                check_read(t, part, "pass 1")
+                yield
             bars["xready", cta, 0].arrive()
             while not ready(bars["xready", cta, 0], t):
                 yield
-            while not ready(bars["half_full", cta, 1 - w], t):
-                yield
-            for part in (0, 1):  # this role's share of half 0, then of half 1
-                other = acc.get((cta, part))
-                if other is None or other[1] != t or other[0] not in ("acc", "read"):
-                    raise ProtocolError("pass 2 of tile %d reads half %d in state %s" % (t, part, other))
-                if other[0] == "acc":
-                    need_p = k_stages * sum(1 for c in range(chunks) if part in halves_of_chunk[c])
-                    if other[2] != need_p:
-                        raise ProtocolError("pass 2 of tile %d reads half %d before its chunks completed" % (t, part))
-                    acc[(cta, part)] = ("read", t, 2)
-                for _ in range(blocks_per_half):
-                    b = kb & 1
-                    if kb >= 2 and bug != "prolog_no_st_empty_wait":
-                        while not ready(bars["st_empty", cta, 2 * w + b], (kb >> 1) - 1):
-                            yield
-                    if buf.get((cta, w, b), ("free",))[0] == "staged":
-                        raise ProtocolError("staging buffer %s overwritten before its store read it" % ((cta, w, b),))
-                    buf[(cta, w, b)] = ("staged", kb)
-                    bars["st_full", cta, 2 * w + b].arrive()
-                    kb += 1
-                    yield
-                st = acc[(cta, part)]
-                left = st[2] - 1
-                acc[(cta, part)] = ("read", t, left) if left else ("free", t)
-                bars["half_free", 0, part].arrive()
-                yield
+            # pass 2: per half, loads of two blocks; the half goes back after the role's last load of it
+            loads = (blocks_per_half + 1) // 2
+            for part in (0, 1):
+                for i in range(loads):
+                    last = i == loads - 1
+                    if last and bug == "prolog_release_before_last_load":
+                        release(t, part)
+                        yield
+                    check_read(t, part, "pass 2")
+                    if last and bug != "prolog_release_before_last_load":
+                        release(t, part)
+                    for _ in range(min(2, blocks_per_half - 2 * i)):
+                        yield from stage()
+            yield
 
     store_reads = []  # TMA stores whose shared-memory read has not happened yet
 
@@ -780,7 +795,8 @@ def test_prolog_protocol_holds_under_random_schedules(d):
 
 
 @pytest.mark.parametrize("bug", ["prolog_lag", "prolog_no_half_free_wait", "prolog_early_half_full",
-                                 "prolog_release_current", "prolog_no_st_empty_wait"])
+                                 "prolog_release_current", "prolog_no_st_empty_wait", "prolog_sum_before_full",
+                                 "prolog_release_before_last_load"])
 def test_prolog_planted_protocol_mistakes_are_caught(bug):
     rng = random.Random(3)
     with pytest.raises(ProtocolError):
