@@ -24,11 +24,13 @@
 //   leader   warp 0: TMA loads of its A rows and B halves; warp 1: MMA issuer for the pair
 //   follower warp 0: TMA loads of its halves; warp 1: relay of its full barriers to the leader's
 //   both     warps 4-11: epilogue, two warps per tensor-memory lane quarter, each owning a quarter
-//            of the head's d channels of its 32 rows (d/4 columns of each half): it sums their
-//            squares half by half as each half's accumulation completes (64-column tensor-memory
-//            loads issued together), the two warps' sums meet through shared memory (an mbarrier per
-//            lane quarter); then per half, per 64 columns: load, scale (and rotate), convert and
-//            stage two 32-column blocks; a half is released after the warp's last load of it
+//            of the head's d channels of its 32 rows (d/4 columns of each half).  Once half 0 is
+//            accumulated the warp copies its columns into registers and hands the half back at
+//            once, so the next tile's first N-chunk runs during the rest of the epilogue; once half
+//            1 is accumulated it adds that half's squares, the two warps' sums meet through shared
+//            memory (an mbarrier per lane quarter), and it scales (and rotates), converts and
+//            stages 32-column blocks: half 0 from registers, half 1 from tensor memory (64 columns
+//            per load), releasing half 1 after its last load
 //            warps 2, 3: TMA stores of the staged blocks of warps 4-7 / 8-11
 // Tiles are static (tile = cluster + i * clusters, head-major so that concurrent clusters share a
 // head's wq_b columns in L2).  The kernel is instantiated per head size (d = 128, 256, 384, 512).
@@ -58,6 +60,13 @@ constexpr int kSmemBytes = kSmemXss + 2 * 128 * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 constexpr int kEpiWarps = 8;
+// warpgroup 0 (producer, MMA issuer / relay, store warps) gives registers to the two epilogue
+// warpgroups, which hold their columns of half 0 (up to 128 per thread) across the second half's
+// accumulation; the split stays within the 168 registers per thread the block is launched with
+constexpr int kRegsLow = 72;
+constexpr int kRegsEpi = 216;
+static_assert(kRegsLow * 128 + kRegsEpi * 256 <= 65536 / kThreads / 8 * 8 * kThreads,
+              "register split exceeds the launch's register file share");
 constexpr int kHalfFreeArrivals = 2 * kEpiWarps;  // every epilogue warp of both CTAs reads part of each half
 constexpr uint64_t kWaitLimitNs = 200000000ull;   // 200 ms
 
@@ -146,49 +155,6 @@ __device__ __forceinline__ void scale_block(const uint32_t *cur, float inv, cons
     }
 }
 
-// Sum of squares of kCols consecutive fp32 columns of this warp's 32 lanes (one row per thread),
-// all loads in flight together.
-template <int kCols>
-__device__ __forceinline__ float sum_squares(uint32_t taddr) {
-    static_assert(kCols == 32 || kCols == 64 || kCols == 96 || kCols == 128, "columns per warp and half");
-    float ss = 0.f;
-    auto add = [&](const uint32_t *r, int n) {
-#pragma unroll
-        for (int e = 0; e < n; ++e) {
-            const float v = __uint_as_float(r[e]);
-            ss = fmaf(v, v, ss);
-        }
-    };
-    if constexpr (kCols == 32) {
-        uint32_t a[32];
-        ptx::tmem_ld32(taddr, a);
-        ptx::tmem_wait_ld_dep(a);
-        add(a, 32);
-    } else if constexpr (kCols == 64) {
-        uint32_t a[64];
-        ptx::tmem_ld64(taddr, a);
-        ptx::tmem_wait_ld_dep64(a);
-        add(a, 64);
-    } else if constexpr (kCols == 96) {
-        uint32_t a[64], b[32];
-        ptx::tmem_ld64(taddr, a);
-        ptx::tmem_ld32(taddr + 64, b);
-        ptx::tmem_wait_ld_dep64(a);
-        ptx::tmem_wait_ld_dep(b);
-        add(a, 64);
-        add(b, 32);
-    } else {
-        uint32_t a[64], b[64];
-        ptx::tmem_ld64(taddr, a);
-        ptx::tmem_ld64(taddr + 64, b);
-        ptx::tmem_wait_ld_dep64(a);
-        ptx::tmem_wait_ld_dep64(b);
-        add(a, 64);
-        add(b, 64);
-    }
-    return ss;
-}
-
 template <int kD>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_prolog_q_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -253,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // before those of its second half.
     const int stages_per_tile = chunks * p.k_stages;
 
+    if (warp < 4) ptx::regs_dec<kRegsLow>();
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -348,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {
         // ---------------------------------------------------------------- epilogue (both CTAs)
+        ptx::regs_inc<kRegsEpi>();
         constexpr int kQ = hd / 2;         // columns of each half this warp owns (32 .. 128)
         constexpr int kBlocks = kQ / 32;   // its 32-column output blocks per half
         const int wq = warp & 3;           // tensor-memory lane quarter
@@ -361,13 +329,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tile = cluster_id; tile < n_tiles && ok; tile += n_clusters, ++tl) {
             const int tb = tile % n_tblocks;
             const int token = tb * kTileTokens + static_cast<int>(cta) * 128 + row;
-            // sums of squares over this warp's columns, half by half as each is accumulated
+            // half 0: this warp's columns into registers, and the half goes straight back to the MMA warp
+            uint32_t keep[kQ];
             float ss = 0.f;
-            for (int hh = 0; hh < 2 && ok; ++hh) {
-                ok = qwait_warp(bar(bars->half_full[hh]), tl & 1, bars, peer_abort, p.status);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                ss += sum_squares<kQ>(tcol + static_cast<uint32_t>(hh * hd));
+            ok = qwait_warp(bar(bars->half_full[0]), tl & 1, bars, peer_abort, p.status);
+            if (!ok) break;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < kQ; j += 32)
+                ptx::tmem_ld32(tcol + static_cast<uint32_t>(j), *reinterpret_cast<uint32_t (*)[32]>(keep + j));
+#pragma unroll
+            for (int j = 0; j < kQ; j += 32) ptx::tmem_wait_ld_dep(*reinterpret_cast<uint32_t (*)[32]>(keep + j));
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->half_free[0]));
+#pragma unroll
+            for (int e = 0; e < kQ; ++e) ss = fmaf(__uint_as_float(keep[e]), __uint_as_float(keep[e]), ss);
+            // half 1: the squares of this warp's columns, 32 per load (the held half leaves few registers)
+            ok = qwait_warp(bar(bars->half_full[1]), tl & 1, bars, peer_abort, p.status);
+            if (!ok) break;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int j = 0; j < kQ; j += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tcol + static_cast<uint32_t>(hd + j), r);
+                ptx::tmem_wait_ld_dep(r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(r[e]), __uint_as_float(r[e]), ss);
             }
             if (!ok) break;
             // the partner warp (same lane quarter) holds the other two quarters of these rows
@@ -404,33 +392,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) ptx::mbar_arrive(bar(bars->st_full[part][b]));
                 ++kb;
             };
-            // the warp's last tensor-memory read of half hh has completed: hand the half back
-            auto release = [&](int hh) {
+            // the warp's last tensor-memory read of half 1 has completed: hand the half back
+            auto release1 = [&]() {
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->half_free[hh]));
+                if (lane == 0) ptx::mbar_arrive_remote(lead_bar(bars->half_free[1]));
             };
-            // per half, 64 columns (two blocks) per load; half 0 first, as the next tile's first
-            // N-chunk waits for it
-            for (int hh = 0; hh < 2 && ok; ++hh) {
-                const int c0 = hh * hd + part * kQ;
+            // half 0 from registers
 #pragma unroll
-                for (int j = 0; j < kBlocks; j += 2) {
-                    if (!ok) break;
-                    if (j + 1 < kBlocks) {
-                        uint32_t r[64];
-                        ptx::tmem_ld64(tcol + static_cast<uint32_t>(hh * hd + 32 * j), r);
-                        ptx::tmem_wait_ld_dep64(r);
-                        if (j + 2 >= kBlocks) release(hh);
-                        emit(c0 + 32 * j, r);
-                        if (ok) emit(c0 + 32 * (j + 1), r + 32);
-                    } else {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(tcol + static_cast<uint32_t>(hh * hd + 32 * j), r);
-                        ptx::tmem_wait_ld_dep(r);
-                        release(hh);
-                        emit(c0 + 32 * j, r);
-                    }
+            for (int j = 0; j < kBlocks; ++j)
+                if (ok) emit(part * kQ + 32 * j, keep + 32 * j);
+            // half 1 from tensor memory, 64 columns (two blocks) per load
+            const int c1 = hd + part * kQ;
+#pragma unroll
+            for (int j = 0; j < kBlocks; j += 2) {
+                if (!ok) break;
+                if (j + 1 < kBlocks) {
+                    uint32_t r[64];
+                    ptx::tmem_ld64(tcol + static_cast<uint32_t>(hd + 32 * j), r);
+                    ptx::tmem_wait_ld_dep64(r);
+                    if (j + 2 >= kBlocks) release1();
+                    emit(c1 + 32 * j, r);
+                    if (ok) emit(c1 + 32 * (j + 1), r + 32);
+                } else {
+                    uint32_t r[32];
+                    ptx::tmem_ld32(tcol + static_cast<uint32_t>(hd + 32 * j), r);
+                    ptx::tmem_wait_ld_dep(r);
+                    release1();
+                    emit(c1 + 32 * j, r);
                 }
             }
         }

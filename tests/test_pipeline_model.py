@@ -683,29 +683,41 @@ def simulate_prolog(n_tiles, chunks, halves_of_chunk, last_chunk_of_half, k_stag
             yield
 
         for t in range(n_tiles):
-            # pass 1: this role's share of each half, as each half's accumulation completes
-            for part in (0, 1):
-                if not (bug == "prolog_sum_before_full" and part == 1):
-                    while not ready(bars["half_full", cta, part], t):
-                        yield
-                check_read(t, part, "pass 1")
+            # half 0: this role's columns copied into registers, the half handed back at once
+            while not ready(bars["half_full", cta, 0], t):
                 yield
+            if bug == "prolog_release_before_copy":
+                release(t, 0)
+                yield
+                check_read(t, 0, "copy")
+            else:
+                check_read(t, 0, "copy")
+                yield
+                release(t, 0)
+            yield
+            # half 1: the squares of this role's columns
+            if bug != "prolog_sum_before_full":
+                while not ready(bars["half_full", cta, 1], t):
+                    yield
+            check_read(t, 1, "pass 1")
+            yield
             bars["xready", cta, 0].arrive()
             while not ready(bars["xready", cta, 0], t):
                 yield
-            # pass 2: per half, loads of two blocks; the half goes back after the role's last load of it
+            for _ in range(blocks_per_half):  # half 0 from registers
+                yield from stage()
+            # half 1, two blocks per load; the half goes back after the role's last load of it
             loads = (blocks_per_half + 1) // 2
-            for part in (0, 1):
-                for i in range(loads):
-                    last = i == loads - 1
-                    if last and bug == "prolog_release_before_last_load":
-                        release(t, part)
-                        yield
-                    check_read(t, part, "pass 2")
-                    if last and bug != "prolog_release_before_last_load":
-                        release(t, part)
-                    for _ in range(min(2, blocks_per_half - 2 * i)):
-                        yield from stage()
+            for i in range(loads):
+                last = i == loads - 1
+                if last and bug == "prolog_release_before_last_load":
+                    release(t, 1)
+                    yield
+                check_read(t, 1, "pass 2")
+                if last and bug != "prolog_release_before_last_load":
+                    release(t, 1)
+                for _ in range(min(2, blocks_per_half - 2 * i)):
+                    yield from stage()
             yield
 
     store_reads = []  # TMA stores whose shared-memory read has not happened yet
@@ -796,7 +808,7 @@ def test_prolog_protocol_holds_under_random_schedules(d):
 
 @pytest.mark.parametrize("bug", ["prolog_lag", "prolog_no_half_free_wait", "prolog_early_half_full",
                                  "prolog_release_current", "prolog_no_st_empty_wait", "prolog_sum_before_full",
-                                 "prolog_release_before_last_load"])
+                                 "prolog_release_before_last_load", "prolog_release_before_copy"])
 def test_prolog_planted_protocol_mistakes_are_caught(bug):
     rng = random.Random(3)
     with pytest.raises(ProtocolError):
