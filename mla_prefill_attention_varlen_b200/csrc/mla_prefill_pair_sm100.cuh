@@ -318,10 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                static_cast<uint32_t>(it));
                     ptx::mbar_arrive(bar(bars->sched_full[slot]));
                     ptx::mbar_arrive_cluster(ptx::mapa_shared(bar(bars->sched_full[slot]), 1));
-                    if (it >= 0) {
-                        next = n_clusters + atomicAdd(p.work_counter, 1);
-                        if (next >= n_items) next = -1;
-                    }
                 } else {
                     ok = wait_pair<true>(bar(bars->sched_full[slot]), (sc / kSched) & 1, bars, peer_abort, p.status);
                     if (!ok) break;
@@ -330,8 +326,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ++sc;
                 if (it < 0) break;
+                // The leader claims the next item when the loads of this one's last key tile are
+                // about to be issued (claimed at an item's start, a pair that drew a long item would
+                // also take the next item of the longest-first list from pairs that free up sooner).
+                auto claim = [&]() {
+                    if (leader) {
+                        next = n_clusters + atomicAdd(p.work_counter, 1);
+                        if (next >= n_items) next = -1;
+                    }
+                };
                 const Item x = decode(p, it, num_units, kCausal, cta);
-                if (x.n_max == 0) continue;
+                if (x.n_max == 0) {
+                    claim();
+                    continue;
+                }
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     if (!ok || x.n[t] == 0) continue;
@@ -348,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++ql;
                 }
                 for (int j = 0; j < x.n_max && ok; ++j) {
+                    if (j == x.n_max - 1) claim();
                     const int tok = x.k_tok0 + j * kKeys;
                     const uint32_t g = tk, slot = g % kSlots, phase = ((g / kSlots) & 1) ^ 1;
                     const uint32_t dst = sRing + slot * kSlotBytes;

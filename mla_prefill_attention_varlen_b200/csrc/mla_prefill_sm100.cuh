@@ -604,7 +604,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 };
                 // Dynamic scheduling: the first item is blockIdx.x, later ones come from a global
                 // counter; each claimed item index (or -1 at the end) is handed to the MMA and
-                // softmax warps through a small ring in shared memory.
+                // softmax warps through a small ring in shared memory.  The next item is claimed
+                // when the loads of the current one's last key tile are about to be issued, about
+                // one key tile before this CTA runs out of work: claimed at an item's start, a
+                // CTA that drew a long item would also take the next item of the longest-first
+                // list from CTAs that free up sooner.
                 uint32_t sc = 0;
                 int next = blockIdx.x < n_items ? (int)blockIdx.x : -1;
                 while (ok) {
@@ -618,13 +622,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ++sc;
                     if (it < 0) break;
-                    if (lead) {
-                        next = (int)gridDim.x + atomicAdd(p.work_counter, 1);
-                        if (next >= n_items) next = -1;
-                    }
-                    if (kW) next = __shfl_sync(0xffffffffu, next, 0);
+                    auto claim = [&]() {
+                        if (lead) {
+                            next = (int)gridDim.x + atomicAdd(p.work_counter, 1);
+                            if (next >= n_items) next = -1;
+                        }
+                        if (kW) next = __shfl_sync(0xffffffffu, next, 0);
+                    };
                     const WorkItem x = decode_item<kGeneral>(p, it, num_entries, kCausal);
-                    if (x.n_max == 0) continue;
+                    if (x.n_max == 0) {
+                        claim();
+                        continue;
+                    }
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         if (!ok || x.n[t] == 0) continue;
@@ -670,6 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int nk = kBN / p.rows_k, nv = 64 / p.rows_v;
                         int id_next = raw_id(x.j0);
                         for (int jl = 0; jl < x.n_max && ok; ++jl) {
+                            if (jl == x.n_max - 1) claim();
                             const int j = x.j0 + jl;  // absolute key tile
                             int id = id_next;
                             if (jl + 1 < x.n_max) id_next = raw_id(j + 1);  // in flight during tile j
@@ -693,6 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     } else {
                         for (int jl = 0; jl < x.n_max && ok; ++jl) {
+                            if (jl == x.n_max - 1) claim();
                             const int tok = x.k_tok0 + (x.j0 + jl) * kBN;
                             const uint32_t g = tk, c0 = 5 * g;
                             uint32_t fb;
