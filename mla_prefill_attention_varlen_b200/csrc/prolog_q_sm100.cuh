@@ -357,7 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(r[e]), __uint_as_float(r[e]), ss);
             }
-            if (!ok) break;
             // the partner warp (same lane quarter) holds the other two quarters of these rows
             xss[part * 128 + row] = ss;
             __syncwarp();
