@@ -54,14 +54,18 @@ def algorithmic_bytes(wl):
 KERNEL_SOURCES = ["mla_prefill_attention_varlen_b200/csrc/mla_prefill_sm100.cuh",
                   "mla_prefill_attention_varlen_b200/csrc/mla_prefill_pair_sm100.cuh",
                   "mla_prefill_attention_varlen_b200/csrc/sm100_ptx.cuh"]
+# the fused MLA Prolog q kernel (its traffic entry in profiles/traffic.json is keyed on these)
+PROLOG_Q_SOURCES = ["mla_prefill_attention_varlen_b200/csrc/prolog_q_sm100.cuh",
+                    "mla_prefill_attention_varlen_b200/csrc/mla_prefill_sm100.cuh",
+                    "mla_prefill_attention_varlen_b200/csrc/sm100_ptx.cuh"]
 
 
-def kernel_sources_hash():
+def kernel_sources_hash(sources=None):
     """sha256 over the device-code sources (a measured traffic figure is only valid for this code)."""
     import hashlib
 
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -71,7 +75,7 @@ def kernel_sources_hash():
 KERNEL_NAMES = {1: "mla_prefill_sm100_kernel", 2: "mla_prefill_pair_kernel"}
 
 
-def measured_traffic(workload):
+def measured_traffic(workload, sources=None):
     """DRAM bytes per launch from the committed ncu figures (profiles/traffic.json), or None when
     there is no figure for this workload or it was taken on different kernel sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -79,7 +83,7 @@ def measured_traffic(workload):
         return None
     with open(path) as f:
         entry = json.load(f).get("launches", {}).get(workload)
-    if not entry or entry.get("kernel_sources_sha256") != kernel_sources_hash():
+    if not entry or entry.get("kernel_sources_sha256") != kernel_sources_hash(sources):
         return None
     try:
         return int(entry["traffic_bytes_per_launch"])
@@ -525,7 +529,8 @@ def bench_prolog(args):
                        (in_bytes + q.numel() * 2) / 1e9),
                    "q_path": "fused tcgen05 q kernel" if fused else "library GEMM + row kernel"},
         "roofline": ({"bound": "tensor", "achieved": q_flops / (kms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
-                      "frac": q_flops / (kms * 1e-3) / 1e12 / peak, "traffic": None, "peak_source": peak_src,
+                      "frac": q_flops / (kms * 1e-3) / 1e12 / peak,
+                      "traffic": measured_traffic("prolog_q_%d" % t, PROLOG_Q_SOURCES), "peak_source": peak_src,
                       "kernel": "mla_prolog_q_kernel (q projection + per-head RmsNorm + RoPE)", "kernel_ms": kms,
                       "algorithmic_flops_per_launch": q_flops, "algorithmic_bytes_per_launch": q_bytes,
                       "hbm_achieved_gbs": q_bytes / (kms * 1e-3) / 1e9, "step_tensor_frac": value / world / peak}
