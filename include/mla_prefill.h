@@ -391,13 +391,15 @@ int mla_prefill_set_profile_events(struct CUevent_st *start, struct CUevent_st *
  * where their key tiles do).
  *   kernel = -1  automatic (the default): the CTA-pair kernel for packed,
  *                unsplit K/V with long sequences (on average 3072 keys or
- *                more per sequence) once its 512-row work units give at least
+ *                more per sequence) once its work units (512 rows of one head,
+ *                or 256 rows of two query heads sharing a kv head when each
+ *                kv head serves an even number of query heads) give at least
  *                one work item per SM pair, else the single-CTA kernel;
  *   kernel =  1  the single-CTA kernel (256-row units, one SM each);
  *   kernel =  2  the CTA-pair kernel wherever it applies (packed K/V without
  *                split-KV); padded or paged K/V and split-KV always run the
  *                single-CTA kernel.
- * The CTA-pair kernel runs each 512-row unit on a cluster of two SMs: M = 256
+ * The CTA-pair kernel runs each unit on a cluster of two SMs: M = 256
  * tensor-core MMAs across the pair (tcgen05 cta_group::2), each SM loading half
  * of every 64-key tile, with two score buffers per 256-row group so that the
  * next tile's scores are computed during the current tile's softmax; the

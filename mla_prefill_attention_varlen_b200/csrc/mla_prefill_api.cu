@@ -432,8 +432,13 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
     // average 3072 keys or more per sequence), where a 512-row unit walks many key tiles; short
     // units (a few key tiles each) run faster on the single-CTA kernel, whose per-unit start and
     // end cost less.  Either needs at least one work item per SM pair to pay off.
-    const int64_t pair_items = ((pr.q.tokens + mla::pair::kUnitRows - 1) / mla::pair::kUnitRows + pr.batch) *
-                               pr.head_num;
+    // With an even number of query heads per kv head the pair kernel's two groups take two heads of
+    // one kv head over the same 256 rows (both walk the same key tiles); else 512 rows of one head,
+    // whose first 256 rows see fewer keys than the second.
+    const bool head_pair = (pr.head_num / pr.kv_head_num) % 2 == 0;
+    const int64_t pair_unit_rows = head_pair ? mla::pair::kGroupRows : mla::pair::kUnitRows;
+    const int64_t pair_items = ((pr.q.tokens + pair_unit_rows - 1) / pair_unit_rows + pr.batch) *
+                               (head_pair ? pr.head_num / 2 : pr.head_num);
     const bool long_keys = pr.batch > 0 && pr.k.tokens >= 3072 * pr.batch;
     const bool use_pair = !general && pair_items > 0 &&
                           (t_kernel == 2 || (t_kernel < 0 && long_keys && pair_items >= sm_count / 2));
@@ -473,7 +478,7 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
         pr.q_seqlen, pr.kv_seqlen, static_cast<int>(pr.batch), pr.q.tokens, pr.k.tokens, pr.kv_pad,
         pr.paged ? 1 : 0, pr.causal ? 1 : 0, seq_info, unit_off, hist, lay.hist_len, units, num_units, work_counter,
         lay.split_tiles, split_off, entry_tab, num_entries, status, reset_status ? 1 : 0,
-        use_pair ? mla::pair::kUnitRows : mla::kUnitRows);
+        use_pair ? static_cast<int>(pair_unit_rows) : mla::kUnitRows);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
 
     mla::Params p;
@@ -489,6 +494,7 @@ int enqueue(const Problem &pr, const WsLayout &lay, uint8_t *ws, int *status, in
                (pr.o.st_head * 2) % 32 == 0;
     p.head_num = pr.head_num;
     p.group = pr.head_num / pr.kv_head_num;
+    p.head_pair = use_pair && head_pair ? 1 : 0;
     // unit-major (longest-first) item order when all of K, K_rope and V fit in 48 MB of the L2
     p.lpt = !pr.paged && pr.k.tokens * pr.kv_head_num * (2 * mla::kDn + mla::kDr) * 2 <= (int64_t(48) << 20);
     p.scale_log2 = pr.qk_scale * 1.4426950408889634f;

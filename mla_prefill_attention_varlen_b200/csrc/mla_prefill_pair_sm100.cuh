@@ -8,7 +8,11 @@
 //
 // Two CTAs of a cluster (ranks 0 and 1, "leader" and "follower", on two SMs) share one work
 // unit: 512 query rows of one sequence for one query head, in two groups t = 0, 1 of 256 rows
-// (rows u0 + 256 t + [0, 128) in the leader, the next 128 in the follower).  The leader's MMA
+// (rows u0 + 256 t + [0, 128) in the leader, the next 128 in the follower); or, when every kv
+// head serves an even number of query heads, 256 rows for two query heads h, h + 1 of one kv head,
+// group t taking head h + t over the same rows (head pairs: both groups walk the same key tiles,
+// where the two halves of a 512-row unit differ by four, and the last unit of a sequence may leave
+// its second group empty).  The leader's MMA
 // warp issues M = 256 tensor-core MMAs over the pair (tcgen05 cta_group::2): each CTA's tensor
 // memory receives its own 128 rows, the A operand (Q or P) comes from each CTA's own shared or
 // tensor memory, and the B operand (K for S, V for P V) is split along N: each CTA loads only
@@ -134,7 +138,8 @@ __device__ __forceinline__ void wait_landed(uint32_t bar, uint32_t parity) {
 }
 
 struct Item {
-    int h, kh;
+    int h, kh;           // query head of group 0 (group t runs head h + t * dh) and its kv head
+    int dh, drow;        // head and row steps from group 0 to group 1: (0, 256), or (1, 0) for head pairs
     int u0;              // first query row of the unit within its sequence
     int q_tok0, k_tok0;  // first packed token of the unit / of the sequence's keys
     int lq, lk, off;     // off = Lk - Lq
@@ -151,15 +156,30 @@ __device__ __forceinline__ int key_tiles(int q0, int rows, int lq, int lk, bool 
     return kv_end > 0 ? (kv_end + kKeys - 1) / kKeys : 0;
 }
 
-// Items are ordered as in the single-CTA kernel (kv-head-major, or unit-major when K/V fits in L2).
+// Items are ordered as in the single-CTA kernel (kv-head-major, or unit-major when K/V fits in L2),
+// over heads or, with p.head_pair, over pairs of heads (2j, 2j + 1) of one kv head.
 __device__ __forceinline__ Item decode(const Params &p, int it, int num_units, bool causal, uint32_t cta) {
     Item x;
-    int e;
-    item_unit_head(p, it, num_units, e, x.h);
+    const int hp = p.head_pair;
+    const int hn = p.head_num >> hp, gr = p.group >> hp;  // heads (pairs) in all and per kv head
+    int e, h;
+    if (p.lpt) {
+        e = it / hn;
+        h = it - e * hn;
+    } else {
+        const int per_kh = num_units * gr;
+        const int kh = it / per_kh;
+        const int rem = it - kh * per_kh;
+        e = rem / gr;
+        h = kh * gr + (rem - e * gr);
+    }
+    x.h = h << hp;
     x.kh = x.h / p.group;
+    x.dh = hp;
+    x.drow = hp ? 0 : kGroupRows;
     const int2 bm = p.units[e];
     const int4 s = p.seq_info[bm.x];
-    x.u0 = bm.y * kUnitRows;
+    x.u0 = bm.y * (hp ? kGroupRows : kUnitRows);
     x.q_tok0 = s.x + x.u0;
     x.k_tok0 = s.y;
     x.lq = s.z;
@@ -167,7 +187,7 @@ __device__ __forceinline__ Item decode(const Params &p, int it, int num_units, b
     x.off = s.w - s.z;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        const int r0 = x.u0 + t * kGroupRows, r1 = r0 + kBM;
+        const int r0 = x.u0 + t * x.drow, r1 = r0 + kBM;
         const int n0 = key_tiles(r0, tile_rows(r0, s.z), s.z, s.w, causal);
         const int n1 = key_tiles(r1, tile_rows(r1, s.z), s.z, s.w, causal);
         x.n[t] = max(n0, n1);
@@ -278,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     ptx::griddep_wait();  // the plan kernel's work list is complete and visible
     const int num_units = *p.num_units;
-    const int n_items = num_units * p.head_num;
+    const int n_items = num_units * (p.head_num >> p.head_pair);
     const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
 
     // Work-item hand-off, consumer side: returns the item of ring slot sc (-1: no more work).
@@ -348,11 +368,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) continue;
                     const uint32_t fb = bar(bars->q_full[t]);
                     const uint32_t dst = sQ + t * kQTileBytes;
-                    const int tok = x.q_tok0 + t * kGroupRows + static_cast<int>(cta) * kBM;
+                    const int tok = x.q_tok0 + t * x.drow + static_cast<int>(cta) * kBM;
+                    const int qh = x.h + t * x.dh;
                     ptx::mbar_arrive_expect_tx(fb, kQTileBytes);
-                    ptx::tma_load_3d(dst, &tm_q, fb, 0, x.h, tok, pol_q);
-                    ptx::tma_load_3d(dst + 16384, &tm_q, fb, 64, x.h, tok, pol_q);
-                    ptx::tma_load_3d(dst + 32768, &tm_qr, fb, 0, x.h, tok, pol_q);
+                    ptx::tma_load_3d(dst, &tm_q, fb, 0, qh, tok, pol_q);
+                    ptx::tma_load_3d(dst + 16384, &tm_q, fb, 64, qh, tok, pol_q);
+                    ptx::tma_load_3d(dst + 32768, &tm_qr, fb, 0, qh, tok, pol_q);
                     ++ql;
                 }
                 for (int j = 0; j < x.n_max && ok; ++j) {
@@ -587,11 +608,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item x = decode(p, it, num_units, kCausal, cta);
             const int n_t = x.n[t];
             const bool row_valid = row < x.rows[t];
-            const int tile_q0 = x.u0 + t * kGroupRows + static_cast<int>(cta) * kBM;
+            const int tile_q0 = x.u0 + t * x.drow + static_cast<int>(cta) * kBM;
             const int i = tile_q0 + row;  // query row within the sequence
-            T *orow = reinterpret_cast<T *>(p.out) + (long long)(x.q_tok0 + t * kGroupRows +
+            T *orow = reinterpret_cast<T *>(p.out) + (long long)(x.q_tok0 + t * x.drow +
                                                                  static_cast<int>(cta) * kBM + row) * p.out_st +
-                      (long long)x.h * p.out_sh;
+                      (long long)(x.h + t * x.dh) * p.out_sh;
             if (n_t == 0) {  // no key visible to any row of the group: no MMA runs for it
                 if (row_valid) {
                     const uint4 z = make_uint4(0, 0, 0, 0);

@@ -92,6 +92,8 @@ struct Params {
     int head_num;
     int group;         // head_num / kv_head_num
     int lpt;           // 1: items unit-major (longest first across all heads); 0: kv-head-major
+    int head_pair;     // CTA-pair kernel only: 1 when its two groups run two query heads of one kv head over the
+                       // same 256 rows (an item is a unit and a head pair), 0 when they run 512 rows of one head
     float scale_log2;  // qk_scale * log2(e)
     // paged K/V only: logical block i of sequence b is physical block tables[b * table_stride + i]
     const int *tables;
