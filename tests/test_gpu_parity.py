@@ -140,6 +140,7 @@ CASES = [
     ([130, 7], [130, 7], 2, 2, torch.bfloat16, 0.07, 0),     # no mask
     ([100, 50], [260, 40], 2, 1, torch.float16, 0.07, 0),    # no mask, Lq != Lk
     ([5], [0], 1, 1, torch.bfloat16, 0.07, 1),               # no keys at all
+    ([300, 50], [100, 50], 4, 2, torch.bfloat16, 0.07, 1),   # Lq > Lk with two query heads per kv head
 ]
 
 # Cases held to the half-ulp form of the bound instead of the literal one, with the reason.
